@@ -1,0 +1,18 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
+
+
+def pytest_collection_modifyitems(config, items):
+    # gpu tests cannot run without a GPU; fail loudly instead of skipping when
+    # a GPU is present but the library is missing (handled in the tests).
+    pass
