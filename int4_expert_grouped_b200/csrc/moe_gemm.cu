@@ -1,0 +1,546 @@
+// Grouped GEMM over int4 expert weights, dequantised on chip (inblix article
+// "Perplexity's Lily engine beats MLX by 35% on M5 Max, no PyTorch needed",
+// paragraph 3: 4-bit dequantisation fused into the grouped GEMM so expanded
+// bf16 weights never reach memory).
+//
+//   prepack_kernel        logical nibbles/scales -> per (expert, tile, K chunk)
+//                         contiguous blocks in the order the GEMM reads them
+//   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
+//       gate/up: D0 = Wg x^T, D1 = Wu x^T over gathered token rows, epilogue
+//                h = silu(D0) * D1 -> bf16 h rows in expert order
+//       down:    D0, D1 = two 128-row tiles of Wd times h^T, epilogue
+//                y_acc[t] += topk_w * D (fp32 reduction in L2)
+//   finalize_kernel       y = bf16(y_acc)
+//
+// One work unit = one block-map tile (<= 128 expert-ordered rows of one
+// expert) x one pair of 128-row weight tiles.  The weights are the MMA A
+// operand (M = 128 per tile), the tokens the B operand (N = rows rounded up to
+// 16), so a partly filled tile wastes at most 15 columns.
+//
+// Warp roles (512 threads, one CTA per SM):
+//   warp 0       bulk-copies packed weight blocks into the W ring (TMA engine)
+//   warp 1       allocates TMEM, issues tcgen05.mma (one thread)
+//   warps 2-3    gather token rows into the B ring (cp.async, 128B swizzle)
+//   warps 4-11   expand int4 -> bf16 from the W ring into the A ring
+//   warps 12-15  epilogue: TMEM -> registers -> h rows / y_acc reductions
+// TMEM holds two accumulator buffers of 2 x 128 columns, so the epilogue of
+// one unit overlaps the main loop of the next.
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpWProducer = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpLoader0 = 2;
+constexpr int kNumLoaderWarps = 2;
+constexpr int kWarpTransform0 = 4;
+constexpr int kNumTransformWarps = 8;
+constexpr int kWarpEpi0 = 12;
+constexpr int kNumEpiWarps = 4;
+constexpr int kGemmThreads = 16 * 32;
+constexpr int kLoaderThreads = kNumLoaderWarps * 32;
+constexpr int kTransformThreads = kNumTransformWarps * 32;
+
+constexpr int kNW = 4;  // packed weight ring
+constexpr int kNA = 2;  // expanded bf16 A ring
+constexpr int kNB = 4;  // token B ring
+constexpr int kATileBytes = 128 * 128;
+constexpr int kAStageBytes = 2 * kATileBytes;
+constexpr int kBStageBytes = kBlockT * 128;
+constexpr int kWStageBytes = packed_block_bytes(32);
+constexpr int kNibbleBytes = 256 * 32;
+constexpr int kEpiRowBytes = 80;  // 32 bf16 + 16 bytes of padding (no bank conflicts)
+constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
+
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kNA * kAStageBytes;
+constexpr int kOffW = kOffB + kNB * kBStageBytes;
+constexpr int kOffEpi = kOffW + kNW * kWStageBytes;
+constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiWarpBytes;
+constexpr int kNumBars = 2 * kNW + 2 * kNA + 2 * kNB + 2 + 2 + 1;
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+constexpr int kSmemUsed = kOffMisc + 16;
+constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
+static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0, "UMMA tiles need 1024-byte alignment");
+static_assert(kOffW % 16 == 0 && kWStageBytes % 16 == 0, "bulk copies need 16-byte alignment");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+constexpr uint32_t kTmemCols = 512;
+
+union BF2 {
+    uint32_t u;
+    __nv_bfloat162 h;
+};
+
+// Expand one 32-bit word of 8 nibbles into 8 bf16 weights (16 bytes).  The
+// word holds K positions 2i (bits 4i..4i+3) and 2i+1 (bits 16+4i..) for
+// i = 0..3, so masking with 0x000F000F and or-ing the bf16 pattern of 128
+// yields the pair (128 + q_2i, 128 + q_2i+1) exactly; subtracting 128 is exact
+// and the fused multiply-add q*s + b rounds once.
+__device__ __forceinline__ uint4 expand8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
+    BF2 k128;
+    k128.u = 0x43004300u;
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        BF2 v, o;
+        v.u = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+        const __nv_bfloat162 q = __hsub2(v.h, k128.h);
+        o.h = __hfma2(q, s2, b2);
+        r[i] = o.u;
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Wait used only while shutting down after an abort: ignores the abort flag.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > 200000000ull) return false;
+    }
+    return true;
+}
+
+template <bool kDown>
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // barrier addresses
+    const uint32_t bar0 = sbase + kOffBar;
+    auto wfull = [&](int s) { return bar0 + 8u * s; };
+    auto wempty = [&](int s) { return bar0 + 8u * (kNW + s); };
+    auto afull = [&](int s) { return bar0 + 8u * (2 * kNW + s); };
+    auto aempty = [&](int s) { return bar0 + 8u * (2 * kNW + kNA + s); };
+    auto bfull = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + s); };
+    auto bempty = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + kNB + s); };
+    auto accfull = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + 2 * kNB + s); };
+    auto accempty = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + 2 * kNB + 2 + s); };
+    const uint32_t drain_bar = bar0 + 8u * (kNumBars - 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kNW; ++s) {
+            mbar_init(wfull(s), 1);
+            mbar_init(wempty(s), kNumTransformWarps);
+        }
+        for (int s = 0; s < kNA; ++s) {
+            mbar_init(afull(s), kNumTransformWarps);
+            mbar_init(aempty(s), 1);
+        }
+        for (int s = 0; s < kNB; ++s) {
+            mbar_init(bfull(s), kLoaderThreads);
+            mbar_init(bempty(s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(accfull(s), 1);
+            mbar_init(accempty(s), kNumEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int NT = a.NT;
+    const int KC = a.K / kKChunk;
+    const int num_units = min(*a.num_blocks * NT, a.max_units);
+
+    auto fail = [&](int where) {
+        *abort_flag = 1;
+        report_error(a.status, MOE_ERR_DEVICE_TIMEOUT, (kDown ? 200 : 100) + where);
+    };
+
+    if (warp == kWarpWProducer) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+                const int b = u / NT;
+                const int j = u - b * NT;
+                const int e = a.block_map[3 * b];
+                const uint8_t* src =
+                    a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
+                for (int c = 0; c < KC; ++c, ++it) {
+                    const int s = it % kNW;
+                    if (!mbar_wait(wempty(s), ((it / kNW) & 1) ^ 1, abort_flag)) {
+                        fail(1);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(wfull(s), a.block_bytes);
+                    bulk_copy_g2s(sbase + kOffW + s * kWStageBytes, src + c * a.block_bytes,
+                                  a.block_bytes, wfull(s));
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA exits
+                const uint32_t first = it > kNW ? it - kNW : 0;
+                for (uint32_t i = first; i < it; ++i)
+                    mbar_wait_drain(wfull(i % kNW), (i / kNW) & 1);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            uint32_t it = 0, ucount = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x, ++ucount) {
+                const int b = u / NT;
+                const int rows = a.block_map[3 * b + 2];
+                const int N = (rows + 15) & ~15;
+                const uint32_t idesc = make_idesc_bf16(128, N);
+                const int buf = ucount & 1;
+                if (!mbar_wait(accempty(buf), ((ucount >> 1) & 1) ^ 1, abort_flag)) {
+                    fail(2);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem + buf * 256;
+                const uint32_t d1 = d0 + 128;
+                for (int c = 0; c < KC; ++c, ++it) {
+                    const int sa = it % kNA;
+                    const int sb = it % kNB;
+                    if (!mbar_wait(afull(sa), (it / kNA) & 1, abort_flag) ||
+                        !mbar_wait(bfull(sb), (it / kNB) & 1, abort_flag)) {
+                        fail(3);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    fence_proxy_async_smem();
+                    const uint32_t abase = sbase + kOffA + sa * kAStageBytes;
+                    const uint64_t da0 = make_sw128_desc(abase);
+                    const uint64_t da1 = make_sw128_desc(abase + kATileBytes);
+                    const uint64_t db = make_sw128_desc(sbase + kOffB + sb * kBStageBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kKChunk / 16; ++kk) {
+                        const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+                        mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, acc);
+                        mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, idesc, acc);
+                    }
+                    mma_commit(aempty(sa));
+                    mma_commit(bempty(sb));
+                }
+                if (ok) mma_commit(accfull(buf));
+            }
+            if (!ok) {
+                mma_commit(drain_bar);
+                mbar_wait_drain(drain_bar, 0);
+            }
+        }
+    } else if (warp >= kWarpLoader0 && warp < kWarpLoader0 + kNumLoaderWarps) {
+        const int ltid = threadIdx.x - kWarpLoader0 * 32;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            const int b = u / NT;
+            const int row0 = a.block_map[3 * b + 1];
+            const int rows = a.block_map[3 * b + 2];
+            const int N = (rows + 15) & ~15;
+            const uint16_t* src[2];
+            uint32_t nbytes[2];
+            bool active[2];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = ltid + kLoaderThreads * rr;
+                active[rr] = r < N;
+                const bool valid = r < rows;
+                long srow = 0;
+                if (valid) srow = kDown ? row0 + r : a.sorted_assign[row0 + r] / a.topk;
+                src[rr] = a.act + srow * a.K;
+                nbytes[rr] = valid ? 16u : 0u;
+            }
+            for (int c = 0; c < KC; ++c, ++it) {
+                const int s = it % kNB;
+                if (!mbar_wait(bempty(s), ((it / kNB) & 1) ^ 1, abort_flag)) {
+                    fail(4);
+                    ok = false;
+                    break;
+                }
+                const uint32_t dst = sbase + kOffB + s * kBStageBytes;
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    if (active[rr]) {
+                        const int r = ltid + kLoaderThreads * rr;
+                        const uint16_t* p = src[rr] + c * kKChunk;
+#pragma unroll
+                        for (int qq = 0; qq < 8; ++qq)
+                            cp_async_16(dst + r * 128 + ((qq ^ (r & 7)) << 4), p + qq * 8,
+                                        nbytes[rr]);
+                    }
+                }
+                cp_async_arrive_noinc(bfull(s));
+            }
+        }
+        cp_async_wait_all();
+    } else if (warp >= kWarpTransform0 && warp < kWarpTransform0 + kNumTransformWarps) {
+        const int ttid = threadIdx.x - kWarpTransform0 * 32;
+        const int gpc = kKChunk / a.group;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            for (int c = 0; c < KC; ++c, ++it) {
+                const int sw = it % kNW;
+                const int sa = it % kNA;
+                if (!mbar_wait(wfull(sw), (it / kNW) & 1, abort_flag) ||
+                    !mbar_wait(aempty(sa), ((it / kNA) & 1) ^ 1, abort_flag)) {
+                    fail(5);
+                    ok = false;
+                    break;
+                }
+                const uint8_t* wst = smem + kOffW + sw * kWStageBytes;
+                const uint32_t ast = sbase + kOffA + sa * kAStageBytes;
+#pragma unroll
+                for (int rep = 0; rep < 2; ++rep) {
+                    const int task = ttid + kTransformThreads * rep;
+                    const int row = task >> 1;  // 0..255: A0 rows then A1 rows
+                    const int half = task & 1;  // K 0..31 or 32..63 of the chunk
+                    const uint4 pk = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
+                    const int g = (half * 32) / a.group;
+                    const uint32_t sb = *reinterpret_cast<const uint32_t*>(
+                        wst + kNibbleBytes + (row * gpc + g) * 4);
+                    BF2 s2, b2;
+                    s2.u = __byte_perm(sb, 0, 0x1010);
+                    b2.u = __byte_perm(sb, 0, 0x3232);
+                    const uint32_t arow = ast + (row >> 7) * kATileBytes + (row & 127) * 128;
+                    const int rsw = row & 7;
+                    st_shared_v4(arow + (((half * 4 + 0) ^ rsw) << 4), expand8(pk.x, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 1) ^ rsw) << 4), expand8(pk.y, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 2) ^ rsw) << 4), expand8(pk.z, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 3) ^ rsw) << 4), expand8(pk.w, s2.h, b2.h));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(afull(sa));
+                    mbar_arrive(wempty(sw));
+                }
+            }
+        }
+    } else {
+        // epilogue warps: warp % 4 selects the TMEM lane quadrant
+        const int q = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        uint8_t* stg = smem + kOffEpi + (warp - kWarpEpi0) * kEpiWarpBytes;
+        uint32_t ucount = 0;
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++ucount) {
+            const int b = u / NT;
+            const int j = u - b * NT;
+            const int row0 = a.block_map[3 * b + 1];
+            const int rows = a.block_map[3 * b + 2];
+            const int ncb = (rows + 31) >> 5;
+            const int buf = ucount & 1;
+            // per-column routing data for the down epilogue: lane holds columns lane + 32*i
+            int tk[4];
+            float wt[4];
+            if (kDown) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = lane + 32 * i;
+                    tk[i] = 0;
+                    wt[i] = 0.0f;
+                    if (c < rows) {
+                        const int asg = a.sorted_assign[row0 + c];
+                        tk[i] = asg / a.topk;
+                        wt[i] = a.topk_w[asg];
+                    }
+                }
+            }
+            if (!mbar_wait(accfull(buf), (ucount >> 1) & 1, abort_flag)) {
+                fail(6);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tb = tmem + lane_base + buf * 256;
+            if (!kDown) {
+#pragma unroll 1
+                for (int cb = 0; cb < ncb; ++cb) {
+                    uint32_t g[32], uu[32];
+                    tmem_ld32(tb + cb * 32, g);
+                    tmem_ld32(tb + 128 + cb * 32, uu);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const float gv = __uint_as_float(g[jj]);
+                        const float uv = __uint_as_float(uu[jj]);
+                        const float hv = __fdividef(gv * uv, 1.0f + __expf(-gv));
+                        *reinterpret_cast<__nv_bfloat16*>(stg + jj * kEpiRowBytes + lane * 2) =
+                            __float2bfloat16_rn(hv);
+                    }
+                    __syncwarp();
+                    const int c = cb * 32 + lane;
+                    if (c < rows) {
+                        const uint4* s4 = reinterpret_cast<const uint4*>(stg + lane * kEpiRowBytes);
+                        uint4* d4 = reinterpret_cast<uint4*>(
+                            a.h_out + static_cast<size_t>(row0 + c) * a.out_ld + j * 128 + q * 32);
+                        d4[0] = s4[0];
+                        d4[1] = s4[1];
+                        d4[2] = s4[2];
+                        d4[3] = s4[3];
+                    }
+                    __syncwarp();
+                }
+            } else {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int m = j * 256 + half * 128 + q * 32 + lane;
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        if (cb < ncb) {
+                            uint32_t o[32];
+                            tmem_ld32(tb + half * 128 + cb * 32, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) {
+                                const int t = __shfl_sync(0xffffffffu, tk[cb], jj);
+                                const float w = __shfl_sync(0xffffffffu, wt[cb], jj);
+                                if (cb * 32 + jj < rows)
+                                    atomicAdd(a.y_acc + static_cast<size_t>(t) * a.out_ld + m,
+                                              w * __uint_as_float(o[jj]));
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accempty(buf));
+        }
+    }
+
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// One thread per (expert, tile, K chunk, packed row): writes 8 words of
+// nibbles and the row's (scale, bias) pairs of that chunk.
+__global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t* __restrict__ out) {
+    const int KC = s.K / kKChunk;
+    const int gpc = kKChunk / group;
+    const int bb = packed_block_bytes(group);
+    const long total = static_cast<long>(E) * s.NT * KC * 256;
+    for (long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<long>(gridDim.x) * blockDim.x) {
+        const int rr = static_cast<int>(idx & 255);
+        long blk = idx >> 8;
+        const int c = static_cast<int>(blk % KC);
+        blk /= KC;
+        const int j = static_cast<int>(blk % s.NT);
+        const int e = static_cast<int>(blk / s.NT);
+        const bool second = rr >= 128;
+        const int n = j * s.row_step + (second ? s.a1_off : 0) + (rr & 127);
+        const uint8_t* qsrc = second ? s.q1 : s.q0;
+        const uint16_t* ssrc = second ? s.s1 : s.s0;
+        const uint16_t* bsrc = second ? s.b1 : s.b0;
+        const size_t row = static_cast<size_t>(e) * s.N + n;
+        const uint8_t* qrow = qsrc + row * (s.K / 2) + c * 32;
+        uint8_t* dst = out + ((static_cast<size_t>(e) * s.NT + j) * KC + c) * bb;
+        uint32_t words[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t byte = qrow[4 * w + i];  // K = 8w+2i (low), 8w+2i+1 (high)
+                word |= (byte & 0xFu) << (4 * i);
+                word |= (byte >> 4) << (16 + 4 * i);
+            }
+            words[w] = word;
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + rr * 32);
+        d4[0] = make_uint4(words[0], words[1], words[2], words[3]);
+        d4[1] = make_uint4(words[4], words[5], words[6], words[7]);
+        const size_t grow = row * (s.K / group) + static_cast<size_t>(c) * gpc;
+        for (int g = 0; g < gpc; ++g) {
+            const uint32_t sv = ssrc[grow + g];
+            const uint32_t bv = bsrc[grow + g];
+            *reinterpret_cast<uint32_t*>(dst + kNibbleBytes + (rr * gpc + g) * 4) = sv | (bv << 16);
+        }
+    }
+}
+
+__global__ void finalize_kernel(const float* __restrict__ y_acc, uint16_t* __restrict__ y, long n) {
+    for (long i = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < n;
+         i += static_cast<long>(gridDim.x) * blockDim.x * 8) {
+        const float4 v0 = *reinterpret_cast<const float4*>(y_acc + i);
+        const float4 v1 = *reinterpret_cast<const float4*>(y_acc + i + 4);
+        BF2 p0, p1, p2, p3;
+        p0.h = __floats2bfloat162_rn(v0.x, v0.y);
+        p1.h = __floats2bfloat162_rn(v0.z, v0.w);
+        p2.h = __floats2bfloat162_rn(v1.x, v1.y);
+        p3.h = __floats2bfloat162_rn(v1.z, v1.w);
+        *reinterpret_cast<uint4*>(y + i) = make_uint4(p0.u, p1.u, p2.u, p3.u);
+    }
+}
+
+}  // namespace
+
+cudaError_t prepare_gemm_kernels() {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(grouped_gemm_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* out,
+                           cudaStream_t st) {
+    const long total = static_cast<long>(E) * src.NT * (src.K / kKChunk) * 256;
+    const int threads = 256;
+    const long blocks = (total + threads - 1) / threads;
+    prepack_kernel<<<static_cast<int>(blocks < 65535 * 16 ? blocks : 65535 * 16), threads, 0, st>>>(
+        src, E, group, out);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaStream_t st) {
+    if (a.max_units <= 0) return cudaSuccess;
+    const int grid = a.max_units < num_sms ? a.max_units : num_sms;
+    if (down)
+        grouped_gemm_kernel<true><<<grid, kGemmThreads, kSmemBytes, st>>>(a);
+    else
+        grouped_gemm_kernel<false><<<grid, kGemmThreads, kSmemBytes, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st) {
+    return launch_gemm(a, num_sms, false, st);
+}
+
+cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st) {
+    return launch_gemm(a, num_sms, true, st);
+}
+
+cudaError_t launch_finalize(const float* y_acc, uint16_t* y, long n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int threads = 256;
+    long blocks = (n / 8 + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    finalize_kernel<<<static_cast<int>(blocks), threads, 0, st>>>(y_acc, y, n);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

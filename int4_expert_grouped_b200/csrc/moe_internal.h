@@ -1,0 +1,81 @@
+// Internal constants and kernel launchers shared by the host API and the
+// kernel files.  Not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;  // experts per layer the routing kernels hold
+constexpr int kMaxTopk = 32;      // one warp lane per selected expert
+constexpr int kRouteGroupT = 256; // tokens per scatter group (one histogram row)
+constexpr int kBlockT = 128;      // block map tile height = largest MMA N
+constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
+
+// Packed weight block: two 128-row A tiles (A0 rows 0..127, A1 rows
+// 128..255) of one 64-wide K chunk: 256 rows x 32 bytes of nibbles, then per
+// row and group one (scale, bias) bf16 pair.
+__host__ __device__ constexpr int packed_block_bytes(int group) {
+    return 256 * 32 + 256 * (kKChunk / group) * 4;
+}
+
+// ---- routing (moe_route.cu) ----
+cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float* b, float* logits,
+                                 int T, int d, int E, int32_t* hist, int hist_n, int32_t* status,
+                                 cudaStream_t st);
+cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                               float* topk_w, int32_t* hist, float* y_acc, int d,
+                               cudaStream_t st);
+cudaError_t launch_route_scan(const int32_t* hist, int ng, int E, int BT, int32_t* counts,
+                              int32_t* offsets, int32_t* gbase, int32_t* block_offsets,
+                              int32_t* block_map, int32_t* num_blocks, int max_blocks,
+                              int32_t* status, cudaStream_t st);
+cudaError_t launch_route_scatter(const int32_t* topk_idx, const int32_t* gbase, int T, int k,
+                                 int E, int32_t* sorted_assign, int32_t* pos, int32_t* status,
+                                 cudaStream_t st);
+
+// ---- weights and GEMM (moe_gemm.cu) ----
+struct PrepackSource {
+    const uint8_t* q0;   // A0 rows come from this projection
+    const uint16_t* s0;
+    const uint16_t* b0;
+    const uint8_t* q1;   // A1 rows come from this projection
+    const uint16_t* s1;
+    const uint16_t* b1;
+    int N;               // rows per expert of the source projections
+    int K;               // reduction length
+    int row_step;        // source row of tile j, row r: j*row_step + r (A0), + a1_off (A1)
+    int a1_off;
+    int NT;              // tiles per expert
+};
+cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* out,
+                           cudaStream_t st);
+
+struct GemmArgs {
+    const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
+    const uint16_t* act;           // B rows: x [T, d] (gate/up) or h [T*k, f] (down)
+    const int32_t* sorted_assign;  // [T*k]
+    const int32_t* block_map;      // [num_blocks, 3]
+    const int32_t* num_blocks;     // [1], device
+    const float* topk_w;           // [T*k] by assignment (down)
+    uint16_t* h_out;               // [T*k, f] (gate/up)
+    float* y_acc;                  // [T, d] fp32 (down)
+    int32_t* status;
+    int K;                         // reduction length
+    int NT;                        // output tile pairs per expert
+    int out_ld;                    // f (gate/up) or d (down)
+    int topk;
+    int group;
+    int block_bytes;
+    int max_units;                 // upper bound of num_blocks * NT
+};
+cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_finalize(const float* y_acc, uint16_t* y, long n, cudaStream_t st);
+cudaError_t prepare_gemm_kernels();
+
+}  // namespace moe

@@ -1,0 +1,231 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Integer outputs (top-k indices, counts, offsets, scatter order, inverse
+positions, block map) must match bit for bit; routing weights within 1e-6
+relative; the layer output within |y - ref| <= 2e-2 * (1 + |ref|) with the
+relative RMS error also reported and bounded.  Small workloads are checked in
+full; the 8K- and 32K-token prefill workloads have their routing checked in
+full and their outputs on sampled tokens (the oracle computes those one
+token at a time).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+Y_ATOL_REL = 2e-2     # |y - ref| <= 2e-2 * (1 + |ref|)
+Y_REL_RMS = 1.5e-2    # ||y - ref|| / ||ref||
+W_REL = 1e-6          # routing weights
+
+
+@pytest.fixture(scope="module")
+def moe():
+    assert torch.cuda.is_available(), "the gpu tests need a GPU"
+    from int4_expert_grouped_b200 import build
+    build.build()
+    import int4_expert_grouped_b200 as m
+    from int4_expert_grouped_b200.layer import MoeLayer, bf16_tensor
+    m.MoeLayer, m.bf16_tensor = MoeLayer, bf16_tensor
+    return m
+
+
+def oracle_route(inp, T=None, block_t=128):
+    x = inp.x if T is None else inp.x[:T]
+    logits = oracle.router_logits(x, inp.w_r, inp.b_r)
+    idx = oracle.topk(logits, inp.shape.k)
+    w = oracle.topk_weights(logits, idx)
+    counts, offsets = oracle.counts_offsets(idx, inp.shape.E)
+    sa, pos = oracle.scatter(idx, offsets)
+    bo, bm, nb = oracle.block_map(counts, offsets, block_t)
+    return dict(topk_idx=idx, topk_w=w, counts=counts, offsets=offsets, sorted_assign=sa,
+                pos=pos, block_offsets=bo, block_map=bm, num_blocks=nb)
+
+
+def check_route(got, ref, T, k):
+    g = {n: t.cpu().numpy() for n, t in got.items()}
+    assert np.array_equal(g["topk_idx"][:T], ref["topk_idx"]), "topk_idx"
+    rel = np.abs(g["topk_w"][:T].astype(np.float64) - ref["topk_w"]) / np.abs(ref["topk_w"])
+    assert rel.max() <= W_REL, ("topk_w", rel.max())
+    assert np.array_equal(g["counts"], ref["counts"]), "counts"
+    assert np.array_equal(g["offsets"], ref["offsets"]), "offsets"
+    assert np.array_equal(g["sorted_assign"][:T * k], ref["sorted_assign"]), "sorted_assign"
+    assert np.array_equal(g["pos"][:T * k], ref["pos"]), "pos"
+    assert np.array_equal(g["block_offsets"], ref["block_offsets"]), "block_offsets"
+    nb = int(g["num_blocks"][0])
+    assert nb == ref["num_blocks"], "num_blocks"
+    assert np.array_equal(g["block_map"][:nb], ref["block_map"]), "block_map"
+
+
+def check_y(y_gpu: torch.Tensor, ref: np.ndarray, what=""):
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(y)), what
+    err = np.abs(y - ref)
+    bound = Y_ATOL_REL * (1.0 + np.abs(ref))
+    worst = float((err / bound).max())
+    rel_rms = float(np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-30))
+    print("%s: max err/bound %.4f, rel-RMS %.3e, max |err| %.3e" % (what, worst, rel_rms, err.max()))
+    assert worst <= 1.0, (what, worst)
+    assert rel_rms <= Y_REL_RMS, (what, rel_rms)
+    return rel_rms
+
+
+_cache = {}
+
+
+def workload(name):
+    if name not in _cache:
+        _cache[name] = mi.workload(name)
+    return _cache[name]
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_t1", "decode_t4", "prefill_t512"])
+def test_layer_full(moe, name):
+    inp = workload(name)
+    s = inp.shape
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bufs = layer.route_buffers(s.T)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    assert layer.read_status() == (0, 0)
+    ref = oracle.forward(inp)
+    rref = oracle_route(inp)
+    check_route(bufs, rref, s.T, s.k)
+    check_y(y[:s.T], ref["y"], name)
+
+
+@pytest.mark.parametrize("name", ["prefill_t8192", "prefill_t32768_zipf"])
+def test_layer_large_sampled(moe, name):
+    inp = workload(name)
+    s = inp.shape
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bufs = layer.route_buffers(s.T)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    assert layer.read_status() == (0, 0)
+    rref = oracle_route(inp)
+    check_route(bufs, rref, s.T, s.k)
+    # sampled tokens: both ends, a spread, and tokens of the most loaded expert
+    rng = np.random.default_rng(1234)
+    hot = int(np.argmax(rref["counts"]))
+    hot_tokens = rref["sorted_assign"][rref["offsets"][hot]:rref["offsets"][hot + 1]] // s.k
+    toks = np.unique(np.concatenate([[0, 1, s.T - 1], rng.choice(s.T, 40, replace=False),
+                                     rng.choice(hot_tokens, 8, replace=False)]))
+    yref, idx, w = oracle.token_outputs(inp, toks)
+    assert np.array_equal(idx, rref["topk_idx"][toks])
+    check_y(y[torch.from_numpy(toks).cuda()], yref, name)
+
+
+def test_route_entry_point_matches_forward(moe):
+    inp = workload("prefill_t512")
+    s = inp.shape
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    a = layer.route(x)
+    b = layer.route_buffers(s.T)
+    layer.forward(x, route_out=b)
+    torch.cuda.synchronize()
+    for n in a:
+        if n == "block_map":
+            nb = int(a["num_blocks"][0])
+            assert torch.equal(a[n][:nb], b[n][:nb])
+        elif n == "num_blocks":
+            assert int(a[n][0]) == int(b[n][0])
+        else:
+            assert torch.equal(a[n], b[n]), n
+
+
+def test_repeat_calls_and_host_path(moe):
+    inp = workload("tiny")
+    s = inp.shape
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    y1 = layer.forward(x).clone()
+    y2 = layer.forward(x).clone()
+    xh = torch.from_numpy(inp.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((s.T, s.d), dtype=torch.bfloat16).pin_memory()
+    layer.forward_host(xh, yh)
+    ref = oracle.forward(inp)["y"]
+    check_y(y1, ref, "first call")
+    check_y(y2, ref, "second call")
+    check_y(yh, ref, "host buffers")
+    # fp32 combine order may differ between calls; both must be within a few bf16 ulps
+    assert (y1.float() - y2.float()).abs().max().item() <= 2e-3
+
+
+def test_empty_batch(moe):
+    inp = workload("tiny")
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = torch.empty((0, inp.shape.d), dtype=torch.bfloat16, device="cuda")
+    bufs = layer.route_buffers(0)
+    layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    assert int(bufs["num_blocks"][0]) == 0
+    assert torch.count_nonzero(bufs["counts"]).item() == 0
+    assert torch.count_nonzero(bufs["offsets"]).item() == 0
+
+
+@pytest.mark.parametrize("T", [1, 3, 31, 77, 129, 255, 257])
+def test_ragged_token_counts(moe, T):
+    shape = mi.Shape(T=300, d=256, E=8, k=2, f=128, group=32)
+    inp = mi.make_inputs(shape, 40 + T)
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x[:T], "cuda")
+    bufs = layer.route_buffers(T)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    sub = mi.Inputs(mi.Shape(T, 256, 8, 2, 128, 32), inp.seed, inp.x[:T], inp.w_r, inp.b_r,
+                    inp.gate, inp.up, inp.down)
+    ref = oracle.forward(sub)
+    check_route(bufs, oracle_route(sub), T, 2)
+    check_y(y[:T], ref["y"], "T=%d" % T)
+
+
+def test_all_tokens_same_experts(moe):
+    # a zero router with a decreasing bias sends every token to experts 0..k-1:
+    # each of those experts gets T rows (several full blocks and a ragged one)
+    shape = mi.Shape(T=300, d=256, E=8, k=2, f=128, group=32)
+    inp = mi.make_inputs(shape, 7)
+    inp.w_r = np.zeros_like(inp.w_r)
+    inp.b_r = -np.arange(8, dtype=np.float32)
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bufs = layer.route_buffers(300)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    rref = oracle_route(inp)
+    assert list(rref["counts"]) == [300, 300, 0, 0, 0, 0, 0, 0]
+    check_route(bufs, rref, 300, 2)
+    check_y(y[:300], oracle.forward(inp)["y"], "concentrated")
+
+
+def test_every_expert_selected(moe):
+    shape = mi.Shape(T=64, d=256, E=8, k=8, f=128, group=64)
+    inp = mi.make_inputs(shape, 17)
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bufs = layer.route_buffers(64)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    check_route(bufs, oracle_route(inp), 64, 8)
+    check_y(y[:64], oracle.forward(inp)["y"], "k=E")
+
+
+def test_tied_logits(moe):
+    # a zero router without bias ties every logit: ids 0..k-1 in id order,
+    # equal weights
+    shape = mi.Shape(T=40, d=256, E=16, k=4, f=128, group=32)
+    inp = mi.make_inputs(shape, 5)
+    inp.w_r = np.zeros_like(inp.w_r)
+    layer = moe.MoeLayer.from_inputs(inp)
+    bufs = layer.route(moe.bf16_tensor(inp.x, "cuda"))
+    torch.cuda.synchronize()
+    idx = bufs["topk_idx"][:40].cpu().numpy()
+    assert (idx == np.arange(4)).all()
+    assert torch.all(bufs["topk_w"][:40] == 0.25)
+    check_route(bufs, oracle_route(inp), 40, 4)
