@@ -223,6 +223,30 @@ MOE_API moe_status_t moe_forward_host(const moe_plan_t *plan, int32_t T,
                               void *stream);
 
 /*
+ * moe_route without a workspace, for callers that cannot allocate device
+ * memory (code running under a stream capture that forbids allocation, a
+ * runtime that owns every byte of device memory, a plugin host that hands a
+ * kernel only its inputs and outputs).  The pages describe no such entry
+ * point; it has no counterpart there.
+ *   Arguments and outputs: as moe_route, without ws / ws_bytes.
+ *   Scratch: a fixed 4 MiB array inside the library, per GPU, held until the
+ *     process exits.  A call needs 256 + 4*T*E + 8*ceil(T/256)*E bytes of it
+ *     (each part rounded up to 256); larger calls return
+ *     MOE_ERR_WORKSPACE_TOO_SMALL before launching anything.
+ *   The first call on a device looks up the array's device address (with
+ *     that device current); make it before any stream capture begins.
+ *   Every call shares the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race and must be serialised by the caller.
+ *   Device-side errors are recorded in the array and cannot be read back.
+ *   It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     call.
+ */
+MOE_API moe_status_t moe_route_noalloc(const moe_plan_t *plan, int32_t T,
+                                       const uint16_t *x, const float *W_r,
+                                       const float *b_r,
+                                       const moe_route_out_t *out, void *stream);
+
+/*
  * Read the device status word of a workspace (synchronises `stream`
  * first).  *code is a moe_status_t (MOE_OK if no device error was
  * recorded); *detail says where.  clear != 0 resets the word afterwards.

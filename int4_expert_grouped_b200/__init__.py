@@ -89,16 +89,18 @@ _lib.moe_forward.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, _P, ctypes.POIN
 _lib.moe_forward_timed.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                    ctypes.POINTER(RouteOut), _P, ctypes.c_size_t, _P,
                                    ctypes.POINTER(StageEvents)]
+_lib.moe_route_noalloc.argtypes = [_P, ctypes.c_int32, _P, _P, _P, ctypes.POINTER(RouteOut), _P]
 _lib.moe_forward_host.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_read_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                  ctypes.c_int32, _P]
 for _fn in ("moe_plan_create", "moe_plan_info", "moe_prepack_weights", "moe_route",
-            "moe_forward", "moe_forward_timed", "moe_forward_host", "moe_read_status"):
+            "moe_forward", "moe_forward_timed", "moe_forward_host", "moe_read_status",
+            "moe_route_noalloc"):
     getattr(_lib, _fn).restype = ctypes.c_int
 
 EXPORTED = ("moe_abi_version", "moe_status_str", "moe_plan_create", "moe_plan_info",
             "moe_plan_destroy", "moe_prepack_weights", "moe_route", "moe_forward",
-            "moe_forward_timed", "moe_forward_host", "moe_read_status")
+            "moe_forward_timed", "moe_forward_host", "moe_read_status", "moe_route_noalloc")
 
 
 def abi_version() -> int:
@@ -173,6 +175,12 @@ class Plan:
         ro = self.route_out(out)
         _check(_lib.moe_route(self._h, T, ptr(x), ptr(w_r), ptr(b_r), ctypes.byref(ro), ptr(ws),
                               ws.numel() * ws.element_size(), _stream_ptr(stream)), "moe_route")
+
+    def route_noalloc(self, T, x, w_r, b_r, out: dict, stream=None):
+        """moe_route_noalloc: routing with the library's own fixed scratch."""
+        ro = self.route_out(out)
+        _check(_lib.moe_route_noalloc(self._h, T, ptr(x), ptr(w_r), ptr(b_r), ctypes.byref(ro),
+                                      _stream_ptr(stream)), "moe_route_noalloc")
 
     def forward(self, T, x, w_r, b_r, packed_w, y, ws, route_out: dict | None = None, stream=None,
                 events=None):

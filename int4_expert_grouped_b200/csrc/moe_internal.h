@@ -8,6 +8,22 @@
 
 #include "moe_common.cuh"
 
+// Plan of one layer shape (opaque to callers of the C ABI).
+struct moe_plan {
+    moe_shape_t s;
+    int block_t;
+    int max_blocks;
+    int ng_max;
+    int group_bytes;  // packed block bytes
+    size_t gu_packed;  // bytes of the gate/up packed blocks
+    size_t dn_packed;
+    size_t packed_bytes;
+    // workspace offsets
+    size_t o_status, o_logits, o_hist, o_gbase, o_idx, o_w, o_counts, o_offsets, o_bo, o_nb,
+        o_sa, o_pos, o_bm, o_h, o_yacc, ws_bytes;
+    size_t o_xstage, o_ystage, host_ws_bytes;
+};
+
 namespace moe {
 
 constexpr int kMaxExperts = 256;  // experts per layer the routing kernels hold
