@@ -43,15 +43,16 @@ constexpr int kLoaderThreads = kNumLoaderWarps * 32;
 constexpr int kTransformThreads = kNumTransformWarps * 32;
 
 constexpr int kNW = 4;  // packed weight ring
-constexpr int kNA = 2;  // expanded bf16 A ring
+constexpr int kNA = 3;  // expanded bf16 A ring
 constexpr int kNB = 4;  // token B ring
 constexpr int kATileBytes = 128 * 128;
 constexpr int kAStageBytes = 2 * kATileBytes;
 constexpr int kBStageBytes = kBlockT * 128;
 constexpr int kWStageBytes = packed_block_bytes(32);
 constexpr int kNibbleBytes = 256 * 32;
-constexpr int kEpiRowBytes = 80;  // 32 bf16 + 16 bytes of padding (no bank conflicts)
-constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
+constexpr int kEpiRowBytes = 80;  // gate/up staging row: 32 bf16 + 16 bytes of padding
+constexpr int kEpiRowFloats = 36;  // down staging row: 32 fp32 + 4 of padding
+constexpr int kEpiWarpBytes = 32 * kEpiRowFloats * 4;
 
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kNA * kAStageBytes;
@@ -96,6 +97,13 @@ __device__ __forceinline__ uint4 expand8(uint32_t w, __nv_bfloat162 s2, __nv_bfl
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// y[0..3] += v (fp32, one 16-byte reduction in L2)
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a),
+                 "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
 
@@ -249,7 +257,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
             }
         }
     } else if (warp >= kWarpLoader0 && warp < kWarpLoader0 + kNumLoaderWarps) {
+        // Lane layout: 8 consecutive lanes copy the 8 16-byte pieces of one
+        // 128-byte row chunk, so a warp instruction reads 4 whole rows.
+        // Thread ltid copies piece (ltid % 8) of rows ltid/8 + 8*jr.
         const int ltid = threadIdx.x - kWarpLoader0 * 32;
+        const int piece = ltid & 7;
+        const int rbase = ltid >> 3;
+        constexpr int kRowsPerThread = kBlockT / (kLoaderThreads / 8);
+        const uint32_t swz = static_cast<uint32_t>((piece ^ rbase) << 4);  // row & 7 == rbase
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
@@ -257,18 +272,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
             const int row0 = a.block_map[3 * b + 1];
             const int rows = a.block_map[3 * b + 2];
             const int N = (rows + 15) & ~15;
-            const uint16_t* src[2];
-            uint32_t nbytes[2];
-            bool active[2];
+            const uint16_t* src[kRowsPerThread];
+            uint32_t valid_mask = 0;
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int r = ltid + kLoaderThreads * rr;
-                active[rr] = r < N;
-                const bool valid = r < rows;
+            for (int jr = 0; jr < kRowsPerThread; ++jr) {
+                const int r = rbase + 8 * jr;
                 long srow = 0;
-                if (valid) srow = kDown ? row0 + r : a.sorted_assign[row0 + r] / a.topk;
-                src[rr] = a.act + srow * a.K;
-                nbytes[rr] = valid ? 16u : 0u;
+                if (r < rows) {
+                    srow = kDown ? row0 + r : a.sorted_assign[row0 + r] / a.topk;
+                    valid_mask |= 1u << jr;
+                }
+                src[jr] = a.act + srow * a.K + piece * 8;
             }
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % kNB;
@@ -277,17 +291,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
                     ok = false;
                     break;
                 }
-                const uint32_t dst = sbase + kOffB + s * kBStageBytes;
+                const uint32_t dst = sbase + kOffB + s * kBStageBytes + swz;
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    if (active[rr]) {
-                        const int r = ltid + kLoaderThreads * rr;
-                        const uint16_t* p = src[rr] + c * kKChunk;
-#pragma unroll
-                        for (int qq = 0; qq < 8; ++qq)
-                            cp_async_16(dst + r * 128 + ((qq ^ (r & 7)) << 4), p + qq * 8,
-                                        nbytes[rr]);
-                    }
+                for (int jr = 0; jr < kRowsPerThread; ++jr) {
+                    const int r = rbase + 8 * jr;
+                    if (r < N)
+                        cp_async_16(dst + r * 128, src[jr] + c * kKChunk,
+                                    (valid_mask >> jr) & 1u ? 16u : 0u);
                 }
                 cp_async_arrive_noinc(bfull(s));
             }
@@ -401,9 +411,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
                     __syncwarp();
                 }
             } else {
+                // D[feature][token] -> staging [token][feature] (fp32), then each
+                // lane reduces 4 consecutive features of one token into y_acc
+                // with one 16-byte red, scaled by the token's routing weight.
+                float* stf = reinterpret_cast<float*>(stg);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    const int m = j * 256 + half * 128 + q * 32 + lane;
+                    const int m0 = j * 256 + half * 128 + q * 32;
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
                         if (cb < ncb) {
@@ -411,13 +425,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
                             tmem_ld32(tb + half * 128 + cb * 32, o);
                             tmem_ld_wait();
 #pragma unroll
-                            for (int jj = 0; jj < 32; ++jj) {
-                                const int t = __shfl_sync(0xffffffffu, tk[cb], jj);
-                                const float w = __shfl_sync(0xffffffffu, wt[cb], jj);
-                                if (cb * 32 + jj < rows)
-                                    atomicAdd(a.y_acc + static_cast<size_t>(t) * a.out_ld + m,
-                                              w * __uint_as_float(o[jj]));
+                            for (int jj = 0; jj < 32; ++jj)
+                                stf[jj * kEpiRowFloats + lane] = __uint_as_float(o[jj]);
+                            __syncwarp();
+#pragma unroll
+                            for (int r = 0; r < 8; ++r) {
+                                const int c = 4 * r + (lane >> 3);
+                                const int fg = lane & 7;
+                                const int t = __shfl_sync(0xffffffffu, tk[cb], c);
+                                const float w = __shfl_sync(0xffffffffu, wt[cb], c);
+                                if (cb * 32 + c < rows) {
+                                    const float4 v = *reinterpret_cast<const float4*>(
+                                        stf + c * kEpiRowFloats + 4 * fg);
+                                    red_add_v4(a.y_acc + static_cast<size_t>(t) * a.out_ld + m0 + 4 * fg,
+                                               w * v.x, w * v.y, w * v.z, w * v.w);
+                                }
                             }
+                            __syncwarp();
                         }
                     }
                 }

@@ -9,6 +9,8 @@
 //                         block map
 //   route_scatter_kernel  stable scatter into expert order (sorted_assign,
 //                         pos)
+#include <atomic>
+
 #include "moe_internal.h"
 
 namespace moe {
@@ -121,6 +123,151 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
             float l = acc[j];
             if (b != nullptr) l = __fadd_rn(l, __ldg(b + e0 + ee));
             logits[static_cast<size_t>(t) * E + e0 + ee] = l;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Router logits for larger batches (same summation order as above).
+//
+// Each CTA owns one slice of ES experts and keeps that slice of W_r in
+// shared memory for its whole life (rows padded to ES+4 floats so the 32
+// lanes, which read 32 different rows, hit distinct banks).  It sweeps token
+// tiles of 64: every warp takes 8 tokens of the tile, lane p accumulates chain
+// p of all 8 x ES (token, expert) pairs, and the tile's x rows stream through a
+// double-buffered shared-memory ring of 256-wide K chunks (cp.async).
+// Grid: (E / ES) * ctas_per_slice; CTA c serves slice c % (E / ES) and tiles
+// c / (E / ES), c / (E / ES) + ctas_per_slice, ...
+// ---------------------------------------------------------------------------
+constexpr int kRouterTile = 64;   // tokens per tile
+constexpr int kRouterKc = 256;    // K chunk of x held in shared memory
+constexpr int kRouterWarps = 8;
+
+__host__ __device__ constexpr int router_smem_bytes(int ES, int d) {
+    return d * (ES + 4) * 4 + 2 * kRouterTile * kRouterKc * 2;
+}
+
+template <int ES>
+__global__ void __launch_bounds__(kRouterWarps * 32, 1)
+router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
+                          const float* __restrict__ b, float* __restrict__ logits, int T, int d,
+                          int E, int32_t* __restrict__ hist, int hist_n,
+                          int32_t* __restrict__ status) {
+    constexpr int TT = kRouterTile / kRouterWarps;  // tokens per warp
+    constexpr int V = TT * ES;                      // values per lane
+    constexpr int WS = ES + 4;                      // padded W row (floats)
+    static_assert(V % 32 == 0, "reduce-scatter needs a multiple of 32 values");
+    extern __shared__ __align__(16) uint8_t rsm[];
+    float* Ws = reinterpret_cast<float*>(rsm);
+    uint16_t* xs = reinterpret_cast<uint16_t*>(rsm + static_cast<size_t>(d) * WS * 4);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int nslices = E / ES;
+    const int slice = blockIdx.x % nslices;
+    const int cta = blockIdx.x / nslices;
+    const int ctas = gridDim.x / nslices;
+    const int e0 = slice * ES;
+
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < hist_n; i += blockDim.x) hist[i] = 0;
+        if (threadIdx.x < 2) status[threadIdx.x] = 0;
+    }
+    // the W_r slice, row i -> Ws[i * WS .. + ES)
+    for (int idx = threadIdx.x; idx < d * (ES / 4); idx += blockDim.x) {
+        const int i = idx / (ES / 4);
+        const int q = idx % (ES / 4);
+        const float4 v = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) + q);
+        *reinterpret_cast<float4*>(Ws + i * WS + 4 * q) = v;
+    }
+    __syncthreads();
+
+    const int ntiles = (T + kRouterTile - 1) / kRouterTile;
+    const int nkc = d / kRouterKc;
+    const uint32_t xs_base = smem_u32(xs);
+    // one K chunk of the tile: 64 rows x 512 bytes = 2048 16-byte pieces, 8 per thread
+    auto load_chunk = [&](int t0, int kc, int buf) {
+#pragma unroll
+        for (int j = 0; j < (kRouterTile * kRouterKc * 2 / 16) / (kRouterWarps * 32); ++j) {
+            const int piece = threadIdx.x + j * kRouterWarps * 32;
+            const int row = piece / (kRouterKc * 2 / 16);
+            const int col = piece % (kRouterKc * 2 / 16);
+            const int t = t0 + row;
+            const uint16_t* src = x + static_cast<size_t>(t < T ? t : 0) * d + kc * kRouterKc + col * 8;
+            cp_async_16(xs_base + ((buf * kRouterTile + row) * kRouterKc + col * 8) * 2, src,
+                        t < T ? 16u : 0u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    for (int tile = cta; tile < ntiles; tile += ctas) {
+        const int t0 = tile * kRouterTile;
+        float acc[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) acc[j] = 0.0f;
+        load_chunk(t0, 0, 0);
+        for (int kc = 0; kc < nkc; ++kc) {
+            if (kc + 1 < nkc) {
+                load_chunk(t0, kc + 1, (kc + 1) & 1);
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+            __syncthreads();
+            const uint16_t* xb = xs + ((kc & 1) * kRouterTile + warp * TT) * kRouterKc;
+            const float* wb = Ws + static_cast<size_t>(kc * kRouterKc) * WS;
+#pragma unroll 2
+            for (int s = 0; s < kRouterKc / 32; ++s) {
+                const int il = s * 32 + lane;
+                float xv[TT];
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt) xv[tt] = bf16_bits_to_float(xb[tt * kRouterKc + il]);
+                float wv[ES];
+#pragma unroll
+                for (int q = 0; q < ES / 4; ++q) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wb + il * WS + 4 * q);
+                    wv[4 * q + 0] = w4.x;
+                    wv[4 * q + 1] = w4.y;
+                    wv[4 * q + 2] = w4.z;
+                    wv[4 * q + 3] = w4.w;
+                }
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int ee = 0; ee < ES; ++ee)
+                        acc[tt * ES + ee] = __fmaf_rn(xv[tt], wv[ee], acc[tt * ES + ee]);
+            }
+            __syncthreads();  // the buffer is refilled by the next chunk's copies
+        }
+        // reduce-scatter butterfly (see router_logits_kernel)
+        int cnt = V;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            const bool upper = (lane & m) != 0;
+            const int half = cnt >> 1;
+#pragma unroll
+            for (int j = 0; j < V / 2; ++j) {
+                if (j < half) {
+                    const float lo = acc[j];
+                    const float hi = acc[j + half];
+                    const float send = upper ? lo : hi;
+                    const float keep = upper ? hi : lo;
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+                    acc[j] = __fadd_rn(keep, recv);
+                }
+            }
+            cnt = half;
+        }
+#pragma unroll
+        for (int j = 0; j < V / 32; ++j) {
+            const int el = lane * (V / 32) + j;
+            const int tt = el / ES;
+            const int ee = el % ES;
+            const int t = t0 + warp * TT + tt;
+            if (t < T) {
+                float l = acc[j];
+                if (b != nullptr) l = __fadd_rn(l, __ldg(b + e0 + ee));
+                logits[static_cast<size_t>(t) * E + e0 + ee] = l;
+            }
         }
     }
 }
@@ -298,34 +445,62 @@ route_scan_kernel(const int32_t* __restrict__ hist, int ng, int E, int BT,
 // ---------------------------------------------------------------------------
 // Scatter: visit assignments a = t*k + j in ascending order and place each at
 // the next free row of its expert, so rows of one expert are in ascending a.
-// One warp per group of kRouteGroupT tokens, starting from the group's bases;
-// inside a 32-assignment chunk the lanes of one expert are ranked by lane id.
+// One CTA of kScatterWarps warps per group of kRouteGroupT tokens; warp w
+// owns a contiguous slice of the group's assignments.  Pass 1 counts each
+// warp's assignments per expert, the warps' bases follow from the group's base
+// (gbase) by a scan over warps, and pass 2 places every assignment: inside a
+// 32-assignment chunk the lanes of one expert are ranked by lane id.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(32)
+constexpr int kScatterWarps = 8;
+
+__global__ void __launch_bounds__(kScatterWarps * 32)
 route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ gbase,
                      int T, int k, int E, int32_t* __restrict__ sorted_assign,
                      int32_t* __restrict__ pos, int32_t* status) {
-    __shared__ int running[kMaxExperts];
-    const int lane = threadIdx.x;
+    __shared__ int cnt[kScatterWarps][kMaxExperts];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int g = blockIdx.x;
-    for (int e = lane; e < E; e += 32) running[e] = gbase[static_cast<size_t>(g) * E + e];
-    __syncwarp();
     const long total = static_cast<long>(T) * k;
     const long a_begin = static_cast<long>(g) * kRouteGroupT * k;
     const long a_end = min(total, a_begin + static_cast<long>(kRouteGroupT) * k);
+    const long per_warp = (static_cast<long>(kRouteGroupT) * k + kScatterWarps - 1) / kScatterWarps;
+    const long w_begin = a_begin + warp * per_warp;
+    const long w_end = min(a_end, w_begin + per_warp);
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (long a0 = a_begin; a0 < a_end; a0 += 32) {
+
+    for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
+    __syncwarp();
+    for (long a0 = w_begin; a0 < w_end; a0 += 32) {
         const long a = a0 + lane;
-        const bool valid = a < a_end;
-        int e = valid ? topk_idx[a] : E + lane;  // distinct non-experts for idle lanes
-        if (valid && (e < 0 || e >= E)) {
+        int e = a < w_end ? topk_idx[a] : E + lane;
+        if (e < 0 || (e >= E && a < w_end)) {
             report_error(status, MOE_ERR_DEVICE_BOUNDS, 2);
             e = E + lane;
         }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e < E && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per-warp bases: exclusive scan over warps, starting at the group's base
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = gbase[static_cast<size_t>(g) * E + e];
+        for (int w = 0; w < kScatterWarps; ++w) {
+            const int c = cnt[w][e];
+            cnt[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    for (long a0 = w_begin; a0 < w_end; a0 += 32) {
+        const long a = a0 + lane;
+        int e = a < w_end ? topk_idx[a] : E + lane;
+        if (e < 0 || e > E + 31) e = E + lane;
         const bool real = e < E;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int rank = __popc(peers & lt_mask);
-        const int base = real ? running[e] : 0;
+        const int base = real ? cnt[warp][e] : 0;
         __syncwarp();
         if (real) {
             const int p = base + rank;
@@ -335,7 +510,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
                 sorted_assign[p] = static_cast<int>(a);
                 pos[a] = p;
             }
-            if (lane == __ffs(peers) - 1) running[e] = base + __popc(peers);
+            if (lane == __ffs(peers) - 1) cnt[warp][e] = base + __popc(peers);
         }
         __syncwarp();
     }
@@ -344,9 +519,58 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
+// per-device set-up of the shared-memory router: opt in to large dynamic
+// shared memory once per device and remember the SM count
+template <int ES>
+static cudaError_t router_smem_setup(int* num_sms) {
+    static std::atomic<int> ready[64];
+    static std::atomic<int> sms[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (ready[dev].load(std::memory_order_acquire) == 0) {
+        e = cudaFuncSetAttribute(router_logits_smem_kernel<ES>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        sms[dev].store(n);
+        ready[dev].store(1, std::memory_order_release);
+    }
+    *num_sms = sms[dev].load();
+    return cudaSuccess;
+}
+
+template <int ES>
+static cudaError_t launch_router_smem(const uint16_t* x, const float* W, const float* b,
+                                      float* logits, int T, int d, int E, int32_t* hist,
+                                      int hist_n, int32_t* status, cudaStream_t st) {
+    const int smem = router_smem_bytes(ES, d);
+    int num_sms = 0;
+    const cudaError_t e = router_smem_setup<ES>(&num_sms);
+    if (e != cudaSuccess) return e;
+    const int nslices = E / ES;
+    const int ntiles = (T + kRouterTile - 1) / kRouterTile;
+    int per_slice = num_sms / nslices;
+    if (per_slice < 1) per_slice = 1;
+    if (per_slice > ntiles) per_slice = ntiles;
+    router_logits_smem_kernel<ES><<<nslices * per_slice, kRouterWarps * 32, smem, st>>>(
+        x, W, b, logits, T, d, E, hist, hist_n, status);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float* b,
                                  float* logits, int T, int d, int E, int32_t* hist, int hist_n,
                                  int32_t* status, cudaStream_t st) {
+    // batches of at least one tile per SM use the shared-memory kernel
+    if (T >= kRouterTile * 2) {
+        if (E % 16 == 0 && router_smem_bytes(16, d) <= 227 * 1024)
+            return launch_router_smem<16>(x, W, b, logits, T, d, E, hist, hist_n, status, st);
+        if (router_smem_bytes(8, d) <= 227 * 1024)
+            return launch_router_smem<8>(x, W, b, logits, T, d, E, hist, hist_n, status, st);
+    }
     const int ty = T > 0 ? (T + kLogitTokPerCta - 1) / kLogitTokPerCta : 1;
     if (E % 16 == 0) {
         dim3 grid(E / 16, ty);
@@ -385,7 +609,8 @@ cudaError_t launch_route_scatter(const int32_t* topk_idx, const int32_t* gbase, 
                                  cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int ng = (T + kRouteGroupT - 1) / kRouteGroupT;
-    route_scatter_kernel<<<ng, 32, 0, st>>>(topk_idx, gbase, T, k, E, sorted_assign, pos, status);
+    route_scatter_kernel<<<ng, kScatterWarps * 32, 0, st>>>(topk_idx, gbase, T, k, E, sorted_assign,
+                                                          pos, status);
     return cudaGetLastError();
 }
 
