@@ -317,6 +317,7 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.NT = s.d / 256;
     g.out_ld = s.d;
     g.max_units = mb * g.NT;
+    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(T) * s.k, s.f, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;
     MOE_CUDA(moe::launch_finalize(y_acc, y, static_cast<long>(T) * s.d, st));

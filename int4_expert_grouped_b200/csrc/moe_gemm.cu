@@ -19,12 +19,17 @@
 //
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0       bulk-copies packed weight blocks into the W ring (TMA engine)
-//   warp 1       allocates TMEM, issues tcgen05.mma (one thread)
-//   warps 2-3    gather token rows into the B ring (cp.async, 128B swizzle)
+//   warp 1       allocates TMEM; runs the MMA loop, one elected lane issues
+//                tcgen05.mma and tcgen05.commit
+//   warps 2-3    gate/up: gather x rows by token index into the B ring
+//                (cp.async, 128B swizzle); down: warp 2 loads 2-D TMA tiles of
+//                h, warp 3 is idle
 //   warps 4-11   expand int4 -> bf16 from the W ring into the A ring
 //   warps 12-15  epilogue: TMEM -> registers -> h rows / y_acc reductions
 // TMEM holds two accumulator buffers of 2 x 128 columns, so the epilogue of
 // one unit overlaps the main loop of the next.
+#include <cudaTypedefs.h>
+
 #include "moe_internal.h"
 
 namespace moe {
@@ -32,14 +37,14 @@ namespace {
 
 constexpr int kWarpWProducer = 0;
 constexpr int kWarpMma = 1;
-constexpr int kWarpLoader0 = 2;
-constexpr int kNumLoaderWarps = 2;
+constexpr int kWarpLoader = 2;   // down: TMA tiles; gate/up: warps 2-3 gather with cp.async
+constexpr int kWarpIdle = 3;     // down only: no role
+constexpr int kGatherThreads = 64;
 constexpr int kWarpTransform0 = 4;
 constexpr int kNumTransformWarps = 8;
 constexpr int kWarpEpi0 = 12;
 constexpr int kNumEpiWarps = 4;
 constexpr int kGemmThreads = 16 * 32;
-constexpr int kLoaderThreads = kNumLoaderWarps * 32;
 constexpr int kTransformThreads = kNumTransformWarps * 32;
 
 constexpr int kNW = 4;  // packed weight ring
@@ -66,6 +71,9 @@ constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
 static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0, "UMMA tiles need 1024-byte alignment");
 static_assert(kOffW % 16 == 0 && kWStageBytes % 16 == 0, "bulk copies need 16-byte alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(kWarpIdle + 1 == kWarpTransform0 && kWarpEpi0 % 4 == 0 &&
+                  kWarpEpi0 + kNumEpiWarps == kGemmThreads / 32,
+              "every warp has exactly one role; epilogue warps cover TMEM quadrants 0..3");
 
 constexpr uint32_t kTmemCols = 512;
 
@@ -107,6 +115,12 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
+// mbar_wait for a whole converged warp: every lane waits and the outcome is
+// voted, so the warp takes the same branch whatever happens at a timeout.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
 // Wait used only while shutting down after an abort: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = globaltimer();
@@ -117,7 +131,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 template <bool kDown>
-__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const GemmArgs a) {
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -149,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
             mbar_init(aempty(s), 1);
         }
         for (int s = 0; s < kNB; ++s) {
-            mbar_init(bfull(s), kLoaderThreads);
+            mbar_init(bfull(s), kDown ? 1 : kGatherThreads);
             mbar_init(bempty(s), 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -179,67 +193,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
     };
 
     if (warp == kWarpWProducer) {
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-                const int b = u / NT;
-                const int j = u - b * NT;
-                const int e = a.block_map[3 * b];
-                const uint8_t* src =
-                    a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
-                for (int c = 0; c < KC; ++c, ++it) {
-                    const int s = it % kNW;
-                    if (!mbar_wait(wempty(s), ((it / kNW) & 1) ^ 1, abort_flag)) {
-                        fail(1);
-                        ok = false;
-                        break;
-                    }
+        // the whole warp runs the loop; one elected lane issues the copies
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            const int b = u / NT;
+            const int j = u - b * NT;
+            const int e = a.block_map[3 * b];
+            const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
+            for (int c = 0; c < KC; ++c, ++it) {
+                const int s = it % kNW;
+                if (!warp_wait(wempty(s), ((it / kNW) & 1) ^ 1, abort_flag)) {
+                    fail(1);
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
                     mbar_arrive_expect_tx(wfull(s), a.block_bytes);
                     bulk_copy_g2s(sbase + kOffW + s * kWStageBytes, src + c * a.block_bytes,
                                   a.block_bytes, wfull(s));
                 }
-            }
-            if (!ok) {
-                // let the copies already issued land before the CTA exits
-                const uint32_t first = it > kNW ? it - kNW : 0;
-                for (uint32_t i = first; i < it; ++i)
-                    mbar_wait_drain(wfull(i % kNW), (i / kNW) & 1);
+                __syncwarp();
             }
         }
+        if (!ok && lane == 0) {
+            // let the copies already issued land before the CTA exits
+            const uint32_t first = it > kNW ? it - kNW : 0;
+            for (uint32_t i = first; i < it; ++i) mbar_wait_drain(wfull(i % kNW), (i / kNW) & 1);
+        }
     } else if (warp == kWarpMma) {
-        if (lane == 0) {
-            uint32_t it = 0, ucount = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x, ++ucount) {
-                const int b = u / NT;
-                const int rows = a.block_map[3 * b + 2];
-                const int N = (rows + 15) & ~15;
-                const uint32_t idesc = make_idesc_bf16(128, N);
-                const int buf = ucount & 1;
-                if (!mbar_wait(accempty(buf), ((ucount >> 1) & 1) ^ 1, abort_flag)) {
-                    fail(2);
+        // The whole warp runs the issue loop so descriptors and ring indices
+        // stay warp-uniform; one elected lane issues each MMA and commit.
+        uint32_t it = 0, ucount = 0;
+        bool ok = true;
+        bool ready = false;  // the current stage was already seen full
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x, ++ucount) {
+            const int b = u / NT;
+            const int rows = a.block_map[3 * b + 2];
+            const int N = (rows + 15) & ~15;
+            const uint32_t idesc = make_idesc_bf16(128, N);
+            const int buf = ucount & 1;
+            if (!warp_wait(accempty(buf), ((ucount >> 1) & 1) ^ 1, abort_flag)) {
+                fail(2);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d0 = tmem + buf * 256;
+            const uint32_t d1 = d0 + 128;
+            for (int c = 0; c < KC; ++c, ++it) {
+                const int sa = it % kNA;
+                const int sb = it % kNB;
+                if (!ready && (!warp_wait(afull(sa), (it / kNA) & 1, abort_flag) ||
+                               !warp_wait(bfull(sb), (it / kNB) & 1, abort_flag))) {
+                    fail(3);
                     ok = false;
                     break;
                 }
+                // order the asynchronous MMAs after the waits, and the B rows
+                // written by cp.async (generic proxy) before the MMA reads them
                 tc_fence_after();
-                const uint32_t d0 = tmem + buf * 256;
-                const uint32_t d1 = d0 + 128;
-                for (int c = 0; c < KC; ++c, ++it) {
-                    const int sa = it % kNA;
-                    const int sb = it % kNB;
-                    if (!mbar_wait(afull(sa), (it / kNA) & 1, abort_flag) ||
-                        !mbar_wait(bfull(sb), (it / kNB) & 1, abort_flag)) {
-                        fail(3);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    fence_proxy_async_smem();
-                    const uint32_t abase = sbase + kOffA + sa * kAStageBytes;
-                    const uint64_t da0 = make_sw128_desc(abase);
-                    const uint64_t da1 = make_sw128_desc(abase + kATileBytes);
-                    const uint64_t db = make_sw128_desc(sbase + kOffB + sb * kBStageBytes);
+                fence_proxy_async_smem();
+                // Test the next stage now and look at the answer only after this
+                // stage's MMAs are issued: a barrier read stalls the issuing
+                // thread for about as long as one MMA runs, and the tensor core's
+                // queue is too short to hide it.
+                const uint32_t nx = it + 1;
+                const uint32_t ra = mbar_test(afull(nx % kNA), (nx / kNA) & 1);
+                const uint32_t rb = mbar_test(bfull(nx % kNB), (nx / kNB) & 1);
+                const uint32_t abase = sbase + kOffA + sa * kAStageBytes;
+                const uint64_t da0 = make_sw128_desc(abase);
+                const uint64_t da1 = make_sw128_desc(abase + kATileBytes);
+                const uint64_t db = make_sw128_desc(sbase + kOffB + sb * kBStageBytes);
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kKChunk / 16; ++kk) {
                         const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
@@ -249,21 +275,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
                     mma_commit(aempty(sa));
                     mma_commit(bempty(sb));
                 }
-                if (ok) mma_commit(accfull(buf));
+                ready = __all_sync(0xffffffffu, (ra & rb) != 0);
             }
-            if (!ok) {
-                mma_commit(drain_bar);
-                mbar_wait_drain(drain_bar, 0);
+            if (ok && elect_one()) mma_commit(accfull(buf));
+            __syncwarp();
+        }
+        if (!ok) {
+            if (elect_one()) mma_commit(drain_bar);
+            __syncwarp();
+            mbar_wait_drain(drain_bar, 0);
+        }
+    } else if (kDown && warp == kWarpLoader) {
+        // down: one 128-row TMA tile of h per stage (rows past the block belong
+        // to the next expert or lie past the end and are zero-filled; the MMA
+        // ignores columns >= N)
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            const int row0 = a.block_map[3 * (u / NT) + 1];
+            for (int c = 0; c < KC; ++c, ++it) {
+                const int s = it % kNB;
+                if (!mbar_wait(bempty(s), ((it / kNB) & 1) ^ 1, abort_flag)) {
+                    fail(4);
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bfull(s), kBStageBytes);
+                    tma_load_2d(sbase + kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
+                }
+                __syncwarp();
             }
         }
-    } else if (warp >= kWarpLoader0 && warp < kWarpLoader0 + kNumLoaderWarps) {
-        // Lane layout: 8 consecutive lanes copy the 8 16-byte pieces of one
-        // 128-byte row chunk, so a warp instruction reads 4 whole rows.
-        // Thread ltid copies piece (ltid % 8) of rows ltid/8 + 8*jr.
-        const int ltid = threadIdx.x - kWarpLoader0 * 32;
+    } else if (!kDown && (warp == kWarpLoader || warp == kWarpLoader + 1)) {
+        // gate/up: gather x rows by token index with 16-byte cp.async.  Lane
+        // layout: 8 consecutive lanes copy the 8 pieces of one 128-byte row, so a
+        // warp instruction reads 4 whole rows; thread ltid copies piece ltid % 8
+        // of rows ltid/8 + 8*jr.  Completion is signalled asynchronously
+        // (cp.async.mbarrier.arrive.noinc), so no thread waits for the copies.
+        const int ltid = threadIdx.x - kWarpLoader * 32;
         const int piece = ltid & 7;
         const int rbase = ltid >> 3;
-        constexpr int kRowsPerThread = kBlockT / (kLoaderThreads / 8);
+        constexpr int kRowsPerThread = kBlockT / (kGatherThreads / 8);
         const uint32_t swz = static_cast<uint32_t>((piece ^ rbase) << 4);  // row & 7 == rbase
         uint32_t it = 0;
         bool ok = true;
@@ -279,7 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
                 const int r = rbase + 8 * jr;
                 long srow = 0;
                 if (r < rows) {
-                    srow = kDown ? row0 + r : a.sorted_assign[row0 + r] / a.topk;
+                    srow = a.sorted_assign[row0 + r] / a.topk;
                     valid_mask |= 1u << jr;
                 }
                 src[jr] = a.act + srow * a.K + piece * 8;
@@ -347,7 +400,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const Gem
                 }
             }
         }
-    } else {
+    } else if (warp >= kWarpEpi0) {
         // epilogue warps: warp % 4 selects the TMEM lane quadrant
         const int q = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
@@ -528,6 +581,28 @@ cudaError_t prepare_gemm_kernels() {
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(grouped_gemm_kernel<true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                                 uint32_t box_rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (encode == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return e != cudaSuccess ? e : cudaErrorInvalidValue;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kKChunk), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* out,

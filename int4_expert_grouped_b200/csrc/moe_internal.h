@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "moe_common.cuh"
@@ -72,6 +73,10 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
                            cudaStream_t st);
 
 struct GemmArgs {
+    // B operand (token rows) for TMA: gate/up gathers rows of x [T, d] four at
+    // a time (box 64 x 1); down reads h [T*k, f] tiles (box 64 x 128).  Both use
+    // the 128-byte swizzle, which is the K-major layout the MMA reads.
+    CUtensorMap bmap;
     const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
     const uint16_t* act;           // B rows: x [T, d] (gate/up) or h [T*k, f] (down)
     const int32_t* sorted_assign;  // [T*k]
@@ -89,6 +94,10 @@ struct GemmArgs {
     int block_bytes;
     int max_units;                 // upper bound of num_blocks * NT
 };
+// Encode the tensor map of a row-major bf16 matrix [rows, cols] read in boxes
+// of 64 columns x box_rows rows with the 128-byte swizzle.
+cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                                 uint32_t box_rows);
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_finalize(const float* y_acc, uint16_t* y, long n, cudaStream_t st);
