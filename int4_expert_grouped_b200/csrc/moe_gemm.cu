@@ -39,7 +39,8 @@ constexpr int kWarpWProducer = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpLoader = 2;   // down: TMA tiles; gate/up: warps 2-3 gather with cp.async
 constexpr int kWarpIdle = 3;     // down only: no role
-constexpr int kGatherThreads = 64;
+constexpr int kGatherThreads = 64;    // gate/up gather warps 2-3
+constexpr int kTransformGroups = 2;   // transform warp groups, alternate chunks
 constexpr int kWarpTransform0 = 4;
 constexpr int kNumTransformWarps = 8;
 constexpr int kWarpEpi0 = 12;
@@ -71,6 +72,16 @@ constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
 static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0, "UMMA tiles need 1024-byte alignment");
 static_assert(kOffW % 16 == 0 && kWStageBytes % 16 == 0, "bulk copies need 16-byte alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+// mbarrier parity waits only tell a phase from the one before it, so no
+// waiter may ever be two phases ahead of a barrier.  With transform groups
+// taking alternate chunks this holds when every W stage is consumed by a
+// single group (kNW a multiple of the group count) and, for the A ring shared
+// by the groups, when there are at most two groups: a group reaches a stage's
+// next use only after the MMA consumed the chunk before it, which needs the
+// other group's fill.  (Three- or four-group variants deadlock in a
+// discrete-event model of this protocol.)
+static_assert(kNW % kTransformGroups == 0 && kTransformGroups <= 2,
+              "transform groups must not alias mbarrier phases");
 static_assert(kWarpIdle + 1 == kWarpTransform0 && kWarpEpi0 % 4 == 0 &&
                   kWarpEpi0 + kNumEpiWarps == kGemmThreads / 32,
               "every warp has exactly one role; epilogue warps cover TMEM quadrants 0..3");
@@ -156,10 +167,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNW; ++s) {
             mbar_init(wfull(s), 1);
-            mbar_init(wempty(s), kNumTransformWarps);
+            mbar_init(wempty(s), kNumTransformWarps / kTransformGroups);
         }
         for (int s = 0; s < kNA; ++s) {
-            mbar_init(afull(s), kNumTransformWarps);
+            mbar_init(afull(s), kNumTransformWarps / kTransformGroups);
             mbar_init(aempty(s), 1);
         }
         for (int s = 0; s < kNB; ++s) {
@@ -310,9 +321,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     } else if (!kDown && (warp == kWarpLoader || warp == kWarpLoader + 1)) {
         // gate/up: gather x rows by token index with 16-byte cp.async.  Lane
         // layout: 8 consecutive lanes copy the 8 pieces of one 128-byte row, so a
-        // warp instruction reads 4 whole rows; thread ltid copies piece ltid % 8
-        // of rows ltid/8 + 8*jr.  Completion is signalled asynchronously
-        // (cp.async.mbarrier.arrive.noinc), so no thread waits for the copies.
+        // warp instruction reads 4 whole rows; thread ltid (0..63) copies piece
+        // ltid % 8 of rows ltid/8 + 8*jr.  Completion is signalled
+        // asynchronously (cp.async.mbarrier.arrive.noinc), so no thread waits
+        // for its copies.
         const int ltid = threadIdx.x - kWarpLoader * 32;
         const int piece = ltid & 7;
         const int rbase = ltid >> 3;
@@ -325,21 +337,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int row0 = a.block_map[3 * b + 1];
             const int rows = a.block_map[3 * b + 2];
             const int N = (rows + 15) & ~15;
-            const uint16_t* src[kRowsPerThread];
-            uint32_t valid_mask = 0;
+            uint32_t off[kRowsPerThread];  // element offset of the source row piece
 #pragma unroll
             for (int jr = 0; jr < kRowsPerThread; ++jr) {
                 const int r = rbase + 8 * jr;
-                long srow = 0;
-                if (r < rows) {
-                    srow = a.sorted_assign[row0 + r] / a.topk;
-                    valid_mask |= 1u << jr;
-                }
-                src[jr] = a.act + srow * a.K + piece * 8;
+                const int t = r < rows ? a.sorted_assign[row0 + r] / a.topk : 0;
+                off[jr] = static_cast<uint32_t>(t) * static_cast<uint32_t>(a.K) + piece * 8;
             }
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % kNB;
-                if (!mbar_wait(bempty(s), ((it / kNB) & 1) ^ 1, abort_flag)) {
+                if (!warp_wait(bempty(s), ((it / kNB) & 1) ^ 1, abort_flag)) {
                     fail(4);
                     ok = false;
                     break;
@@ -349,24 +356,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 for (int jr = 0; jr < kRowsPerThread; ++jr) {
                     const int r = rbase + 8 * jr;
                     if (r < N)
-                        cp_async_16(dst + r * 128, src[jr] + c * kKChunk,
-                                    (valid_mask >> jr) & 1u ? 16u : 0u);
+                        cp_async_16(dst + r * 128, a.act + off[jr] + c * kKChunk, r < rows ? 16u : 0u);
                 }
                 cp_async_arrive_noinc(bfull(s));
             }
         }
         cp_async_wait_all();
     } else if (warp >= kWarpTransform0 && warp < kWarpTransform0 + kNumTransformWarps) {
+        // Two groups of transform warps take alternate chunks, so each warp
+        // pays one round of barrier waits per two chunks.
+        constexpr int kGroupThreads = kTransformThreads / kTransformGroups;
+        constexpr int kTasks = 512 / kGroupThreads;  // (row, half) tasks per thread
         const int ttid = threadIdx.x - kWarpTransform0 * 32;
+        const int grp = ttid / kGroupThreads;
+        const int gtid = ttid % kGroupThreads;
         const int gpc = kKChunk / a.group;
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
             for (int c = 0; c < KC; ++c, ++it) {
+                if (static_cast<int>(it % kTransformGroups) != grp) continue;
                 const int sw = it % kNW;
                 const int sa = it % kNA;
-                if (!mbar_wait(wfull(sw), (it / kNW) & 1, abort_flag) ||
-                    !mbar_wait(aempty(sa), ((it / kNA) & 1) ^ 1, abort_flag)) {
+                if (!warp_wait(wfull(sw), (it / kNW) & 1, abort_flag) ||
+                    !warp_wait(aempty(sa), ((it / kNA) & 1) ^ 1, abort_flag)) {
                     fail(5);
                     ok = false;
                     break;
@@ -374,8 +387,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 const uint8_t* wst = smem + kOffW + sw * kWStageBytes;
                 const uint32_t ast = sbase + kOffA + sa * kAStageBytes;
 #pragma unroll
-                for (int rep = 0; rep < 2; ++rep) {
-                    const int task = ttid + kTransformThreads * rep;
+                for (int rep = 0; rep < kTasks; ++rep) {
+                    const int task = gtid + kGroupThreads * rep;
                     const int row = task >> 1;  // 0..255: A0 rows then A1 rows
                     const int half = task & 1;  // K 0..31 or 32..63 of the chunk
                     const uint4 pk = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
