@@ -8,14 +8,21 @@
 //   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
 //       gate/up: D0 = Wg x^T, D1 = Wu x^T over gathered token rows, epilogue
 //                h = silu(D0) * D1 -> bf16 h rows in expert order
-//       down:    D0, D1 = two 128-row tiles of Wd times h^T, epilogue
+//       down:    D = 128-row tile of Wd times h^T, epilogue
 //                y_acc[t] += topk_w * D (fp32 reduction in L2)
 //   finalize_kernel       y = bf16(y_acc)
 //
-// One work unit = one block-map tile (<= 128 expert-ordered rows of one
-// expert) x one pair of 128-row weight tiles.  The weights are the MMA A
-// operand (M = 128 per tile), the tokens the B operand (N = rows rounded up to
-// 16), so a partly filled tile wastes at most 15 columns.
+// One work unit = one block-map tile (<= 256 expert-ordered rows of one
+// expert) x one output tile of 128 features (gate/up: the gate and the up
+// rows of those features).  The weights are the MMA A operand (M = 128 per
+// tile), the tokens the B operand (N = rows rounded up to 16 <= 256), so a
+// partly filled tile wastes at most 15 columns.
+//
+// Shapes are set by two limits measured on B200: expanding int4 costs about
+// two instructions per weight, so every expanded weight must serve up to 256
+// tokens; and the MMA's shared-memory operand reads share the read port with
+// ordinary loads, so each MMA should read as little shared memory per flop as
+// possible (M = 128 x N = 256 reads 96 bytes per clock at full rate).
 //
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0       bulk-copies packed weight blocks into the W ring (TMA engine)
@@ -24,10 +31,12 @@
 //   warps 2-3    gate/up: gather x rows by token index into the B ring
 //                (cp.async, 128B swizzle); down: warp 2 loads 2-D TMA tiles of
 //                h, warp 3 is idle
-//   warps 4-11   expand int4 -> bf16 from the W ring into the A ring
+//   warps 4-11   expand int4 -> bf16 from the W ring into the A ring, in two
+//                groups that take alternate K chunks
 //   warps 12-15  epilogue: TMEM -> registers -> h rows / y_acc reductions
-// TMEM holds two accumulator buffers of 2 x 128 columns, so the epilogue of
-// one unit overlaps the main loop of the next.
+// TMEM: gate/up holds one buffer of 2 x 256 columns (gate, up), so its
+// epilogue runs between units; down holds two buffers of 256 columns, so its
+// epilogue overlaps the next unit's main loop.
 #include <cudaTypedefs.h>
 
 #include "moe_internal.h"
@@ -47,46 +56,57 @@ constexpr int kWarpEpi0 = 12;
 constexpr int kNumEpiWarps = 4;
 constexpr int kGemmThreads = 16 * 32;
 constexpr int kTransformThreads = kNumTransformWarps * 32;
+constexpr int kGroupThreads = kTransformThreads / kTransformGroups;
+constexpr int kATileBytes = 128 * 128;     // 128 rows x 64 bf16 (128B swizzle)
+constexpr int kBStageBytes = kBlockT * 128;  // up to 256 token rows x 64 bf16
+constexpr int kEpiRowBytes = 80;    // gate/up staging row: 32 bf16 + 16 bytes of padding
+constexpr int kEpiRowFloats = 36;   // down staging row: 32 fp32 + 4 of padding
+constexpr uint32_t kTmemCols = 512;
 
-constexpr int kNW = 4;  // packed weight ring
-constexpr int kNA = 3;  // expanded bf16 A ring
-constexpr int kNB = 4;  // token B ring
-constexpr int kATileBytes = 128 * 128;
-constexpr int kAStageBytes = 2 * kATileBytes;
-constexpr int kBStageBytes = kBlockT * 128;
-constexpr int kWStageBytes = packed_block_bytes(32);
-constexpr int kNibbleBytes = 256 * 32;
-constexpr int kEpiRowBytes = 80;  // gate/up staging row: 32 bf16 + 16 bytes of padding
-constexpr int kEpiRowFloats = 36;  // down staging row: 32 fp32 + 4 of padding
-constexpr int kEpiWarpBytes = 32 * kEpiRowFloats * 4;
+// Per-projection configuration.
+template <bool kDown>
+struct Cfg {
+    static constexpr int kTiles = kDown ? 1 : 2;             // A tiles (of 128 rows) per unit
+    static constexpr int kNW = 4;                             // packed weight ring
+    static constexpr int kNA = kDown ? 4 : 2;                 // expanded bf16 A ring
+    static constexpr int kNB = 3;                             // token B ring
+    static constexpr int kAccBufs = kDown ? 2 : 1;            // TMEM accumulator buffers
+    static constexpr int kAccCols = kTiles * kBlockT;         // columns per buffer
+    static constexpr int kAStageBytes = kTiles * kATileBytes;
+    static constexpr int kWStageBytes = packed_block_bytes(kTiles, 32);  // largest (group 32)
+    static constexpr int kNibbleBytes = kTiles * 128 * 32;
+    static constexpr int kEpiWarpBytes = kDown ? 32 * kEpiRowFloats * 4 : 32 * kEpiRowBytes;
+    static constexpr int kTasks = kTiles * 256 / kGroupThreads;  // (row, half) tasks per thread
 
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kNA * kAStageBytes;
-constexpr int kOffW = kOffB + kNB * kBStageBytes;
-constexpr int kOffEpi = kOffW + kNW * kWStageBytes;
-constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiWarpBytes;
-constexpr int kNumBars = 2 * kNW + 2 * kNA + 2 * kNB + 2 + 2 + 1;
-constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-constexpr int kSmemUsed = kOffMisc + 16;
-constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
-static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0, "UMMA tiles need 1024-byte alignment");
-static_assert(kOffW % 16 == 0 && kWStageBytes % 16 == 0, "bulk copies need 16-byte alignment");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-// mbarrier parity waits only tell a phase from the one before it, so no
-// waiter may ever be two phases ahead of a barrier.  With transform groups
-// taking alternate chunks this holds when every W stage is consumed by a
-// single group (kNW a multiple of the group count) and, for the A ring shared
-// by the groups, when there are at most two groups: a group reaches a stage's
-// next use only after the MMA consumed the chunk before it, which needs the
-// other group's fill.  (Three- or four-group variants deadlock in a
-// discrete-event model of this protocol.)
-static_assert(kNW % kTransformGroups == 0 && kTransformGroups <= 2,
-              "transform groups must not alias mbarrier phases");
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kOffA + kNA * kAStageBytes;
+    static constexpr int kOffW = kOffB + kNB * kBStageBytes;
+    static constexpr int kOffEpi = kOffW + kNW * kWStageBytes;
+    static constexpr int kOffBar = kOffEpi + kNumEpiWarps * kEpiWarpBytes;
+    static constexpr int kNumBars = 2 * kNW + 2 * kNA + 2 * kNB + 2 * kAccBufs + 1;
+    static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base
+
+    static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0 && kAStageBytes % 1024 == 0,
+                  "UMMA tiles need 1024-byte alignment");
+    static_assert(kOffW % 16 == 0 && kWStageBytes % 16 == 0, "bulk copies need 16-byte alignment");
+    static_assert(kOffBar % 8 == 0, "mbarriers are 8-byte aligned");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kAccBufs * kAccCols <= static_cast<int>(kTmemCols), "TMEM budget");
+    // mbarrier parity waits only tell a phase from the one before it, so no
+    // waiter may ever be two phases ahead of a barrier.  Transform groups take
+    // alternate chunks; with ring sizes that are multiples of the group count
+    // every W and A stage is filled and released by one group only, which
+    // keeps each group at most one phase ahead.  (A shared A ring with three
+    // or four groups deadlocks in a discrete-event model of this protocol.)
+    static_assert(kNW % kTransformGroups == 0 && kNA % kTransformGroups == 0,
+                  "transform groups must not alias mbarrier phases");
+    static_assert(kTasks * kGroupThreads == kTiles * 256, "transform task split");
+};
+
 static_assert(kWarpIdle + 1 == kWarpTransform0 && kWarpEpi0 % 4 == 0 &&
                   kWarpEpi0 + kNumEpiWarps == kGemmThreads / 32,
               "every warp has exactly one role; epilogue warps cover TMEM quadrants 0..3");
-
-constexpr uint32_t kTmemCols = 512;
 
 union BF2 {
     uint32_t u;
@@ -143,6 +163,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
 
 template <bool kDown>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
+    using C = Cfg<kDown>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -151,33 +172,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     const int lane = threadIdx.x & 31;
 
     // barrier addresses
-    const uint32_t bar0 = sbase + kOffBar;
+    const uint32_t bar0 = sbase + C::kOffBar;
     auto wfull = [&](int s) { return bar0 + 8u * s; };
-    auto wempty = [&](int s) { return bar0 + 8u * (kNW + s); };
-    auto afull = [&](int s) { return bar0 + 8u * (2 * kNW + s); };
-    auto aempty = [&](int s) { return bar0 + 8u * (2 * kNW + kNA + s); };
-    auto bfull = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + s); };
-    auto bempty = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + kNB + s); };
-    auto accfull = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + 2 * kNB + s); };
-    auto accempty = [&](int s) { return bar0 + 8u * (2 * kNW + 2 * kNA + 2 * kNB + 2 + s); };
-    const uint32_t drain_bar = bar0 + 8u * (kNumBars - 1);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    auto wempty = [&](int s) { return bar0 + 8u * (C::kNW + s); };
+    auto afull = [&](int s) { return bar0 + 8u * (2 * C::kNW + s); };
+    auto aempty = [&](int s) { return bar0 + 8u * (2 * C::kNW + C::kNA + s); };
+    auto bfull = [&](int s) { return bar0 + 8u * (2 * C::kNW + 2 * C::kNA + s); };
+    auto bempty = [&](int s) { return bar0 + 8u * (2 * C::kNW + 2 * C::kNA + C::kNB + s); };
+    auto accfull = [&](int s) { return bar0 + 8u * (2 * C::kNW + 2 * C::kNA + 2 * C::kNB + s); };
+    auto accempty = [&](int s) {
+        return bar0 + 8u * (2 * C::kNW + 2 * C::kNA + 2 * C::kNB + C::kAccBufs + s);
+    };
+    const uint32_t drain_bar = bar0 + 8u * (C::kNumBars - 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNW; ++s) {
+        for (int s = 0; s < C::kNW; ++s) {
             mbar_init(wfull(s), 1);
             mbar_init(wempty(s), kNumTransformWarps / kTransformGroups);
         }
-        for (int s = 0; s < kNA; ++s) {
+        for (int s = 0; s < C::kNA; ++s) {
             mbar_init(afull(s), kNumTransformWarps / kTransformGroups);
             mbar_init(aempty(s), 1);
         }
-        for (int s = 0; s < kNB; ++s) {
+        for (int s = 0; s < C::kNB; ++s) {
             mbar_init(bfull(s), kDown ? 1 : kGatherThreads);
             mbar_init(bempty(s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::kAccBufs; ++s) {
             mbar_init(accfull(s), 1);
             mbar_init(accempty(s), kNumEpiWarps);
         }
@@ -213,15 +236,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int e = a.block_map[3 * b];
             const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
             for (int c = 0; c < KC; ++c, ++it) {
-                const int s = it % kNW;
-                if (!warp_wait(wempty(s), ((it / kNW) & 1) ^ 1, abort_flag)) {
+                const int s = it % C::kNW;
+                if (!warp_wait(wempty(s), ((it / C::kNW) & 1) ^ 1, abort_flag)) {
                     fail(1);
                     ok = false;
                     break;
                 }
                 if (elect_one()) {
                     mbar_arrive_expect_tx(wfull(s), a.block_bytes);
-                    bulk_copy_g2s(sbase + kOffW + s * kWStageBytes, src + c * a.block_bytes,
+                    bulk_copy_g2s(sbase + C::kOffW + s * C::kWStageBytes, src + c * a.block_bytes,
                                   a.block_bytes, wfull(s));
                 }
                 __syncwarp();
@@ -229,8 +252,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         }
         if (!ok && lane == 0) {
             // let the copies already issued land before the CTA exits
-            const uint32_t first = it > kNW ? it - kNW : 0;
-            for (uint32_t i = first; i < it; ++i) mbar_wait_drain(wfull(i % kNW), (i / kNW) & 1);
+            const uint32_t first = it > C::kNW ? it - C::kNW : 0;
+            for (uint32_t i = first; i < it; ++i)
+                mbar_wait_drain(wfull(i % C::kNW), (i / C::kNW) & 1);
         }
     } else if (warp == kWarpMma) {
         // The whole warp runs the issue loop so descriptors and ring indices
@@ -243,20 +267,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int rows = a.block_map[3 * b + 2];
             const int N = (rows + 15) & ~15;
             const uint32_t idesc = make_idesc_bf16(128, N);
-            const int buf = ucount & 1;
-            if (!warp_wait(accempty(buf), ((ucount >> 1) & 1) ^ 1, abort_flag)) {
+            const int buf = ucount % C::kAccBufs;
+            const uint32_t use = ucount / C::kAccBufs;
+            if (!warp_wait(accempty(buf), (use & 1) ^ 1, abort_flag)) {
                 fail(2);
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t d0 = tmem + buf * 256;
-            const uint32_t d1 = d0 + 128;
+            const uint32_t dacc = tmem + buf * C::kAccCols;
             for (int c = 0; c < KC; ++c, ++it) {
-                const int sa = it % kNA;
-                const int sb = it % kNB;
-                if (!ready && (!warp_wait(afull(sa), (it / kNA) & 1, abort_flag) ||
-                               !warp_wait(bfull(sb), (it / kNB) & 1, abort_flag))) {
+                const int sa = it % C::kNA;
+                const int sb = it % C::kNB;
+                if (!ready && (!warp_wait(afull(sa), (it / C::kNA) & 1, abort_flag) ||
+                               !warp_wait(bfull(sb), (it / C::kNB) & 1, abort_flag))) {
                     fail(3);
                     ok = false;
                     break;
@@ -270,18 +294,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 // thread for about as long as one MMA runs, and the tensor core's
                 // queue is too short to hide it.
                 const uint32_t nx = it + 1;
-                const uint32_t ra = mbar_test(afull(nx % kNA), (nx / kNA) & 1);
-                const uint32_t rb = mbar_test(bfull(nx % kNB), (nx / kNB) & 1);
-                const uint32_t abase = sbase + kOffA + sa * kAStageBytes;
-                const uint64_t da0 = make_sw128_desc(abase);
-                const uint64_t da1 = make_sw128_desc(abase + kATileBytes);
-                const uint64_t db = make_sw128_desc(sbase + kOffB + sb * kBStageBytes);
+                const uint32_t ra = mbar_test(afull(nx % C::kNA), (nx / C::kNA) & 1);
+                const uint32_t rb = mbar_test(bfull(nx % C::kNB), (nx / C::kNB) & 1);
+                const uint32_t abase = sbase + C::kOffA + sa * C::kAStageBytes;
+                const uint64_t db = make_sw128_desc(sbase + C::kOffB + sb * kBStageBytes);
+                uint64_t da[C::kTiles];
+#pragma unroll
+                for (int t = 0; t < C::kTiles; ++t) da[t] = make_sw128_desc(abase + t * kATileBytes);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kKChunk / 16; ++kk) {
                         const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
-                        mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, acc);
-                        mma_bf16(d1, da1 + 2 * kk, db + 2 * kk, idesc, acc);
+#pragma unroll
+                        for (int t = 0; t < C::kTiles; ++t)
+                            mma_bf16(dacc + t * kBlockT, da[t] + 2 * kk, db + 2 * kk, idesc, acc);
                     }
                     mma_commit(aempty(sa));
                     mma_commit(bempty(sb));
@@ -297,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             mbar_wait_drain(drain_bar, 0);
         }
     } else if (kDown && warp == kWarpLoader) {
-        // down: one 128-row TMA tile of h per stage (rows past the block belong
+        // down: one 256-row TMA tile of h per stage (rows past the block belong
         // to the next expert or lie past the end and are zero-filled; the MMA
         // ignores columns >= N)
         uint32_t it = 0;
@@ -305,15 +331,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
             const int row0 = a.block_map[3 * (u / NT) + 1];
             for (int c = 0; c < KC; ++c, ++it) {
-                const int s = it % kNB;
-                if (!mbar_wait(bempty(s), ((it / kNB) & 1) ^ 1, abort_flag)) {
+                const int s = it % C::kNB;
+                if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
                     fail(4);
                     ok = false;
                     break;
                 }
-                if (lane == 0) {
+                if (elect_one()) {
                     mbar_arrive_expect_tx(bfull(s), kBStageBytes);
-                    tma_load_2d(sbase + kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
+                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
                 }
                 __syncwarp();
             }
@@ -345,13 +371,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 off[jr] = static_cast<uint32_t>(t) * static_cast<uint32_t>(a.K) + piece * 8;
             }
             for (int c = 0; c < KC; ++c, ++it) {
-                const int s = it % kNB;
-                if (!warp_wait(bempty(s), ((it / kNB) & 1) ^ 1, abort_flag)) {
+                const int s = it % C::kNB;
+                if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
                     fail(4);
                     ok = false;
                     break;
                 }
-                const uint32_t dst = sbase + kOffB + s * kBStageBytes + swz;
+                const uint32_t dst = sbase + C::kOffB + s * kBStageBytes + swz;
 #pragma unroll
                 for (int jr = 0; jr < kRowsPerThread; ++jr) {
                     const int r = rbase + 8 * jr;
@@ -365,8 +391,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     } else if (warp >= kWarpTransform0 && warp < kWarpTransform0 + kNumTransformWarps) {
         // Two groups of transform warps take alternate chunks, so each warp
         // pays one round of barrier waits per two chunks.
-        constexpr int kGroupThreads = kTransformThreads / kTransformGroups;
-        constexpr int kTasks = 512 / kGroupThreads;  // (row, half) tasks per thread
         const int ttid = threadIdx.x - kWarpTransform0 * 32;
         const int grp = ttid / kGroupThreads;
         const int gtid = ttid % kGroupThreads;
@@ -376,25 +400,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
             for (int c = 0; c < KC; ++c, ++it) {
                 if (static_cast<int>(it % kTransformGroups) != grp) continue;
-                const int sw = it % kNW;
-                const int sa = it % kNA;
-                if (!warp_wait(wfull(sw), (it / kNW) & 1, abort_flag) ||
-                    !warp_wait(aempty(sa), ((it / kNA) & 1) ^ 1, abort_flag)) {
+                const int sw = it % C::kNW;
+                const int sa = it % C::kNA;
+                if (!warp_wait(wfull(sw), (it / C::kNW) & 1, abort_flag) ||
+                    !warp_wait(aempty(sa), ((it / C::kNA) & 1) ^ 1, abort_flag)) {
                     fail(5);
                     ok = false;
                     break;
                 }
-                const uint8_t* wst = smem + kOffW + sw * kWStageBytes;
-                const uint32_t ast = sbase + kOffA + sa * kAStageBytes;
+                const uint8_t* wst = smem + C::kOffW + sw * C::kWStageBytes;
+                const uint32_t ast = sbase + C::kOffA + sa * C::kAStageBytes;
 #pragma unroll
-                for (int rep = 0; rep < kTasks; ++rep) {
+                for (int rep = 0; rep < C::kTasks; ++rep) {
                     const int task = gtid + kGroupThreads * rep;
-                    const int row = task >> 1;  // 0..255: A0 rows then A1 rows
+                    const int row = task >> 1;  // packed row: tile row>>7, row & 127 within it
                     const int half = task & 1;  // K 0..31 or 32..63 of the chunk
                     const uint4 pk = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
-                    const int g = (half * 32) / a.group;
+                    const int g = half * (gpc - 1);  // group 64: 0; group 32: half
                     const uint32_t sb = *reinterpret_cast<const uint32_t*>(
-                        wst + kNibbleBytes + (row * gpc + g) * 4);
+                        wst + C::kNibbleBytes + (row * gpc + g) * 4);
                     BF2 s2, b2;
                     s2.u = __byte_perm(sb, 0, 0x1010);
                     b2.u = __byte_perm(sb, 0, 0x3232);
@@ -417,7 +441,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         // epilogue warps: warp % 4 selects the TMEM lane quadrant
         const int q = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        uint8_t* stg = smem + kOffEpi + (warp - kWarpEpi0) * kEpiWarpBytes;
+        uint8_t* stg = smem + C::kOffEpi + (warp - kWarpEpi0) * C::kEpiWarpBytes;
+        constexpr int kMaxCb = kBlockT / 32;
         uint32_t ucount = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++ucount) {
             const int b = u / NT;
@@ -425,13 +450,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int row0 = a.block_map[3 * b + 1];
             const int rows = a.block_map[3 * b + 2];
             const int ncb = (rows + 31) >> 5;
-            const int buf = ucount & 1;
+            const int buf = ucount % C::kAccBufs;
+            const uint32_t use = ucount / C::kAccBufs;
             // per-column routing data for the down epilogue: lane holds columns lane + 32*i
-            int tk[4];
-            float wt[4];
+            int tk[kMaxCb];
+            float wt[kMaxCb];
             if (kDown) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < kMaxCb; ++i) {
                     const int c = lane + 32 * i;
                     tk[i] = 0;
                     wt[i] = 0.0f;
@@ -442,18 +468,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     }
                 }
             }
-            if (!mbar_wait(accfull(buf), (ucount >> 1) & 1, abort_flag)) {
+            if (!warp_wait(accfull(buf), use & 1, abort_flag)) {
                 fail(6);
                 break;
             }
             tc_fence_after();
-            const uint32_t tb = tmem + lane_base + buf * 256;
+            const uint32_t tb = tmem + lane_base + buf * C::kAccCols;
             if (!kDown) {
 #pragma unroll 1
                 for (int cb = 0; cb < ncb; ++cb) {
                     uint32_t g[32], uu[32];
                     tmem_ld32(tb + cb * 32, g);
-                    tmem_ld32(tb + 128 + cb * 32, uu);
+                    tmem_ld32(tb + kBlockT + cb * 32, uu);
                     tmem_ld_wait();
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
@@ -481,34 +507,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 // lane reduces 4 consecutive features of one token into y_acc
                 // with one 16-byte red, scaled by the token's routing weight.
                 float* stf = reinterpret_cast<float*>(stg);
+                const int m0 = j * 128 + q * 32;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int m0 = j * 256 + half * 128 + q * 32;
+                for (int cb = 0; cb < kMaxCb; ++cb) {
+                    if (cb < ncb) {
+                        uint32_t o[32];
+                        tmem_ld32(tb + cb * 32, o);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int cb = 0; cb < 4; ++cb) {
-                        if (cb < ncb) {
-                            uint32_t o[32];
-                            tmem_ld32(tb + half * 128 + cb * 32, o);
-                            tmem_ld_wait();
+                        for (int jj = 0; jj < 32; ++jj)
+                            stf[jj * kEpiRowFloats + lane] = __uint_as_float(o[jj]);
+                        __syncwarp();
 #pragma unroll
-                            for (int jj = 0; jj < 32; ++jj)
-                                stf[jj * kEpiRowFloats + lane] = __uint_as_float(o[jj]);
-                            __syncwarp();
-#pragma unroll
-                            for (int r = 0; r < 8; ++r) {
-                                const int c = 4 * r + (lane >> 3);
-                                const int fg = lane & 7;
-                                const int t = __shfl_sync(0xffffffffu, tk[cb], c);
-                                const float w = __shfl_sync(0xffffffffu, wt[cb], c);
-                                if (cb * 32 + c < rows) {
-                                    const float4 v = *reinterpret_cast<const float4*>(
-                                        stf + c * kEpiRowFloats + 4 * fg);
-                                    red_add_v4(a.y_acc + static_cast<size_t>(t) * a.out_ld + m0 + 4 * fg,
-                                               w * v.x, w * v.y, w * v.z, w * v.w);
-                                }
+                        for (int r = 0; r < 8; ++r) {
+                            const int c = 4 * r + (lane >> 3);
+                            const int fg = lane & 7;
+                            const int t = __shfl_sync(0xffffffffu, tk[cb], c);
+                            const float w = __shfl_sync(0xffffffffu, wt[cb], c);
+                            if (cb * 32 + c < rows) {
+                                const float4 v = *reinterpret_cast<const float4*>(
+                                    stf + c * kEpiRowFloats + 4 * fg);
+                                red_add_v4(a.y_acc + static_cast<size_t>(t) * a.out_ld + m0 + 4 * fg,
+                                           w * v.x, w * v.y, w * v.z, w * v.w);
                             }
-                            __syncwarp();
                         }
+                        __syncwarp();
                     }
                 }
             }
@@ -526,16 +549,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 }
 
 // One thread per (expert, tile, K chunk, packed row): writes 8 words of
-// nibbles and the row's (scale, bias) pairs of that chunk.
+// nibbles and the row's (scale, bias) pairs of that chunk.  A block holds
+// s.tiles tiles of 128 rows; packed row rr comes from tile rr / 128.
 __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t* __restrict__ out) {
     const int KC = s.K / kKChunk;
     const int gpc = kKChunk / group;
-    const int bb = packed_block_bytes(group);
-    const long total = static_cast<long>(E) * s.NT * KC * 256;
+    const int bb = packed_block_bytes(s.tiles, group);
+    const int rows = 128 * s.tiles;
+    const int nibble_bytes = rows * 32;
+    const long total = static_cast<long>(E) * s.NT * KC * rows;
     for (long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<long>(gridDim.x) * blockDim.x) {
-        const int rr = static_cast<int>(idx & 255);
-        long blk = idx >> 8;
+        const int rr = static_cast<int>(idx % rows);
+        long blk = idx / rows;
         const int c = static_cast<int>(blk % KC);
         blk /= KC;
         const int j = static_cast<int>(blk % s.NT);
@@ -567,7 +593,7 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
         for (int g = 0; g < gpc; ++g) {
             const uint32_t sv = ssrc[grow + g];
             const uint32_t bv = bsrc[grow + g];
-            *reinterpret_cast<uint32_t*>(dst + kNibbleBytes + (rr * gpc + g) * 4) = sv | (bv << 16);
+            *reinterpret_cast<uint32_t*>(dst + nibble_bytes + (rr * gpc + g) * 4) = sv | (bv << 16);
         }
     }
 }
@@ -590,10 +616,11 @@ __global__ void finalize_kernel(const float* __restrict__ y_acc, uint16_t* __res
 
 cudaError_t prepare_gemm_kernels() {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<false>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(grouped_gemm_kernel<true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    return cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<true>::kSmemBytes);
 }
 
 cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
@@ -620,7 +647,7 @@ cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t ro
 
 cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* out,
                            cudaStream_t st) {
-    const long total = static_cast<long>(E) * src.NT * (src.K / kKChunk) * 256;
+    const long total = static_cast<long>(E) * src.NT * (src.K / kKChunk) * 128 * src.tiles;
     const int threads = 256;
     const long blocks = (total + threads - 1) / threads;
     prepack_kernel<<<static_cast<int>(blocks < 65535 * 16 ? blocks : 65535 * 16), threads, 0, st>>>(
@@ -632,9 +659,9 @@ static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaSt
     if (a.max_units <= 0) return cudaSuccess;
     const int grid = a.max_units < num_sms ? a.max_units : num_sms;
     if (down)
-        grouped_gemm_kernel<true><<<grid, kGemmThreads, kSmemBytes, st>>>(a);
+        grouped_gemm_kernel<true><<<grid, kGemmThreads, Cfg<true>::kSmemBytes, st>>>(a);
     else
-        grouped_gemm_kernel<false><<<grid, kGemmThreads, kSmemBytes, st>>>(a);
+        grouped_gemm_kernel<false><<<grid, kGemmThreads, Cfg<false>::kSmemBytes, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -15,7 +15,8 @@ struct moe_plan {
     int block_t;
     int max_blocks;
     int ng_max;
-    int group_bytes;  // packed block bytes
+    int group_bytes;  // packed block bytes, gate/up (two tiles)
+    int down_block_bytes;  // packed block bytes, down (one tile)
     size_t gu_packed;  // bytes of the gate/up packed blocks
     size_t dn_packed;
     size_t packed_bytes;
@@ -30,14 +31,15 @@ namespace moe {
 constexpr int kMaxExperts = 256;  // experts per layer the routing kernels hold
 constexpr int kMaxTopk = 32;      // one warp lane per selected expert
 constexpr int kRouteGroupT = 256; // tokens per scatter group (one histogram row)
-constexpr int kBlockT = 128;      // block map tile height = largest MMA N
+constexpr int kBlockT = 256;      // block map tile height = largest MMA N
 constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
 
-// Packed weight block: two 128-row A tiles (A0 rows 0..127, A1 rows
-// 128..255) of one 64-wide K chunk: 256 rows x 32 bytes of nibbles, then per
-// row and group one (scale, bias) bf16 pair.
-__host__ __device__ constexpr int packed_block_bytes(int group) {
-    return 256 * 32 + 256 * (kKChunk / group) * 4;
+// Packed weight block: `tiles` 128-row A tiles of one 64-wide K chunk
+// (gate/up: the gate rows, then the up rows of 128 features; down: 128 rows):
+// 128*tiles rows x 32 bytes of nibbles, then per row and group one
+// (scale, bias) bf16 pair.
+__host__ __device__ constexpr int packed_block_bytes(int tiles, int group) {
+    return 128 * tiles * 32 + 128 * tiles * (kKChunk / group) * 4;
 }
 
 // ---- routing (moe_route.cu) ----
@@ -67,7 +69,8 @@ struct PrepackSource {
     int K;               // reduction length
     int row_step;        // source row of tile j, row r: j*row_step + r (A0), + a1_off (A1)
     int a1_off;
-    int NT;              // tiles per expert
+    int NT;              // output tiles per expert
+    int tiles;           // 128-row A tiles per packed block (1 or 2)
 };
 cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* out,
                            cudaStream_t st);

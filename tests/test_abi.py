@@ -50,8 +50,8 @@ def test_plan_sizes(moe, shape):
     T, d, E, k, f, G = shape
     p = moe.Plan(*shape)
     info = p.info
-    assert info.block_t == 128
-    assert info.max_blocks == -(-T * k // 128) + min(E, T * k)
+    assert info.block_t == 256
+    assert info.max_blocks == -(-T * k // 256) + min(E, T * k)
     logical = 3 * E * f * d // 2 + 3 * E * f * (d // G) * 4
     assert logical <= info.packed_weight_bytes <= logical + 256
     need = T * k * f * 2 + T * d * 4  # h and the fp32 combine accumulator at least

@@ -33,7 +33,7 @@ def moe():
     return m
 
 
-def oracle_route(inp, T=None, block_t=128):
+def oracle_route(inp, T=None, block_t=256):
     x = inp.x if T is None else inp.x[:T]
     logits = oracle.router_logits(x, inp.w_r, inp.b_r)
     idx = oracle.topk(logits, inp.shape.k)
