@@ -35,7 +35,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer prefill tokens/s (int4 fused grouped GEMM) and % of roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
-KERNELS_PER_STEP = 7  # logits, top-k, scan, scatter, gate/up GEMM, down GEMM, finalize
+KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, down GEMM, combine
 
 
 def load_peaks():
@@ -243,10 +243,10 @@ def run_ours(args, name):
     clk = clocks.stop()
     step_ms = [r[0].elapsed_time(r[4]) for r in evs]
     stage_ms = {
-        "routing": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
+        "routing_and_dispatch": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
         "gate_up_gemm": float(np.mean([r[1].elapsed_time(r[2]) for r in evs])),
         "down_gemm": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
-        "finalize": float(np.mean([r[3].elapsed_time(r[4]) for r in evs])),
+        "combine": float(np.mean([r[3].elapsed_time(r[4]) for r in evs])),
     }
     total_ms = float(sum(step_ms))
     if world > 1:

@@ -180,7 +180,9 @@ MOE_API moe_status_t moe_route(const moe_plan_t *plan, int32_t T, const uint16_t
  *   route_out: NULL, or buffers that receive the routing results.
  * Rounding: x is bf16, weights are expanded to bf16 (one rounding of
  * nibble*scale+bias), products accumulate in fp32, the SwiGLU output is
- * rounded to bf16 before the down projection, y is rounded to bf16.
+ * rounded to bf16 before the down projection, each expert's down output is
+ * rounded to bf16, the k weighted outputs of a token are summed in fp32 in
+ * slot order j = 0..k-1 and y is rounded to bf16.
  */
 MOE_API moe_status_t moe_forward(const moe_plan_t *plan, int32_t T, const uint16_t *x,
                          const float *W_r, const float *b_r,
@@ -194,11 +196,12 @@ MOE_API moe_status_t moe_forward(const moe_plan_t *plan, int32_t T, const uint16
  * Any field may be NULL.
  */
 typedef struct moe_stage_events {
-    void *start;   /* before the routing kernels                       */
-    void *routed;  /* after top-k, prefix scan, scatter and block map  */
-    void *gate_up; /* after the gate/up grouped GEMM (SwiGLU fused)    */
-    void *down;    /* after the down grouped GEMM (combine fused)      */
-    void *end;     /* after the final bf16 conversion of y             */
+    void *start;   /* before the routing kernels                         */
+    void *routed;  /* after top-k, prefix scan, scatter, block map and
+                      the copy of the token rows into expert order       */
+    void *gate_up; /* after the gate/up grouped GEMM (SwiGLU fused)      */
+    void *down;    /* after the down grouped GEMM                        */
+    void *end;     /* after the routing-weighted combine into y          */
 } moe_stage_events_t;
 
 /* moe_forward, also recording *events (may be NULL) between the stages. */

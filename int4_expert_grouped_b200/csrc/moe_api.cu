@@ -97,10 +97,9 @@ moe_status_t check_route_out(const moe_route_out_t* o) {
         if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
     } while (0)
 
-// Steps 1-4 (routing).  y_acc, when given, is zeroed for the T tokens.
+// Steps 1-4 (routing).
 moe_status_t run_route(const moe_plan* p, int T, const uint16_t* x, const float* W_r,
-                       const float* b_r, const RoutePtrs& r, void* ws, float* y_acc,
-                       cudaStream_t st) {
+                       const float* b_r, const RoutePtrs& r, void* ws, cudaStream_t st) {
     const moe_shape_t& s = p->s;
     int32_t* status = at<int32_t>(ws, p->o_status);
     int32_t* hist = at<int32_t>(ws, p->o_hist);
@@ -108,7 +107,7 @@ moe_status_t run_route(const moe_plan* p, int T, const uint16_t* x, const float*
     MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, at<float>(ws, p->o_logits), T, s.d, s.E, hist,
                                        std::max(ng, 1) * s.E, status, st));
     MOE_CUDA(moe::launch_router_topk(at<float>(ws, p->o_logits), T, s.E, s.k, r.idx, r.w, hist,
-                                     y_acc, s.d, st));
+                                     st));
     MOE_CUDA(moe::launch_route_scan(hist, ng, s.E, p->block_t, r.counts, r.offsets,
                                     at<int32_t>(ws, p->o_gbase), r.bo, r.bm, r.nb, p->max_blocks,
                                     status, st));
@@ -181,8 +180,8 @@ moe_status_t moe_plan_create(const moe_shape_t* shape, moe_plan_t** plan, moe_pl
     p->o_sa = take(T * k * 4);
     p->o_pos = take(T * k * 4);
     p->o_bm = take(static_cast<size_t>(p->max_blocks) * 12);
+    p->o_xs = take(T * k * s.d * 2);  // x rows in expert order, later the down outputs o
     p->o_h = take(T * k * s.f * 2);
-    p->o_yacc = take(T * s.d * 4);
     p->ws_bytes = o;
     p->o_xstage = take(T * s.d * 2);
     p->o_ystage = take(T * s.d * 2);
@@ -240,7 +239,7 @@ moe_status_t moe_route(const moe_plan_t* plan, int32_t T, const uint16_t* x, con
     if (!aligned16(ws) || !aligned16(W_r) || (x && !aligned16(x)) || (b_r && !aligned16(b_r)))
         return MOE_ERR_ALIGNMENT;
     if (ws_bytes < plan->ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    return run_route(plan, T, x, W_r, b_r, route_ptrs(plan, ws, out), ws, nullptr,
+    return run_route(plan, T, x, W_r, b_r, route_ptrs(plan, ws, out), ws,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -275,54 +274,55 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     const moe_shape_t& s = plan->s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RoutePtrs r = route_ptrs(plan, ws, route_out);
-    float* y_acc = at<float>(ws, plan->o_yacc);
+    uint16_t* xs = at<uint16_t>(ws, plan->o_xs);
     uint16_t* h = at<uint16_t>(ws, plan->o_h);
     int32_t* status = at<int32_t>(ws, plan->o_status);
     auto mark = [&](void* e) -> bool {
         return e == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(e), st) == cudaSuccess;
     };
     if (ev && !mark(ev->start)) return MOE_ERR_CUDA;
-    moe_status_t rs = run_route(plan, T, x, W_r, b_r, r, ws, y_acc, st);
+    moe_status_t rs = run_route(plan, T, x, W_r, b_r, r, ws, st);
     if (rs != MOE_OK) return rs;
-    if (ev && !mark(ev->routed)) return MOE_ERR_CUDA;
     if (T == 0) {
-        if (ev && !(mark(ev->gate_up) && mark(ev->down) && mark(ev->end))) return MOE_ERR_CUDA;
+        if (ev && !(mark(ev->routed) && mark(ev->gate_up) && mark(ev->down) && mark(ev->end)))
+            return MOE_ERR_CUDA;
         return MOE_OK;
     }
+    const int Tk = T * s.k;
+    // step 5 (dispatch): token rows into expert order
+    MOE_CUDA(moe::launch_dispatch(x, r.sa, Tk, s.k, s.d, xs, status, num_sms, st));
+    if (ev && !mark(ev->routed)) return MOE_ERR_CUDA;
 
     const int mb = max_blocks_for(s, T);
     const uint8_t* wp = static_cast<const uint8_t*>(packed_w);
     moe::GemmArgs g{};
     g.wpack = wp;
-    g.act = x;
-    g.sorted_assign = r.sa;
     g.block_map = r.bm;
     g.num_blocks = r.nb;
-    g.topk_w = r.w;
-    g.h_out = h;
-    g.y_acc = y_acc;
+    g.out = h;
     g.status = status;
     g.K = s.d;
     g.NT = s.f / 128;
     g.out_ld = s.f;
-    g.topk = s.k;
     g.group = s.group;
     g.block_bytes = plan->group_bytes;
     g.max_units = mb * g.NT;
+    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
     if (ev && !mark(ev->gate_up)) return MOE_ERR_CUDA;
 
+    // the down outputs o reuse the storage of xs, which gate/up has finished reading
     g.wpack = wp + align_up(plan->gu_packed, 256);
-    g.act = h;
+    g.out = xs;
     g.K = s.f;
     g.NT = s.d / 128;
     g.out_ld = s.d;
     g.block_bytes = plan->down_block_bytes;
     g.max_units = mb * g.NT;
-    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(T) * s.k, s.f, moe::kBlockT));
+    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;
-    MOE_CUDA(moe::launch_finalize(y_acc, y, static_cast<long>(T) * s.d, st));
+    MOE_CUDA(moe::launch_combine(xs, r.pos, r.w, T, s.k, s.d, y, status, num_sms, st));
     if (ev && !mark(ev->end)) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -6,11 +6,12 @@
 //   prepack_kernel        logical nibbles/scales -> per (expert, tile, K chunk)
 //                         contiguous blocks in the order the GEMM reads them
 //   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
-//       gate/up: D0 = Wg x^T, D1 = Wu x^T over gathered token rows, epilogue
-//                h = silu(D0) * D1 -> bf16 h rows in expert order
-//       down:    D = 128-row tile of Wd times h^T, epilogue
-//                y_acc[t] += topk_w * D (fp32 reduction in L2)
-//   finalize_kernel       y = bf16(y_acc)
+//       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order,
+//                epilogue h = silu(D0) * D1 -> bf16 h rows
+//       down:    D = 128-row tile of Wd times h^T, epilogue o = bf16(D) rows
+//                (the routing-weighted sum over a token's experts is a
+//                separate pass, so no output element is ever accumulated by
+//                two CTAs)
 //
 // One work unit = one block-map tile (<= 256 expert-ordered rows of one
 // expert) x one output tile of 128 features (gate/up: the gate and the up
@@ -28,12 +29,11 @@
 //   warp 0       bulk-copies packed weight blocks into the W ring (TMA engine)
 //   warp 1       allocates TMEM; runs the MMA loop, one elected lane issues
 //                tcgen05.mma and tcgen05.commit
-//   warps 2-3    gate/up: gather x rows by token index into the B ring
-//                (cp.async, 128B swizzle); down: warp 2 loads 2-D TMA tiles of
-//                h, warp 3 is idle
+//   warp 2       loads 2-D TMA tiles of the token rows (xs or h) into the
+//                B ring (128-byte swizzle); warp 3 has no role
 //   warps 4-11   expand int4 -> bf16 from the W ring into the A ring, in two
 //                groups that take alternate K chunks
-//   warps 12-15  epilogue: TMEM -> registers -> h rows / y_acc reductions
+//   warps 12-15  epilogue: TMEM -> registers -> bf16 rows of h or o
 // TMEM: gate/up holds one buffer of 2 x 256 columns (gate, up), so its
 // epilogue runs between units; down holds two buffers of 256 columns, so its
 // epilogue overlaps the next unit's main loop.
@@ -46,9 +46,8 @@ namespace {
 
 constexpr int kWarpWProducer = 0;
 constexpr int kWarpMma = 1;
-constexpr int kWarpLoader = 2;   // down: TMA tiles; gate/up: warps 2-3 gather with cp.async
-constexpr int kWarpIdle = 3;     // down only: no role
-constexpr int kGatherThreads = 64;    // gate/up gather warps 2-3
+constexpr int kWarpLoader = 2;
+constexpr int kWarpIdle = 3;     // no role
 constexpr int kTransformGroups = 2;   // transform warp groups, alternate chunks
 constexpr int kWarpTransform0 = 4;
 constexpr int kNumTransformWarps = 8;
@@ -59,8 +58,7 @@ constexpr int kTransformThreads = kNumTransformWarps * 32;
 constexpr int kGroupThreads = kTransformThreads / kTransformGroups;
 constexpr int kATileBytes = 128 * 128;     // 128 rows x 64 bf16 (128B swizzle)
 constexpr int kBStageBytes = kBlockT * 128;  // up to 256 token rows x 64 bf16
-constexpr int kEpiRowBytes = 80;    // gate/up staging row: 32 bf16 + 16 bytes of padding
-constexpr int kEpiRowFloats = 36;   // down staging row: 32 fp32 + 4 of padding
+constexpr int kEpiRowBytes = 80;    // staging row: 32 bf16 + 16 bytes of padding
 constexpr uint32_t kTmemCols = 512;
 
 // Per-projection configuration.
@@ -75,7 +73,7 @@ struct Cfg {
     static constexpr int kAStageBytes = kTiles * kATileBytes;
     static constexpr int kWStageBytes = packed_block_bytes(kTiles, 32);  // largest (group 32)
     static constexpr int kNibbleBytes = kTiles * 128 * 32;
-    static constexpr int kEpiWarpBytes = kDown ? 32 * kEpiRowFloats * 4 : 32 * kEpiRowBytes;
+    static constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
     static constexpr int kTasks = kTiles * 256 / kGroupThreads;  // (row, half) tasks per thread
 
     static constexpr int kOffA = 0;
@@ -139,13 +137,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
-// y[0..3] += v (fp32, one 16-byte reduction in L2)
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a),
-                 "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-
 // mbar_wait for a whole converged warp: every lane waits and the outcome is
 // voted, so the warp takes the same branch whatever happens at a timeout.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -197,7 +188,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             mbar_init(aempty(s), 1);
         }
         for (int s = 0; s < C::kNB; ++s) {
-            mbar_init(bfull(s), kDown ? 1 : kGatherThreads);
+            mbar_init(bfull(s), 1);
             mbar_init(bempty(s), 1);
         }
         for (int s = 0; s < C::kAccBufs; ++s) {
@@ -322,10 +313,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             __syncwarp();
             mbar_wait_drain(drain_bar, 0);
         }
-    } else if (kDown && warp == kWarpLoader) {
-        // down: one 256-row TMA tile of h per stage (rows past the block belong
-        // to the next expert or lie past the end and are zero-filled; the MMA
-        // ignores columns >= N)
+    } else if (warp == kWarpLoader) {
+        // one 2-D TMA tile of kBlockT token rows per stage (rows past the block
+        // belong to the next expert or lie past the end and are zero-filled;
+        // the MMA ignores columns >= N and the epilogue columns >= rows)
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
@@ -344,50 +335,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 __syncwarp();
             }
         }
-    } else if (!kDown && (warp == kWarpLoader || warp == kWarpLoader + 1)) {
-        // gate/up: gather x rows by token index with 16-byte cp.async.  Lane
-        // layout: 8 consecutive lanes copy the 8 pieces of one 128-byte row, so a
-        // warp instruction reads 4 whole rows; thread ltid (0..63) copies piece
-        // ltid % 8 of rows ltid/8 + 8*jr.  Completion is signalled
-        // asynchronously (cp.async.mbarrier.arrive.noinc), so no thread waits
-        // for its copies.
-        const int ltid = threadIdx.x - kWarpLoader * 32;
-        const int piece = ltid & 7;
-        const int rbase = ltid >> 3;
-        constexpr int kRowsPerThread = kBlockT / (kGatherThreads / 8);
-        const uint32_t swz = static_cast<uint32_t>((piece ^ rbase) << 4);  // row & 7 == rbase
-        uint32_t it = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-            const int b = u / NT;
-            const int row0 = a.block_map[3 * b + 1];
-            const int rows = a.block_map[3 * b + 2];
-            const int N = (rows + 15) & ~15;
-            uint32_t off[kRowsPerThread];  // element offset of the source row piece
-#pragma unroll
-            for (int jr = 0; jr < kRowsPerThread; ++jr) {
-                const int r = rbase + 8 * jr;
-                const int t = r < rows ? a.sorted_assign[row0 + r] / a.topk : 0;
-                off[jr] = static_cast<uint32_t>(t) * static_cast<uint32_t>(a.K) + piece * 8;
-            }
-            for (int c = 0; c < KC; ++c, ++it) {
-                const int s = it % C::kNB;
-                if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
-                    fail(4);
-                    ok = false;
-                    break;
-                }
-                const uint32_t dst = sbase + C::kOffB + s * kBStageBytes + swz;
-#pragma unroll
-                for (int jr = 0; jr < kRowsPerThread; ++jr) {
-                    const int r = rbase + 8 * jr;
-                    if (r < N)
-                        cp_async_16(dst + r * 128, a.act + off[jr] + c * kKChunk, r < rows ? 16u : 0u);
-                }
-                cp_async_arrive_noinc(bfull(s));
-            }
+        if (!ok && lane == 0) {
+            const uint32_t first = it > C::kNB ? it - C::kNB : 0;
+            for (uint32_t i = first; i < it; ++i)
+                mbar_wait_drain(bfull(i % C::kNB), (i / C::kNB) & 1);
         }
-        cp_async_wait_all();
     } else if (warp >= kWarpTransform0 && warp < kWarpTransform0 + kNumTransformWarps) {
         // Two groups of transform warps take alternate chunks, so each warp
         // pays one round of barrier waits per two chunks.
@@ -438,11 +390,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             }
         }
     } else if (warp >= kWarpEpi0) {
-        // epilogue warps: warp % 4 selects the TMEM lane quadrant
+        // epilogue warps: warp % 4 selects the TMEM lane quadrant, i.e. the
+        // 32 output features q*32 .. q*32+31 of the tile.  D[feature][token]
+        // goes through a staging tile [token][feature] so that each lane then
+        // writes 64 contiguous bytes of one token row.
         const int q = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint8_t* stg = smem + C::kOffEpi + (warp - kWarpEpi0) * C::kEpiWarpBytes;
-        constexpr int kMaxCb = kBlockT / 32;
         uint32_t ucount = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++ucount) {
             const int b = u / NT;
@@ -452,88 +406,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int ncb = (rows + 31) >> 5;
             const int buf = ucount % C::kAccBufs;
             const uint32_t use = ucount / C::kAccBufs;
-            // per-column routing data for the down epilogue: lane holds columns lane + 32*i
-            int tk[kMaxCb];
-            float wt[kMaxCb];
-            if (kDown) {
-#pragma unroll
-                for (int i = 0; i < kMaxCb; ++i) {
-                    const int c = lane + 32 * i;
-                    tk[i] = 0;
-                    wt[i] = 0.0f;
-                    if (c < rows) {
-                        const int asg = a.sorted_assign[row0 + c];
-                        tk[i] = asg / a.topk;
-                        wt[i] = a.topk_w[asg];
-                    }
-                }
-            }
             if (!warp_wait(accfull(buf), use & 1, abort_flag)) {
                 fail(6);
                 break;
             }
             tc_fence_after();
             const uint32_t tb = tmem + lane_base + buf * C::kAccCols;
-            if (!kDown) {
 #pragma unroll 1
-                for (int cb = 0; cb < ncb; ++cb) {
-                    uint32_t g[32], uu[32];
-                    tmem_ld32(tb + cb * 32, g);
+            for (int cb = 0; cb < ncb; ++cb) {
+                uint32_t v[32];
+                tmem_ld32(tb + cb * 32, v);
+                if constexpr (kDown) {
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        *reinterpret_cast<__nv_bfloat16*>(stg + jj * kEpiRowBytes + lane * 2) =
+                            __float2bfloat16_rn(__uint_as_float(v[jj]));
+                } else {
+                    uint32_t uu[32];
                     tmem_ld32(tb + kBlockT + cb * 32, uu);
                     tmem_ld_wait();
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
-                        const float gv = __uint_as_float(g[jj]);
+                        const float gv = __uint_as_float(v[jj]);
                         const float uv = __uint_as_float(uu[jj]);
                         const float hv = __fdividef(gv * uv, 1.0f + __expf(-gv));
                         *reinterpret_cast<__nv_bfloat16*>(stg + jj * kEpiRowBytes + lane * 2) =
                             __float2bfloat16_rn(hv);
                     }
-                    __syncwarp();
-                    const int c = cb * 32 + lane;
-                    if (c < rows) {
-                        const uint4* s4 = reinterpret_cast<const uint4*>(stg + lane * kEpiRowBytes);
-                        uint4* d4 = reinterpret_cast<uint4*>(
-                            a.h_out + static_cast<size_t>(row0 + c) * a.out_ld + j * 128 + q * 32);
-                        d4[0] = s4[0];
-                        d4[1] = s4[1];
-                        d4[2] = s4[2];
-                        d4[3] = s4[3];
-                    }
-                    __syncwarp();
                 }
-            } else {
-                // D[feature][token] -> staging [token][feature] (fp32), then each
-                // lane reduces 4 consecutive features of one token into y_acc
-                // with one 16-byte red, scaled by the token's routing weight.
-                float* stf = reinterpret_cast<float*>(stg);
-                const int m0 = j * 128 + q * 32;
-#pragma unroll
-                for (int cb = 0; cb < kMaxCb; ++cb) {
-                    if (cb < ncb) {
-                        uint32_t o[32];
-                        tmem_ld32(tb + cb * 32, o);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            stf[jj * kEpiRowFloats + lane] = __uint_as_float(o[jj]);
-                        __syncwarp();
-#pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            const int c = 4 * r + (lane >> 3);
-                            const int fg = lane & 7;
-                            const int t = __shfl_sync(0xffffffffu, tk[cb], c);
-                            const float w = __shfl_sync(0xffffffffu, wt[cb], c);
-                            if (cb * 32 + c < rows) {
-                                const float4 v = *reinterpret_cast<const float4*>(
-                                    stf + c * kEpiRowFloats + 4 * fg);
-                                red_add_v4(a.y_acc + static_cast<size_t>(t) * a.out_ld + m0 + 4 * fg,
-                                           w * v.x, w * v.y, w * v.z, w * v.w);
-                            }
-                        }
-                        __syncwarp();
-                    }
+                __syncwarp();
+                const int c = cb * 32 + lane;
+                if (c < rows) {
+                    const uint4* s4 = reinterpret_cast<const uint4*>(stg + lane * kEpiRowBytes);
+                    uint4* d4 = reinterpret_cast<uint4*>(
+                        a.out + static_cast<size_t>(row0 + c) * a.out_ld + j * 128 + q * 32);
+                    d4[0] = s4[0];
+                    d4[1] = s4[1];
+                    d4[2] = s4[2];
+                    d4[3] = s4[3];
                 }
+                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
@@ -598,20 +511,6 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
     }
 }
 
-__global__ void finalize_kernel(const float* __restrict__ y_acc, uint16_t* __restrict__ y, long n) {
-    for (long i = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < n;
-         i += static_cast<long>(gridDim.x) * blockDim.x * 8) {
-        const float4 v0 = *reinterpret_cast<const float4*>(y_acc + i);
-        const float4 v1 = *reinterpret_cast<const float4*>(y_acc + i + 4);
-        BF2 p0, p1, p2, p3;
-        p0.h = __floats2bfloat162_rn(v0.x, v0.y);
-        p1.h = __floats2bfloat162_rn(v0.z, v0.w);
-        p2.h = __floats2bfloat162_rn(v1.x, v1.y);
-        p3.h = __floats2bfloat162_rn(v1.z, v1.w);
-        *reinterpret_cast<uint4*>(y + i) = make_uint4(p0.u, p1.u, p2.u, p3.u);
-    }
-}
-
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
@@ -671,15 +570,6 @@ cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st) 
 
 cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st) {
     return launch_gemm(a, num_sms, true, st);
-}
-
-cudaError_t launch_finalize(const float* y_acc, uint16_t* y, long n, cudaStream_t st) {
-    if (n <= 0) return cudaSuccess;
-    const int threads = 256;
-    long blocks = (n / 8 + threads - 1) / threads;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    finalize_kernel<<<static_cast<int>(blocks), threads, 0, st>>>(y_acc, y, n);
-    return cudaGetLastError();
 }
 
 }  // namespace moe

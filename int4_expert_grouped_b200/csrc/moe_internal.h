@@ -22,7 +22,7 @@ struct moe_plan {
     size_t packed_bytes;
     // workspace offsets
     size_t o_status, o_logits, o_hist, o_gbase, o_idx, o_w, o_counts, o_offsets, o_bo, o_nb,
-        o_sa, o_pos, o_bm, o_h, o_yacc, ws_bytes;
+        o_sa, o_pos, o_bm, o_xs, o_h, ws_bytes;
     size_t o_xstage, o_ystage, host_ws_bytes;
 };
 
@@ -47,8 +47,7 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float*
                                  int T, int d, int E, int32_t* hist, int hist_n, int32_t* status,
                                  cudaStream_t st);
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
-                               float* topk_w, int32_t* hist, float* y_acc, int d,
-                               cudaStream_t st);
+                               float* topk_w, int32_t* hist, cudaStream_t st);
 cudaError_t launch_route_scan(const int32_t* hist, int ng, int E, int BT, int32_t* counts,
                               int32_t* offsets, int32_t* gbase, int32_t* block_offsets,
                               int32_t* block_map, int32_t* num_blocks, int max_blocks,
@@ -76,23 +75,18 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
                            cudaStream_t st);
 
 struct GemmArgs {
-    // B operand (token rows) for TMA: gate/up gathers rows of x [T, d] four at
-    // a time (box 64 x 1); down reads h [T*k, f] tiles (box 64 x 128).  Both use
-    // the 128-byte swizzle, which is the K-major layout the MMA reads.
+    // B operand (token rows in expert order) for 2-D TMA tiles of 64 columns x
+    // kBlockT rows with the 128-byte swizzle, the K-major layout the MMA
+    // reads: gate/up reads xs [T*k, d], down reads h [T*k, f].
     CUtensorMap bmap;
     const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
-    const uint16_t* act;           // B rows: x [T, d] (gate/up) or h [T*k, f] (down)
-    const int32_t* sorted_assign;  // [T*k]
     const int32_t* block_map;      // [num_blocks, 3]
     const int32_t* num_blocks;     // [1], device
-    const float* topk_w;           // [T*k] by assignment (down)
-    uint16_t* h_out;               // [T*k, f] (gate/up)
-    float* y_acc;                  // [T, d] fp32 (down)
+    uint16_t* out;                 // h [T*k, f] (gate/up) or o [T*k, d] (down), bf16
     int32_t* status;
     int K;                         // reduction length
-    int NT;                        // output tile pairs per expert
+    int NT;                        // output tiles of 128 features per expert
     int out_ld;                    // f (gate/up) or d (down)
-    int topk;
     int group;
     int block_bytes;
     int max_units;                 // upper bound of num_blocks * NT
@@ -103,7 +97,15 @@ cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t ro
                                  uint32_t box_rows);
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st);
-cudaError_t launch_finalize(const float* y_acc, uint16_t* y, long n, cudaStream_t st);
 cudaError_t prepare_gemm_kernels();
+
+// ---- dispatch and combine (moe_combine.cu) ----
+// xs[p] = x[sorted_assign[p] / k] for p < T*k
+cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
+                            uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st);
+// y[t] = bf16(sum_i topk_w[t*k+i] * o[pos[t*k+i]])
+cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T,
+                           int k, int d, uint16_t* y, int32_t* status, int num_sms,
+                           cudaStream_t st);
 
 }  // namespace moe

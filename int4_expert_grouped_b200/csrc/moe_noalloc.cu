@@ -103,8 +103,8 @@ extern "C" MOE_API moe_status_t moe_route_noalloc(const moe_plan_t* plan, int32_
     if (moe::launch_router_logits(x, W_r, b_r, logits, T, s.d, s.E, hist,
                                   static_cast<int>(hist_n), status, cs) != cudaSuccess)
         return MOE_ERR_CUDA;
-    if (moe::launch_router_topk(logits, T, s.E, s.k, out->topk_idx, out->topk_w, hist, nullptr,
-                                s.d, cs) != cudaSuccess)
+    if (moe::launch_router_topk(logits, T, s.E, s.k, out->topk_idx, out->topk_w, hist, cs) !=
+        cudaSuccess)
         return MOE_ERR_CUDA;
     if (moe::launch_route_scan(hist, ng, s.E, plan->block_t, out->counts, out->offsets, gbase,
                                out->block_offsets, out->block_map, out->num_blocks,

@@ -4,7 +4,7 @@
 // host round trip):
 //   router_logits_kernel  fp32 logits in the fixed chain-and-butterfly order
 //   router_topk_kernel    top-k (ties to the lower id), softmax weights,
-//                         per-group expert histograms, zeroing of y_acc
+//                         per-group expert histograms
 //   route_scan_kernel     counts, prefix offsets, per-group scatter bases,
 //                         block map
 //   route_scatter_kernel  stable scatter into expert order (sorted_assign,
@@ -279,8 +279,7 @@ router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restric
 // selected logits, w_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0), with the sum
 // taken in a fixed butterfly order.  Each selected expert adds one to the
 // histogram of the token's group of kRouteGroupT tokens (integer atomics, so
-// the counts do not depend on their order).  The warp also zeroes row t of
-// the fp32 combine accumulator y_acc (when given).
+// the counts do not depend on their order).
 // ---------------------------------------------------------------------------
 constexpr int kTopkWarps = 8;
 
@@ -299,7 +298,7 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
 __global__ void __launch_bounds__(kTopkWarps * 32)
 router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                   int32_t* __restrict__ hist, float* __restrict__ y_acc, int d) {
+                   int32_t* __restrict__ hist) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int t = blockIdx.x * kTopkWarps + warp;
@@ -350,10 +349,6 @@ router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
         topk_idx[static_cast<size_t>(t) * k + lane] = my_id;
         topk_w[static_cast<size_t>(t) * k + lane] = __fdiv_rn(ex, sum);
         atomicAdd(hist + static_cast<size_t>(t / kRouteGroupT) * E + my_id, 1);
-    }
-    if (y_acc != nullptr) {
-        float4* row = reinterpret_cast<float4*>(y_acc + static_cast<size_t>(t) * d);
-        for (int i = lane; i < (d >> 2); i += 32) row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
@@ -585,12 +580,10 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float*
 }
 
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
-                               float* topk_w, int32_t* hist, float* y_acc, int d,
-                               cudaStream_t st) {
+                               float* topk_w, int32_t* hist, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int grid = (T + kTopkWarps - 1) / kTopkWarps;
-    router_topk_kernel<<<grid, kTopkWarps * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_w, hist,
-                                                         y_acc, d);
+    router_topk_kernel<<<grid, kTopkWarps * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_w, hist);
     return cudaGetLastError();
 }
 
