@@ -362,24 +362,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 }
                 const uint8_t* wst = smem + C::kOffW + sw * C::kWStageBytes;
                 const uint32_t ast = sbase + C::kOffA + sa * C::kAStageBytes;
+                // Task rep of this thread: packed row (gtid + kGroupThreads*rep) / 2
+                // (tile row >> 7, row & 127 within it), K half gtid & 1.  All
+                // loads of the chunk are issued before the first store so their
+                // latencies overlap.
+                const int half = gtid & 1;       // K 0..31 or 32..63 of the chunk
+                const int g = half * (gpc - 1);  // group 64: 0; group 32: half
+                uint4 pk[C::kTasks];
+                uint32_t sb[C::kTasks];
 #pragma unroll
                 for (int rep = 0; rep < C::kTasks; ++rep) {
-                    const int task = gtid + kGroupThreads * rep;
-                    const int row = task >> 1;  // packed row: tile row>>7, row & 127 within it
-                    const int half = task & 1;  // K 0..31 or 32..63 of the chunk
-                    const uint4 pk = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
-                    const int g = half * (gpc - 1);  // group 64: 0; group 32: half
-                    const uint32_t sb = *reinterpret_cast<const uint32_t*>(
-                        wst + C::kNibbleBytes + (row * gpc + g) * 4);
+                    const int row = (gtid + kGroupThreads * rep) >> 1;
+                    pk[rep] = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
+                    sb[rep] = *reinterpret_cast<const uint32_t*>(wst + C::kNibbleBytes +
+                                                                 (row * gpc + g) * 4);
+                }
+#pragma unroll
+                for (int rep = 0; rep < C::kTasks; ++rep) {
+                    const int row = (gtid + kGroupThreads * rep) >> 1;
                     BF2 s2, b2;
-                    s2.u = __byte_perm(sb, 0, 0x1010);
-                    b2.u = __byte_perm(sb, 0, 0x3232);
+                    s2.u = __byte_perm(sb[rep], 0, 0x1010);
+                    b2.u = __byte_perm(sb[rep], 0, 0x3232);
                     const uint32_t arow = ast + (row >> 7) * kATileBytes + (row & 127) * 128;
                     const int rsw = row & 7;
-                    st_shared_v4(arow + (((half * 4 + 0) ^ rsw) << 4), expand8(pk.x, s2.h, b2.h));
-                    st_shared_v4(arow + (((half * 4 + 1) ^ rsw) << 4), expand8(pk.y, s2.h, b2.h));
-                    st_shared_v4(arow + (((half * 4 + 2) ^ rsw) << 4), expand8(pk.z, s2.h, b2.h));
-                    st_shared_v4(arow + (((half * 4 + 3) ^ rsw) << 4), expand8(pk.w, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 0) ^ rsw) << 4), expand8(pk[rep].x, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 1) ^ rsw) << 4), expand8(pk[rep].y, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 2) ^ rsw) << 4), expand8(pk[rep].z, s2.h, b2.h));
+                    st_shared_v4(arow + (((half * 4 + 3) ^ rsw) << 4), expand8(pk[rep].w, s2.h, b2.h));
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -390,13 +399,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             }
         }
     } else if (warp >= kWarpEpi0) {
-        // epilogue warps: warp % 4 selects the TMEM lane quadrant, i.e. the
-        // 32 output features q*32 .. q*32+31 of the tile.  D[feature][token]
-        // goes through a staging tile [token][feature] so that each lane then
-        // writes 64 contiguous bytes of one token row.
+        // Epilogue warps: warp % 4 selects the TMEM lane quadrant, i.e. output
+        // features q*32 .. q*32+31 of the tile; the accumulator is
+        // D[feature][token].  Per block of 32 tokens the warp reads two 16-lane
+        // halves in the m16n8 fragment layout, rounds pairs of neighbouring
+        // tokens to bf16x2, and writes them transposed with stmatrix into a
+        // staging tile [token][32 features]; each lane then copies one
+        // token's 64 bytes to global memory.
         const int q = warp & 3;
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        uint8_t* stg = smem + C::kOffEpi + (warp - kWarpEpi0) * C::kEpiWarpBytes;
+        const uint32_t stg = sbase + C::kOffEpi + (warp - kWarpEpi0) * C::kEpiWarpBytes;
+        // stmatrix row address of this thread: matrix m = lane / 8 is the
+        // feature octet (16 bytes), row c = lane % 8 the token within a group of 8
+        const uint32_t st_addr = stg + (lane & 7) * kEpiRowBytes + (lane >> 3) * 16;
         uint32_t ucount = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++ucount) {
             const int b = u / NT;
@@ -411,34 +425,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 break;
             }
             tc_fence_after();
-            const uint32_t tb = tmem + lane_base + buf * C::kAccCols;
+            const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
 #pragma unroll 1
             for (int cb = 0; cb < ncb; ++cb) {
-                uint32_t v[32];
-                tmem_ld32(tb + cb * 32, v);
-                if constexpr (kDown) {
-                    tmem_ld_wait();
+                // p[h][i]: lane half h (features 16h + t/4 (+8)), register i
+                uint32_t p[2][8];
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        *reinterpret_cast<__nv_bfloat16*>(stg + jj * kEpiRowBytes + lane * 2) =
-                            __float2bfloat16_rn(__uint_as_float(v[jj]));
-                } else {
-                    uint32_t uu[32];
-                    tmem_ld32(tb + kBlockT + cb * 32, uu);
-                    tmem_ld_wait();
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t v[16];
+                    const uint32_t ta = tb + (static_cast<uint32_t>(16 * h) << 16) + cb * 32;
+                    tmem_ld_16x256b_x4(ta, v);
+                    if constexpr (kDown) {
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const float gv = __uint_as_float(v[jj]);
-                        const float uv = __uint_as_float(uu[jj]);
-                        const float hv = __fdividef(gv * uv, 1.0f + __expf(-gv));
-                        *reinterpret_cast<__nv_bfloat16*>(stg + jj * kEpiRowBytes + lane * 2) =
-                            __float2bfloat16_rn(hv);
+                        for (int i = 0; i < 8; ++i) {
+                            BF2 o;
+                            o.h = __floats2bfloat162_rn(__uint_as_float(v[2 * i]),
+                                                        __uint_as_float(v[2 * i + 1]));
+                            p[h][i] = o.u;
+                        }
+                    } else {
+                        uint32_t uu[16];
+                        tmem_ld_16x256b_x4(ta + kBlockT, uu);
+                        tmem_ld_wait();
+                        float hv[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float gv = __uint_as_float(v[i]);
+                            const float uv = __uint_as_float(uu[i]);
+                            hv[i] = __fdividef(gv * uv, 1.0f + __expf(-gv));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            BF2 o;
+                            o.h = __floats2bfloat162_rn(hv[2 * i], hv[2 * i + 1]);
+                            p[h][i] = o.u;
+                        }
                     }
                 }
+                // token group g (8 tokens): matrices (h, octet) = registers
+                // p[h][2g] (features 16h + 0..7) and p[h][2g+1] (16h + 8..15)
+#pragma unroll
+                for (int g = 0; g < 4; ++g)
+                    stmatrix_x4_trans(st_addr + g * 8 * kEpiRowBytes, p[0][2 * g], p[0][2 * g + 1],
+                                      p[1][2 * g], p[1][2 * g + 1]);
                 __syncwarp();
                 const int c = cb * 32 + lane;
                 if (c < rows) {
-                    const uint4* s4 = reinterpret_cast<const uint4*>(stg + lane * kEpiRowBytes);
+                    const uint4* s4 = reinterpret_cast<const uint4*>(
+                        smem + C::kOffEpi + (warp - kWarpEpi0) * C::kEpiWarpBytes + lane * kEpiRowBytes);
                     uint4* d4 = reinterpret_cast<uint4*>(
                         a.out + static_cast<size_t>(row0 + c) * a.out_ld + j * 128 + q * 32);
                     d4[0] = s4[0];
