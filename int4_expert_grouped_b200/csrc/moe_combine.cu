@@ -6,19 +6,18 @@
 //   dispatch_kernel   xs[p] = x[sorted_assign[p] / k]        p < T*k
 //   combine_kernel    y[t]  = bf16( sum_{j<k} w[t,j] * o[pos[t,j]] )
 //
-// Both are bound by HBM bandwidth: one warp moves one row of d bf16 values
-// with 16-byte accesses, so every warp instruction touches 512 contiguous
-// bytes.  Copying the token rows into expert order once lets both grouped
-// GEMMs read their token operand as dense 2-D TMA tiles (a gather of single
-// rows runs at a small fraction of that rate), and writing the down outputs
-// per assignment lets the sum over a token's experts run in a fixed order
-// with no atomics.
+// Both are bound by HBM bandwidth and move 16-byte vectors, consecutive
+// threads on consecutive vectors of a row.  Copying the token rows into
+// expert order once lets both grouped GEMMs read their token operand as dense
+// 2-D TMA tiles (a gather of single rows runs at a small fraction of that
+// rate), and writing the down outputs per assignment lets the sum over a
+// token's experts run in a fixed order with no atomics.
 #include "moe_internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kRowWarps = 8;  // warps per CTA, one row (token) per warp at a time
+constexpr int kThreads = 256;
 
 __device__ __forceinline__ uint4 ld_nc_v4(const uint4* p) {
     uint4 v;
@@ -28,31 +27,44 @@ __device__ __forceinline__ uint4 ld_nc_v4(const uint4* p) {
     return v;
 }
 
-__global__ void __launch_bounds__(kRowWarps * 32)
+// One warp per row (grid-stride): lane l moves 16-byte vectors l, l + 32, ...
+// of the row, up to kDispatchVecs of them loaded before the first store (all
+// of a row for d <= 2048), with the next row's source index read before the
+// stores.
+constexpr int kDispatchVecs = 8;
+
+__global__ void __launch_bounds__(kThreads)
 dispatch_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_assign, int Tk,
                 int k, int d, uint16_t* __restrict__ xs, int32_t* status) {
     const int lane = threadIdx.x & 31;
     const int nv = d >> 3;  // 16-byte vectors per row
-    for (int p = blockIdx.x * kRowWarps + (threadIdx.x >> 5); p < Tk; p += gridDim.x * kRowWarps) {
-        const int a = sorted_assign[p];
+    const int warps = gridDim.x * (kThreads / 32);
+    const uint4* x4 = reinterpret_cast<const uint4*>(x);
+    uint4* xs4 = reinterpret_cast<uint4*>(xs);
+    int p = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    int a = p < Tk ? sorted_assign[p] : 0;
+    for (; p < Tk; p += warps) {
+        const int a_next = p + warps < Tk ? sorted_assign[p + warps] : 0;
         if (static_cast<unsigned>(a) >= static_cast<unsigned>(Tk)) {
             if (lane == 0) report_error(status, MOE_ERR_DEVICE_BOUNDS, 300);
-            continue;
+            a = 0;
         }
-        const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(a / k) * d);
-        uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<size_t>(p) * d);
-        int i = lane;
-        for (; i + 96 < nv; i += 128) {
-            const uint4 v0 = ld_nc_v4(src + i);
-            const uint4 v1 = ld_nc_v4(src + i + 32);
-            const uint4 v2 = ld_nc_v4(src + i + 64);
-            const uint4 v3 = ld_nc_v4(src + i + 96);
-            dst[i] = v0;
-            dst[i + 32] = v1;
-            dst[i + 64] = v2;
-            dst[i + 96] = v3;
+        const uint4* src = x4 + static_cast<size_t>(a / k) * nv;
+        uint4* dst = xs4 + static_cast<size_t>(p) * nv;
+        for (int i0 = 0; i0 < nv; i0 += 32 * kDispatchVecs) {
+            uint4 v[kDispatchVecs];
+#pragma unroll
+            for (int u = 0; u < kDispatchVecs; ++u) {
+                const int i = i0 + 32 * u + lane;
+                v[u] = i < nv ? ld_nc_v4(src + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kDispatchVecs; ++u) {
+                const int i = i0 + 32 * u + lane;
+                if (i < nv) dst[i] = v[u];
+            }
         }
-        for (; i < nv; i += 32) dst[i] = ld_nc_v4(src + i);
+        a = a_next;
     }
 }
 
@@ -73,48 +85,47 @@ __device__ __forceinline__ void fma8(float* acc, float w, const uint4& v) {
     }
 }
 
-// One warp per token.  Lane j < k holds the position and weight of slot j;
-// each lane then sums 8 features at a time over the slots in order
-// j = 0 .. k-1 (fp32 fused multiply-add), loading up to 8 slots' vectors
-// before using any of them.
-__global__ void __launch_bounds__(kRowWarps * 32)
+// One CTA per token (grid-stride over tokens): the token's k positions and
+// weights go to shared memory, then thread i sums the 8 features of vector i
+// over the slots in order j = 0 .. k-1 (fp32 fused multiply-add), with the
+// loads of up to 8 slots issued before the first of them is used.
+__global__ void __launch_bounds__(kThreads)
 combine_kernel(const uint16_t* __restrict__ o, const int32_t* __restrict__ pos,
                const float* __restrict__ topk_w, int T, int k, int d, uint16_t* __restrict__ y,
                int32_t* status) {
-    const int lane = threadIdx.x & 31;
+    __shared__ int32_t sp[kMaxTopk];
+    __shared__ float sw[kMaxTopk];
     const int nv = d >> 3;
     const int Tk = T * k;
-    for (int t = blockIdx.x * kRowWarps + (threadIdx.x >> 5); t < T; t += gridDim.x * kRowWarps) {
-        int my_p = 0;
-        float my_w = 0.0f;
-        if (lane < k) {
-            my_p = pos[static_cast<size_t>(t) * k + lane];
-            my_w = topk_w[static_cast<size_t>(t) * k + lane];
-            if (static_cast<unsigned>(my_p) >= static_cast<unsigned>(Tk)) {
+    const uint4* o4 = reinterpret_cast<const uint4*>(o);
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();  // the previous token's slots are no longer read
+        if (threadIdx.x < k) {
+            int p = pos[static_cast<size_t>(t) * k + threadIdx.x];
+            float w = topk_w[static_cast<size_t>(t) * k + threadIdx.x];
+            if (static_cast<unsigned>(p) >= static_cast<unsigned>(Tk)) {
                 report_error(status, MOE_ERR_DEVICE_BOUNDS, 301);
-                my_p = 0;
-                my_w = 0.0f;
+                p = 0;
+                w = 0.0f;
             }
+            sp[threadIdx.x] = p;
+            sw[threadIdx.x] = w;
         }
+        __syncthreads();
         uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * d);
-        for (int i = lane; i < nv; i += 32) {
+        for (int i = threadIdx.x; i < nv; i += kThreads) {
             float acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
             for (int j0 = 0; j0 < k; j0 += 8) {
                 uint4 v[8];
-                float w[8];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int j = j0 + jj;
-                    const int p = __shfl_sync(0xffffffffu, my_p, j & 31);
-                    w[jj] = __shfl_sync(0xffffffffu, my_w, j & 31);
-                    v[jj] = j < k ? ld_nc_v4(reinterpret_cast<const uint4*>(o + static_cast<size_t>(p) * d) + i)
-                                  : make_uint4(0u, 0u, 0u, 0u);
-                }
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj)
-                    if (j0 + jj < k) fma8(acc, w[jj], v[jj]);
+                    v[jj] = j0 + jj < k ? ld_nc_v4(o4 + static_cast<size_t>(sp[j0 + jj]) * nv + i)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    if (j0 + jj < k) fma8(acc, sw[j0 + jj], v[jj]);
             }
             BF8 r;
 #pragma unroll
@@ -124,27 +135,24 @@ combine_kernel(const uint16_t* __restrict__ o, const int32_t* __restrict__ pos,
     }
 }
 
-int row_grid(long rows, int num_sms) {
-    const long need = (rows + kRowWarps - 1) / kRowWarps;
-    const long cap = static_cast<long>(num_sms) * 8;  // 8 CTAs of 8 warps per SM
-    return static_cast<int>(need < cap ? need : cap);
-}
-
 }  // namespace
 
 cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
                             uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st) {
     if (Tk <= 0) return cudaSuccess;
-    dispatch_kernel<<<row_grid(Tk, num_sms), kRowWarps * 32, 0, st>>>(x, sorted_assign, Tk, k, d, xs,
-                                                                      status);
+    const long need = (static_cast<long>(Tk) + kThreads / 32 - 1) / (kThreads / 32);
+    const long cap = static_cast<long>(num_sms) * 8;  // 8 CTAs of 8 warps per SM
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    dispatch_kernel<<<grid, kThreads, 0, st>>>(x, sorted_assign, Tk, k, d, xs, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T, int k,
                            int d, uint16_t* y, int32_t* status, int num_sms, cudaStream_t st) {
     if (T <= 0) return cudaSuccess;
-    combine_kernel<<<row_grid(T, num_sms), kRowWarps * 32, 0, st>>>(o, pos, topk_w, T, k, d, y,
-                                                                    status);
+    const long cap = static_cast<long>(num_sms) * 8;
+    const int grid = static_cast<int>(T < cap ? T : cap);
+    combine_kernel<<<grid, kThreads, 0, st>>>(o, pos, topk_w, T, k, d, y, status);
     return cudaGetLastError();
 }
 

@@ -48,14 +48,12 @@ constexpr int kWarpWProducer = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpLoader = 2;
 constexpr int kWarpIdle = 3;     // no role
-constexpr int kTransformGroups = 2;   // transform warp groups, alternate chunks
 constexpr int kWarpTransform0 = 4;
 constexpr int kNumTransformWarps = 8;
 constexpr int kWarpEpi0 = 12;
 constexpr int kNumEpiWarps = 4;
 constexpr int kGemmThreads = 16 * 32;
 constexpr int kTransformThreads = kNumTransformWarps * 32;
-constexpr int kGroupThreads = kTransformThreads / kTransformGroups;
 constexpr int kATileBytes = 128 * 128;     // 128 rows x 64 bf16 (128B swizzle)
 constexpr int kBStageBytes = kBlockT * 128;  // up to 256 token rows x 64 bf16
 constexpr int kEpiRowBytes = 80;    // staging row: 32 bf16 + 16 bytes of padding
@@ -65,8 +63,8 @@ constexpr uint32_t kTmemCols = 512;
 template <bool kDown>
 struct Cfg {
     static constexpr int kTiles = kDown ? 1 : 2;             // A tiles (of 128 rows) per unit
-    static constexpr int kNW = 4;                             // packed weight ring
-    static constexpr int kNA = kDown ? 4 : 2;                 // expanded bf16 A ring
+    static constexpr int kNW = kDown ? 4 : 2;                 // packed weight ring
+    static constexpr int kNA = kDown ? 4 : 3;                 // expanded bf16 A ring
     static constexpr int kNB = 3;                             // token B ring
     static constexpr int kAccBufs = kDown ? 2 : 1;            // TMEM accumulator buffers
     static constexpr int kAccCols = kTiles * kBlockT;         // columns per buffer
@@ -74,6 +72,9 @@ struct Cfg {
     static constexpr int kWStageBytes = packed_block_bytes(kTiles, 32);  // largest (group 32)
     static constexpr int kNibbleBytes = kTiles * 128 * 32;
     static constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
+    // transform warp groups; group g expands the chunks it with it % kGroups == g
+    static constexpr int kGroups = kDown ? 2 : 1;
+    static constexpr int kGroupThreads = kTransformThreads / kGroups;
     static constexpr int kTasks = kTiles * 256 / kGroupThreads;  // (row, half) tasks per thread
 
     static constexpr int kOffA = 0;
@@ -97,7 +98,7 @@ struct Cfg {
     // every W and A stage is filled and released by one group only, which
     // keeps each group at most one phase ahead.  (A shared A ring with three
     // or four groups deadlocks in a discrete-event model of this protocol.)
-    static_assert(kNW % kTransformGroups == 0 && kNA % kTransformGroups == 0,
+    static_assert(kNW % kGroups == 0 && kNA % kGroups == 0,
                   "transform groups must not alias mbarrier phases");
     static_assert(kTasks * kGroupThreads == kTiles * 256, "transform task split");
 };
@@ -181,10 +182,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kNW; ++s) {
             mbar_init(wfull(s), 1);
-            mbar_init(wempty(s), kNumTransformWarps / kTransformGroups);
+            mbar_init(wempty(s), kNumTransformWarps / C::kGroups);
         }
         for (int s = 0; s < C::kNA; ++s) {
-            mbar_init(afull(s), kNumTransformWarps / kTransformGroups);
+            mbar_init(afull(s), kNumTransformWarps / C::kGroups);
             mbar_init(aempty(s), 1);
         }
         for (int s = 0; s < C::kNB; ++s) {
@@ -276,10 +277,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     ok = false;
                     break;
                 }
-                // order the asynchronous MMAs after the waits, and the B rows
-                // written by cp.async (generic proxy) before the MMA reads them
+                // order the asynchronous MMAs after the waits (the transform
+                // warps fence their generic-proxy stores to A before arriving;
+                // B arrives through the TMA, already in the async proxy)
                 tc_fence_after();
-                fence_proxy_async_smem();
                 // Test the next stage now and look at the answer only after this
                 // stage's MMAs are issued: a barrier read stalls the issuing
                 // thread for about as long as one MMA runs, and the tensor core's
@@ -344,14 +345,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         // Two groups of transform warps take alternate chunks, so each warp
         // pays one round of barrier waits per two chunks.
         const int ttid = threadIdx.x - kWarpTransform0 * 32;
-        const int grp = ttid / kGroupThreads;
-        const int gtid = ttid % kGroupThreads;
+        const int grp = ttid / C::kGroupThreads;
+        const int gtid = ttid % C::kGroupThreads;
         const int gpc = kKChunk / a.group;
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
             for (int c = 0; c < KC; ++c, ++it) {
-                if (static_cast<int>(it % kTransformGroups) != grp) continue;
+                if (static_cast<int>(it % C::kGroups) != grp) continue;
                 const int sw = it % C::kNW;
                 const int sa = it % C::kNA;
                 if (!warp_wait(wfull(sw), (it / C::kNW) & 1, abort_flag) ||
@@ -372,14 +373,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 uint32_t sb[C::kTasks];
 #pragma unroll
                 for (int rep = 0; rep < C::kTasks; ++rep) {
-                    const int row = (gtid + kGroupThreads * rep) >> 1;
+                    const int row = (gtid + C::kGroupThreads * rep) >> 1;
                     pk[rep] = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
                     sb[rep] = *reinterpret_cast<const uint32_t*>(wst + C::kNibbleBytes +
                                                                  (row * gpc + g) * 4);
                 }
 #pragma unroll
                 for (int rep = 0; rep < C::kTasks; ++rep) {
-                    const int row = (gtid + kGroupThreads * rep) >> 1;
+                    const int row = (gtid + C::kGroupThreads * rep) >> 1;
                     BF2 s2, b2;
                     s2.u = __byte_perm(sb[rep], 0, 0x1010);
                     b2.u = __byte_perm(sb[rep], 0, 0x3232);
@@ -430,22 +431,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             for (int cb = 0; cb < ncb; ++cb) {
                 // p[h][i]: lane half h (features 16h + t/4 (+8)), register i
                 uint32_t p[2][8];
+                if constexpr (kDown) {
+                    // both lane halves in flight before the one wait
+                    uint32_t v[2][16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t v[16];
-                    const uint32_t ta = tb + (static_cast<uint32_t>(16 * h) << 16) + cb * 32;
-                    tmem_ld_16x256b_x4(ta, v);
-                    if constexpr (kDown) {
-                        tmem_ld_wait();
+                    for (int h = 0; h < 2; ++h)
+                        tmem_ld_16x256b_x4(tb + (static_cast<uint32_t>(16 * h) << 16) + cb * 32, v[h]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             BF2 o;
-                            o.h = __floats2bfloat162_rn(__uint_as_float(v[2 * i]),
-                                                        __uint_as_float(v[2 * i + 1]));
+                            o.h = __floats2bfloat162_rn(__uint_as_float(v[h][2 * i]),
+                                                        __uint_as_float(v[h][2 * i + 1]));
                             p[h][i] = o.u;
                         }
-                    } else {
-                        uint32_t uu[16];
+                } else {
+                    // gate and up of one lane half per wait (64 registers)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t v[16], uu[16];
+                        const uint32_t ta = tb + (static_cast<uint32_t>(16 * h) << 16) + cb * 32;
+                        tmem_ld_16x256b_x4(ta, v);
                         tmem_ld_16x256b_x4(ta + kBlockT, uu);
                         tmem_ld_wait();
                         float hv[16];

@@ -201,9 +201,12 @@ router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restric
 
     for (int tile = cta; tile < ntiles; tile += ctas) {
         const int t0 = tile * kRouterTile;
-        float acc[V];
+        // accumulators of experts (2q, 2q+1) of token tt are the pair acc2[tt*ES/2 + q],
+        // advanced together by one packed fp32 fused multiply-add (each half
+        // rounds exactly like a scalar fmaf)
+        float2 acc2[V / 2];
 #pragma unroll
-        for (int j = 0; j < V; ++j) acc[j] = 0.0f;
+        for (int j = 0; j < V / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
         load_chunk(t0, 0, 0);
         for (int kc = 0; kc < nkc; ++kc) {
             if (kc + 1 < nkc) {
@@ -221,22 +224,28 @@ router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restric
                 float xv[TT];
 #pragma unroll
                 for (int tt = 0; tt < TT; ++tt) xv[tt] = bf16_bits_to_float(xb[tt * kRouterKc + il]);
-                float wv[ES];
+                float2 wv[ES / 2];
 #pragma unroll
                 for (int q = 0; q < ES / 4; ++q) {
                     const float4 w4 = *reinterpret_cast<const float4*>(wb + il * WS + 4 * q);
-                    wv[4 * q + 0] = w4.x;
-                    wv[4 * q + 1] = w4.y;
-                    wv[4 * q + 2] = w4.z;
-                    wv[4 * q + 3] = w4.w;
+                    wv[2 * q + 0] = make_float2(w4.x, w4.y);
+                    wv[2 * q + 1] = make_float2(w4.z, w4.w);
                 }
 #pragma unroll
-                for (int tt = 0; tt < TT; ++tt)
+                for (int tt = 0; tt < TT; ++tt) {
+                    const float2 xx = make_float2(xv[tt], xv[tt]);
 #pragma unroll
-                    for (int ee = 0; ee < ES; ++ee)
-                        acc[tt * ES + ee] = __fmaf_rn(xv[tt], wv[ee], acc[tt * ES + ee]);
+                    for (int q = 0; q < ES / 2; ++q)
+                        acc2[tt * (ES / 2) + q] = __ffma2_rn(xx, wv[q], acc2[tt * (ES / 2) + q]);
+                }
             }
             __syncthreads();  // the buffer is refilled by the next chunk's copies
+        }
+        float acc[V];
+#pragma unroll
+        for (int j = 0; j < V / 2; ++j) {
+            acc[2 * j] = acc2[j].x;
+            acc[2 * j + 1] = acc2[j].y;
         }
         // reduce-scatter butterfly (see router_logits_kernel)
         int cnt = V;
