@@ -46,6 +46,7 @@ moe_status_t device_setup(int* num_sms) {
     DeviceCache& c = g_dev[dev];
     if (c.prepared.load() == 0) {
         if (moe::prepare_gemm_kernels() != cudaSuccess) return MOE_ERR_CUDA;
+        if (moe::prepare_decode_kernels() != cudaSuccess) return MOE_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -281,6 +282,36 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
         return e == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(e), st) == cudaSuccess;
     };
     if (ev && !mark(ev->start)) return MOE_ERR_CUDA;
+    if (moe::decode_supported(s, T)) {
+        // a few tokens: three launches bound by reading the selected experts' weights
+        const uint8_t* wp = static_cast<const uint8_t*>(packed_w);
+        moe::DecodeArgs da{};
+        da.s = s;
+        da.T = T;
+        da.x = x;
+        da.W_r = W_r;
+        da.b_r = b_r;
+        da.wpack_gu = wp;
+        da.wpack_dn = wp + align_up(plan->gu_packed, 256);
+        da.gu_block_bytes = plan->group_bytes;
+        da.dn_block_bytes = plan->down_block_bytes;
+        da.max_blocks = plan->max_blocks;
+        da.topk_idx = r.idx;
+        da.topk_w = r.w;
+        da.counts = r.counts;
+        da.offsets = r.offsets;
+        da.sorted_assign = r.sa;
+        da.pos = r.pos;
+        da.block_offsets = r.bo;
+        da.block_map = r.bm;
+        da.num_blocks = r.nb;
+        da.h = h;
+        da.y = y;
+        da.status = status;
+        MOE_CUDA(moe::launch_decode(da, st, ev ? ev->routed : nullptr, ev ? ev->gate_up : nullptr));
+        if (ev && !(mark(ev->down) && mark(ev->end))) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
     moe_status_t rs = run_route(plan, T, x, W_r, b_r, r, ws, st);
     if (rs != MOE_OK) return rs;
     if (T == 0) {

@@ -270,4 +270,33 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// ---------------------------------------------------------------------------
+// int4 -> bf16 expansion of the prepacked weights (shared by the grouped GEMM
+// and the small-batch path, so both produce the same bf16 weights)
+// ---------------------------------------------------------------------------
+union BF2 {
+    uint32_t u;
+    __nv_bfloat162 h;
+};
+
+// Expand one 32-bit word of 8 nibbles into 8 bf16 weights (16 bytes).  The
+// word holds K positions 2i (bits 4i..4i+3) and 2i+1 (bits 16+4i..) for
+// i = 0..3, so masking with 0x000F000F and or-ing the bf16 pattern of 128
+// yields the pair (128 + q_2i, 128 + q_2i+1) exactly; subtracting 128 is exact
+// and the fused multiply-add q*s + b rounds once.
+__device__ __forceinline__ uint4 expand8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
+    BF2 k128;
+    k128.u = 0x43004300u;
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        BF2 v, o;
+        v.u = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+        const __nv_bfloat162 q = __hsub2(v.h, k128.h);
+        o.h = __hfma2(q, s2, b2);
+        r[i] = o.u;
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
 }  // namespace moe

@@ -33,6 +33,7 @@ constexpr int kMaxTopk = 32;      // one warp lane per selected expert
 constexpr int kRouteGroupT = 256; // tokens per scatter group (one histogram row)
 constexpr int kBlockT = 256;      // block map tile height = largest MMA N
 constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
+constexpr int kDecodeMaxT = 8;    // largest batch the small-batch (decode) path takes
 
 // Packed weight block: `tiles` 128-row A tiles of one 64-wide K chunk
 // (gate/up: the gate rows, then the up rows of 128 features; down: 128 rows):
@@ -107,5 +108,32 @@ cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T,
                            int k, int d, uint16_t* y, int32_t* status, int num_sms,
                            cudaStream_t st);
+
+// ---- small-batch path (moe_decode.cu) ----
+struct DecodeArgs {
+    moe_shape_t s;
+    int T;
+    const uint16_t* x;
+    const float* W_r;
+    const float* b_r;
+    const uint8_t* wpack_gu;     // packed gate/up blocks
+    const uint8_t* wpack_dn;     // packed down blocks
+    int gu_block_bytes;
+    int dn_block_bytes;
+    int max_blocks;
+    int32_t *topk_idx, *counts, *offsets, *sorted_assign, *pos, *block_offsets, *block_map,
+        *num_blocks;
+    float* topk_w;
+    uint16_t* h;                 // workspace [T*k, f]
+    uint16_t* y;                 // [T, d]
+    int32_t* status;
+};
+// Whether the small-batch kernels take this shape at batch T (otherwise the
+// batched path runs).
+bool decode_supported(const moe_shape_t& s, int T);
+cudaError_t prepare_decode_kernels();
+// Records ev_routed after the routing kernel and ev_gate_up after the gate/up
+// kernel when they are not null.
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed, void* ev_gate_up);
 
 }  // namespace moe

@@ -11,7 +11,7 @@
 //                         pos)
 #include <atomic>
 
-#include "moe_internal.h"
+#include "moe_route_common.cuh"
 
 namespace moe {
 
@@ -292,18 +292,6 @@ router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restric
 // ---------------------------------------------------------------------------
 constexpr int kTopkWarps = 8;
 
-struct Cand {
-    float v;
-    int id;  // >= kInvalidId means none
-};
-constexpr int kInvalidId = 1 << 30;
-
-__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
-    if (a.id >= kInvalidId) return false;
-    if (b.id >= kInvalidId) return true;
-    return a.v > b.v || (a.v == b.v && a.id < b.id);
-}
-
 __global__ void __launch_bounds__(kTopkWarps * 32)
 router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
@@ -312,51 +300,12 @@ router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
     const int warp = threadIdx.x >> 5;
     const int t = blockIdx.x * kTopkWarps + warp;
     if (t >= T) return;
-
-    constexpr int kMaxPerLane = kMaxExperts / 32;
-    float v[kMaxPerLane];
-    bool taken[kMaxPerLane];
-#pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = e < E ? logits[static_cast<size_t>(t) * E + e] : 0.0f;
-        taken[i] = e >= E;
-    }
-
-    int my_id = 0;
-    float my_v = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        Cand best{0.0f, kInvalidId};
-#pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i) {
-            const Cand c{v[i], taken[i] ? kInvalidId : lane + 32 * i};
-            if (better(c, best)) best = c;
-        }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) {
-            Cand o;
-            o.v = __shfl_xor_sync(0xffffffffu, best.v, m);
-            o.id = __shfl_xor_sync(0xffffffffu, best.id, m);
-            if (better(o, best)) best = o;
-        }
-        // every lane now holds the same winner
-#pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i)
-            if (best.id == lane + 32 * i) taken[i] = true;
-        if (lane == j) {
-            my_id = best.id;
-            my_v = best.v;
-        }
-    }
-
-    const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
-    float ex = lane < k ? expf(__fsub_rn(my_v, l0)) : 0.0f;
-    float sum = ex;
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, m));
+    int my_id;
+    float my_w;
+    warp_topk(logits + static_cast<size_t>(t) * E, E, k, lane, my_id, my_w);
     if (lane < k) {
         topk_idx[static_cast<size_t>(t) * k + lane] = my_id;
-        topk_w[static_cast<size_t>(t) * k + lane] = __fdiv_rn(ex, sum);
+        topk_w[static_cast<size_t>(t) * k + lane] = my_w;
         atomicAdd(hist + static_cast<size_t>(t / kRouteGroupT) * E + my_id, 1);
     }
 }
@@ -371,34 +320,6 @@ router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 256;
 
-__device__ __forceinline__ int block_exclusive_scan(int v, int* sh_warp, int* total) {
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    int inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
-    }
-    if (lane == 31) sh_warp[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < (kScanThreads / 32) ? sh_warp[lane] : 0;
-        int wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += n;
-        }
-        if (lane < (kScanThreads / 32)) sh_warp[lane] = wi - w;  // exclusive warp offsets
-        if (lane == (kScanThreads / 32) - 1) sh_warp[kScanThreads / 32] = wi;
-    }
-    __syncthreads();
-    const int res = sh_warp[warp] + inc - v;
-    *total = sh_warp[kScanThreads / 32];
-    __syncthreads();
-    return res;
-}
 
 __global__ void __launch_bounds__(kScanThreads)
 route_scan_kernel(const int32_t* __restrict__ hist, int ng, int E, int BT,
@@ -412,7 +333,7 @@ route_scan_kernel(const int32_t* __restrict__ hist, int ng, int E, int BT,
     if (e < E)
         for (int g = 0; g < ng; ++g) c += hist[static_cast<size_t>(g) * E + e];
     int total = 0;
-    const int off = block_exclusive_scan(e < E ? c : 0, sh_warp, &total);
+    const int off = block_exclusive_scan<kScanThreads>(e < E ? c : 0, sh_warp, &total);
     if (e < E) {
         counts[e] = c;
         offsets[e] = off;
@@ -426,7 +347,7 @@ route_scan_kernel(const int32_t* __restrict__ hist, int ng, int E, int BT,
 
     const int nt = e < E ? (c + BT - 1) / BT : 0;
     int nb_total = 0;
-    const int bo = block_exclusive_scan(nt, sh_warp, &nb_total);
+    const int bo = block_exclusive_scan<kScanThreads>(nt, sh_warp, &nb_total);
     if (e < E) {
         block_offsets[e] = bo;
         for (int i = 0; i < nt; ++i) {
