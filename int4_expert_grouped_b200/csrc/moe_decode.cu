@@ -41,7 +41,10 @@ constexpr int kRouteCtas = 8;       // cluster size of the routing kernel: E/8 e
 constexpr int kRowThreads = 512;    // 16 warps, one weight row each
 constexpr int kGuWords = 8;         // nibble words per lane and gate/up row: d <= 2048
 constexpr int kDnWords = 4;         // nibble words per lane and down row: f <= 1024
-constexpr int kDnBlockBatch = 4;    // experts whose down loads a lane issues together
+// experts whose down loads a lane issues together (fewer for larger batches,
+// whose operand loops need the registers)
+template <int kT>
+constexpr int dn_block_batch() { return kT <= 4 ? 8 : 4; }
 
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -104,14 +107,16 @@ __device__ __forceinline__ uint16_t bf16_round_bits(float v) {
 
 // ---------------------------------------------------------------------------
 // Routing of the few tokens in shared memory (CTA 0 of the routing cluster,
-// kRowThreads threads) from the logits lg [T][E]: top-k (warp per token),
-// counts (integer atomics), offsets (exclusive scan), block map
+// kRowThreads threads) from the logits lg [T][E]: top-k (each (token, expert)
+// pair finds its slot in parallel; the warp of a token then forms the
+// weights), counts (integer atomics), offsets (exclusive scan), block map
 // (ceil(count / kBlockT) tiles per expert in ascending expert order), and the
 // stable scatter (the rank of assignment a within its expert is the number of
 // earlier assignments to that expert).
 // ---------------------------------------------------------------------------
 struct DecodeRoute {
     float lg[kDecodeMaxT * kMaxExperts];
+    float sel[kDecodeMaxAssign];  // logit of each selected slot
     int idx[kDecodeMaxAssign];
     float w[kDecodeMaxAssign];
     int sa[kDecodeMaxAssign];
@@ -131,14 +136,19 @@ __device__ void route_from_logits(int T, int E, int k, int max_blocks, DecodeRou
     const int tid = threadIdx.x;
     const int Tk = T * k;
     if (tid < E) R.cnt[tid] = 0;
-    for (int t = warp; t < T; t += kRowThreads / 32) {
-        int id;
-        float wt;
-        warp_topk(R.lg + t * E, E, k, lane, id, wt);
-        if (lane < k) {
-            R.idx[t * k + lane] = id;
-            R.w[t * k + lane] = wt;
+    for (int it = tid; it < T * E; it += kRowThreads) {
+        const int t = it / E;
+        const int e = it - t * E;
+        const int slot = expert_slot(R.lg + t * E, E, e);
+        if (slot < k) {
+            R.idx[t * k + slot] = e;
+            R.sel[t * k + slot] = R.lg[it];
         }
+    }
+    __syncthreads();
+    for (int t = warp; t < T; t += kRowThreads / 32) {
+        const float wt = warp_slot_weights(lane < k ? R.sel[t * k + lane] : 0.0f, k, lane);
+        if (lane < k) R.w[t * k + lane] = wt;
     }
     __syncthreads();
     for (int a = tid; a < Tk; a += kRowThreads) atomicAdd(&R.cnt[R.idx[a]], 1);
@@ -210,9 +220,11 @@ __device__ void write_route(const DecodeRoute& R, const DecodeRouteOut& o, int T
 // lane p holds after step m is v_p + v_{p^m}, so the result is the tree that
 // adds chains q and q + m for q < m, m = 16..1), plus the bias.  Item
 // (p, el) of a CTA runs chain p of expert e0 + el for all T tokens: a group
-// of EC lanes reads EC consecutive floats of a W_r row per step.  The logits
-// go to CTA 0's shared memory (distributed shared memory), which then routes.
-// Dynamic shared memory: x [T][d] bf16, then the chains [T][32][33] fp32.
+// of EC lanes reads EC consecutive floats of a W_r row per step, from a copy
+// of the CTA's W_r columns that all threads load with 16-byte vectors first.
+// The logits go to CTA 0's shared memory (distributed shared memory), which
+// then routes.  Dynamic shared memory: x [T][d] bf16, the W_r columns [d][EC]
+// fp32, the chains [T][32][33] fp32.
 // ---------------------------------------------------------------------------
 __global__ void __cluster_dims__(kRouteCtas, 1, 1) __launch_bounds__(kRowThreads)
 decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
@@ -223,7 +235,8 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     __shared__ DecodeRoute R;
     extern __shared__ __align__(16) uint8_t dsm[];
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(dsm);
-    float* cs = reinterpret_cast<float*>(dsm + static_cast<size_t>(T) * d * 2);  // [t][p][33]
+    float* ws = reinterpret_cast<float*>(dsm + static_cast<size_t>(T) * d * 2);  // [i][EC]
+    float* cs = ws + static_cast<size_t>(d) * (E / kRouteCtas);                  // [t][p][33]
     pdl_launch_dependents();
     const int rank = static_cast<int>(cluster.block_rank());
     // the status word reports the most recent call: the first kernel clears it
@@ -233,36 +246,40 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     const int nsteps = d >> 5;
     const int items = 32 * EC;
     cta_copy16(dsm, x, T * d / 8);
-    // The first W batch of the thread's first item is in flight across the
-    // barrier that publishes x.
-    float w[64];
-    auto load_w = [&](int it, int s0) {
-        const int p = it / EC;
-        const int el = it - p * EC;
+    {
+        // W_r[:, e0 .. e0+EC) -> ws: 16-byte vectors (EC % 4 == 0), 16 in
+        // flight per thread before their stores
+        const int nv = d * (EC / 4);
+        const int vrow = EC / 4;
+        for (int v0 = threadIdx.x; v0 < nv; v0 += 16 * kRowThreads) {
+            float4 v[16];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-            const int s = s0 + j;
-            w[j] = (it < items && s < nsteps) ? __ldg(W + static_cast<size_t>(32 * s + p) * E + e0 + el)
-                                               : 0.0f;
+            for (int u = 0; u < 16; ++u) {
+                const int vi = v0 + u * kRowThreads;
+                if (vi < nv) {
+                    const int i = vi / vrow;
+                    v[u] = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) +
+                                 (vi - i * vrow));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int vi = v0 + u * kRowThreads;
+                if (vi < nv) reinterpret_cast<float4*>(ws)[vi] = v[u];
+            }
         }
-    };
-    load_w(threadIdx.x, 0);
+    }
     __syncthreads();
     for (int it = threadIdx.x; it < items; it += kRowThreads) {
         const int p = it / EC;
         const int el = it - p * EC;
-        for (int s0 = 0; s0 < nsteps; s0 += 64) {
-            if (it != static_cast<int>(threadIdx.x) || s0 != 0) load_w(it, s0);
 #pragma unroll 1
-            for (int t = 0; t < T; ++t) {
-                float* c = cs + (t * 32 + p) * 33 + el;
-                float a = s0 == 0 ? 0.0f : *c;
-#pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    if (s0 + j < nsteps)
-                        a = __fmaf_rn(bf16_bits_to_float(xs[t * d + 32 * (s0 + j) + p]), w[j], a);
-                *c = a;
-            }
+        for (int t = 0; t < T; ++t) {
+            float a = 0.0f;
+#pragma unroll 16
+            for (int s = 0; s < nsteps; ++s)
+                a = __fmaf_rn(bf16_bits_to_float(xs[t * d + 32 * s + p]), ws[(32 * s + p) * EC + el], a);
+            cs[(t * 32 + p) * 33 + el] = a;
         }
     }
     __syncthreads();
@@ -342,23 +359,22 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------------------
 // Gate/up and SwiGLU for a batch of kT tokens.  Grid: min(E, kT*k) blocks x
-// f/8 feature slices (CTAs past the number of blocks return).  Warp r < 8
-// takes the gate row of feature 8q' + r of tile j, warp 8 + r the up row of
-// the same feature; rows of the block beyond its count repeat its first row
-// and are not stored.  Dynamic shared memory: x [kT][d].
+// f/16 feature slices (CTAs past the number of blocks return).  Warp r takes
+// feature 16q' + r of tile j: its gate row and its up row, so SwiGLU needs
+// no exchange between warps.  Rows of the block beyond its count repeat its
+// first row and are not stored.  Dynamic shared memory: x [kT][d].
 // ---------------------------------------------------------------------------
 template <int kT>
 __global__ void __launch_bounds__(kRowThreads)
 decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wpack, int d,
                      int k, int f, int group, int bb, DecodeRouteOut ro, uint16_t* __restrict__ h) {
-    __shared__ float gu[16][kT];
     __shared__ int sblk[3 + kT];  // expert, first row, rows, token of each row
     extern __shared__ __align__(16) uint8_t dsm[];
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(dsm);
     pdl_launch_dependents();
     cta_copy16(dsm, x, kT * d / 8);  // x does not depend on the routing kernel
     pdl_wait();
-    const int nq = f / 8;
+    const int nq = f / 16;
     const int b = blockIdx.x / nq;
     const int q = blockIdx.x - b * nq;
     if (b >= min(ro.num_blocks[0], kDecodeMaxAssign)) return;
@@ -366,39 +382,38 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
     __syncthreads();
     const int row0 = sblk[1];
     const int nrows = min(sblk[2], kT);
-    if (threadIdx.x < kT) sblk[3 + threadIdx.x] = ro.sorted_assign[row0 + min(static_cast<int>(threadIdx.x), nrows - 1)] / k;
+    if (threadIdx.x < kT)
+        sblk[3 + threadIdx.x] =
+            ro.sorted_assign[row0 + min(static_cast<int>(threadIdx.x), nrows - 1)] / k;
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int j = q >> 4;
-    const int r0 = (q & 15) * 8;
-    const int prow = warp < 8 ? r0 + warp : 128 + r0 + (warp - 8);
+    const int j = q >> 3;
+    const int feat = (q & 7) * 16 + warp;  // feature within tile j
     const int NT = f / 128;
     const int KC = d / kKChunk;
+    const int gpc = kKChunk / group;
     const uint8_t* base = wpack + (static_cast<size_t>(sblk[0]) * NT + j) * KC * bb;
-    RowLoads<kGuWords> L;
-    row_load(L, base, bb, prow, 2 * 128 * 32, kKChunk / group, d / 8, lane);
+    RowLoads<kGuWords> Lg, Lu;
+    row_load(Lg, base, bb, feat, 2 * 128 * 32, gpc, d / 8, lane);
+    row_load(Lu, base, bb, 128 + feat, 2 * 128 * 32, gpc, d / 8, lane);
     const uint16_t* rows[kT];
-    float acc[kT];
+    float ag[kT], au[kT];
 #pragma unroll
     for (int i = 0; i < kT; ++i) {
         rows[i] = xs + static_cast<size_t>(sblk[3 + i]) * d;
-        acc[i] = 0.0f;
+        ag[i] = 0.0f;
+        au[i] = 0.0f;
     }
-    row_dots<kT>(L, rows, d / 8, lane, acc);
+    row_dots<kT>(Lg, rows, d / 8, lane, ag);
+    row_dots<kT>(Lu, rows, d / 8, lane, au);
 #pragma unroll
     for (int i = 0; i < kT; ++i) {
-        const float v = warp_sum(acc[i]);
-        if (lane == 0) gu[warp][i] = v;
-    }
-    __syncthreads();
-    if (threadIdx.x < 8 * nrows) {
-        const int ff = threadIdx.x & 7;
-        const int i = threadIdx.x >> 3;
-        const float gv = gu[ff][i];
-        const float uv = gu[8 + ff][i];
-        h[static_cast<size_t>(row0 + i) * f + j * 128 + r0 + ff] =
-            bf16_round_bits(__fdividef(gv * uv, 1.0f + __expf(-gv)));
+        const float gv = warp_sum(ag[i]);
+        const float uv = warp_sum(au[i]);
+        if (lane == 0 && i < nrows)
+            h[static_cast<size_t>(row0 + i) * f + j * 128 + feat] =
+                bf16_round_bits(__fdividef(gv * uv, 1.0f + __expf(-gv)));
     }
 }
 
@@ -441,6 +456,7 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
     const int NTd = d / 128;
     const int KCd = f / kKChunk;
     const int nw = f / 8;
+    constexpr int kDnBlockBatch = dn_block_batch<kT>();
     for (int b0 = 0; b0 < nb; b0 += kDnBlockBatch) {
         RowLoads<kDnWords> L[kDnBlockBatch];
 #pragma unroll
@@ -496,6 +512,12 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, int threads, size_t smem, cudaStr
 }
 
 constexpr size_t kDecodeSmemLimit = 96 * 1024;
+constexpr size_t kRouteSmemLimit = 200 * 1024;
+
+size_t route_smem_bytes(const moe_shape_t& s, int T) {
+    return static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(s.d) * (s.E / kRouteCtas) * 4 +
+           static_cast<size_t>(T) * 32 * 33 * 4;
+}
 
 template <int kT>
 cudaError_t set_expert_kernel_smem() {
@@ -512,7 +534,7 @@ cudaError_t launch_experts(const DecodeArgs& a, const DecodeRouteOut& ro, cudaSt
                            void* ev_gate_up) {
     const moe_shape_t& s = a.s;
     const int nb_max = std::min(s.E, kT * s.k);
-    cudaError_t e = launch_pdl(decode_gateup_kernel<kT>, dim3(nb_max * (s.f / 8)), kRowThreads,
+    cudaError_t e = launch_pdl(decode_gateup_kernel<kT>, dim3(nb_max * (s.f / 16)), kRowThreads,
                                static_cast<size_t>(kT) * s.d * 2, st, a.x, a.wpack_gu, s.d, s.k,
                                s.f, s.group, a.gu_block_bytes, ro, a.h);
     if (e != cudaSuccess) return e;
@@ -528,7 +550,9 @@ cudaError_t launch_experts(const DecodeArgs& a, const DecodeRouteOut& ro, cudaSt
 
 bool decode_supported(const moe_shape_t& s, int T) {
     if (T < 1 || T > kDecodeMaxT) return false;
-    if (T * s.k > kDecodeMaxAssign || s.E > kMaxExperts || s.E % kRouteCtas != 0) return false;
+    if (T * s.k > kDecodeMaxAssign || s.E > kMaxExperts) return false;
+    // whole 16-byte vectors of W_r columns per routing CTA
+    if (s.E % (4 * kRouteCtas) != 0 || route_smem_bytes(s, T) > kRouteSmemLimit) return false;
     // nibble words (8 K values each) per lane and row
     if (s.d > 8 * 32 * kGuWords || s.f > 8 * 32 * kDnWords) return false;
     const size_t x_bytes = static_cast<size_t>(T) * s.d * 2;
@@ -539,7 +563,7 @@ bool decode_supported(const moe_shape_t& s, int T) {
 cudaError_t prepare_decode_kernels() {
     cudaError_t e = cudaFuncSetAttribute(decode_route_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kDecodeSmemLimit));
+                                         static_cast<int>(kRouteSmemLimit));
     if (e != cudaSuccess) return e;
     static_assert(kDecodeMaxT == 8, "one instantiation per batch size");
     if ((e = set_expert_kernel_smem<1>()) != cudaSuccess) return e;
@@ -557,7 +581,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed,
     const int T = a.T;
     const DecodeRouteOut ro{a.topk_idx, a.topk_w,        a.counts,    a.offsets,   a.sorted_assign,
                             a.pos,      a.block_offsets, a.block_map, a.num_blocks};
-    const size_t route_smem = static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(T) * 32 * 33 * 4;
+    const size_t route_smem = route_smem_bytes(s, T);
     decode_route_kernel<<<kRouteCtas, kRowThreads, route_smem, st>>>(
         a.x, a.W_r, a.b_r, T, s.d, s.E, s.k, a.max_blocks, ro, a.status);
     cudaError_t e = cudaGetLastError();

@@ -22,6 +22,19 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
     return a.v > b.v || (a.v == b.v && a.id < b.id);
 }
 
+// Routing weights of one token by one warp: lane j < k holds the logit of
+// slot j; softmax over the k slots, w_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0),
+// the sum in a fixed xor butterfly order.  Returns lane j's weight (0 for
+// lanes >= k).
+__device__ __forceinline__ float warp_slot_weights(float my_v, int k, int lane) {
+    const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = lane < k ? expf(__fsub_rn(my_v, l0)) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, m));
+    return lane < k ? __fdiv_rn(ex, sum) : 0.0f;
+}
+
 // Top-k of one token's E logits by one warp: lane holds experts lane,
 // lane+32, ...; k rounds of a warp-wide arg-max over the unselected experts.
 // Routing weights: softmax over the k selected logits,
@@ -63,12 +76,17 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, 
             my_v = best.v;
         }
     }
-    const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
-    const float ex = lane < k ? expf(__fsub_rn(my_v, l0)) : 0.0f;
-    float sum = ex;
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, m));
-    my_w = lane < k ? __fdiv_rn(ex, sum) : 0.0f;
+    my_w = warp_slot_weights(my_v, k, lane);
+}
+
+// Slot of expert e among one token's E logits: the number of experts that
+// come before it in the order (logit descending, id ascending).  The experts
+// with slot < k are exactly the ones warp_topk selects, in the same order.
+__device__ __forceinline__ int expert_slot(const float* __restrict__ row, int E, int e) {
+    const Cand me{row[e], e};
+    int r = 0;
+    for (int e2 = 0; e2 < E; ++e2) r += better(Cand{row[e2], e2}, me);
+    return r;
 }
 
 // Exclusive prefix sum of one int per thread over a CTA of kThreads threads
