@@ -155,10 +155,10 @@ moe_status_t moe_plan_create(const moe_shape_t* shape, moe_plan_t** plan, moe_pl
     p->max_blocks = max_blocks_for(s, s.T_max);
     p->ng_max = (s.T_max + kRouteGroupT - 1) / kRouteGroupT;
     p->group_bytes = moe::packed_block_bytes(2, s.group);
-    p->down_block_bytes = moe::packed_block_bytes(1, s.group);
+    p->down_block_bytes = moe::packed_block_bytes(moe::kDownTiles, s.group);
     const size_t E = s.E;
     p->gu_packed = E * (s.f / 128) * (s.d / moe::kKChunk) * p->group_bytes;
-    p->dn_packed = E * (s.d / 128) * (s.f / moe::kKChunk) * p->down_block_bytes;
+    p->dn_packed = E * (s.d / (128 * moe::kDownTiles)) * (s.f / moe::kKChunk) * p->down_block_bytes;
     p->packed_bytes = align_up(p->gu_packed, 256) + p->dn_packed;
 
     const size_t T = s.T_max, k = s.k;
@@ -223,7 +223,8 @@ moe_status_t moe_prepack_weights(const moe_plan_t* plan, const moe_expert_weight
                           lw->up.bias, s.f, s.d, 128, 0, s.f / 128, 2};
     MOE_CUDA(moe::launch_prepack(gu, s.E, s.group, out, st));
     moe::PrepackSource dn{lw->down.q, lw->down.scale, lw->down.bias, lw->down.q, lw->down.scale,
-                          lw->down.bias, s.d, s.f, 128, 0, s.d / 128, 1};
+                          lw->down.bias, s.d, s.f, 128 * moe::kDownTiles, 128,
+                          s.d / (128 * moe::kDownTiles), moe::kDownTiles};
     MOE_CUDA(moe::launch_prepack(dn, s.E, s.group, out + align_up(plan->gu_packed, 256), st));
     return MOE_OK;
 }
@@ -346,7 +347,7 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.wpack = wp + align_up(plan->gu_packed, 256);
     g.out = xs;
     g.K = s.f;
-    g.NT = s.d / 128;
+    g.NT = s.d / (128 * moe::kDownTiles);
     g.out_ld = s.d;
     g.block_bytes = plan->down_block_bytes;
     g.max_units = mb * g.NT;

@@ -419,8 +419,8 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
 
 // ---------------------------------------------------------------------------
 // Down projection and combine for a batch of kT tokens.  Grid: d/16 CTAs;
-// warp r of CTA m owns output feature 16m + r (row (16m + r) % 128 of down
-// tile (16m + r) / 128).  For every block (expert) the warp dots that
+// warp r of CTA m owns output feature 16m + r (row (16m + r) % (128 *
+// kDownTiles) of down block (16m + r) / (128 * kDownTiles)).  For every block (expert) the warp dots that
 // expert's row with the block's h rows, rounds each sum to bf16 (the expert
 // output o), and after all blocks thread (t, r) sums o over token t's slots
 // in slot order.  Dynamic shared memory: h [kT*k][f] bf16.
@@ -451,9 +451,9 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
     __syncthreads();
     const int nb = snb;
     const int m = blockIdx.x * 16 + warp;
-    const int jd = m / 128;
-    const int prow = m % 128;
-    const int NTd = d / 128;
+    const int jd = m / (128 * kDownTiles);
+    const int prow = m % (128 * kDownTiles);
+    const int NTd = d / (128 * kDownTiles);
     const int KCd = f / kKChunk;
     const int nw = f / 8;
     constexpr int kDnBlockBatch = dn_block_batch<kT>();
@@ -463,7 +463,7 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
         for (int u = 0; u < kDnBlockBatch; ++u)
             if (b0 + u < nb)
                 row_load(L[u], wpack + (static_cast<size_t>(sbm[3 * (b0 + u)]) * NTd + jd) * KCd * bb,
-                         bb, prow, 128 * 32, kKChunk / group, nw, lane);
+                         bb, prow, 128 * kDownTiles * 32, kKChunk / group, nw, lane);
 #pragma unroll
         for (int u = 0; u < kDnBlockBatch; ++u) {
             if (b0 + u < nb) {

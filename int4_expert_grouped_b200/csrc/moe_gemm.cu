@@ -8,7 +8,8 @@
 //   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
 //       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order,
 //                epilogue h = silu(D0) * D1 -> bf16 h rows
-//       down:    D = 128-row tile of Wd times h^T, epilogue o = bf16(D) rows
+//       down:    D = kDownTiles 128-row tiles of Wd times h^T, epilogue
+//                o = bf16(D) rows
 //                (the routing-weighted sum over a token's experts is a
 //                separate pass, so no output element is ever accumulated by
 //                two CTAs)
@@ -35,8 +36,10 @@
 //                groups that take alternate K chunks
 //   warps 12-15  epilogue: TMEM -> registers -> bf16 rows of h or o
 // TMEM: gate/up holds one buffer of 2 x 256 columns (gate, up), so its
-// epilogue runs between units; down holds two buffers of 256 columns, so its
-// epilogue overlaps the next unit's main loop.
+// epilogue runs between units.  Down with one tile per unit holds two buffers
+// of 256 columns, so its epilogue overlaps the next unit's main loop (measured
+// faster than two tiles per unit, which halves the token-operand traffic per
+// MMA but exposes the epilogue).
 #include <cudaTypedefs.h>
 
 #include "moe_internal.h"
@@ -62,18 +65,19 @@ constexpr uint32_t kTmemCols = 512;
 // Per-projection configuration.
 template <bool kDown>
 struct Cfg {
-    static constexpr int kTiles = kDown ? 1 : 2;             // A tiles (of 128 rows) per unit
-    static constexpr int kNW = kDown ? 4 : 2;                 // packed weight ring
-    static constexpr int kNA = kDown ? 4 : 3;                 // expanded bf16 A ring
+    static constexpr int kTiles = kDown ? kDownTiles : 2;     // A tiles (of 128 rows) per unit
+    static constexpr bool kOneTile = kTiles == 1;
+    static constexpr int kNW = kOneTile ? 4 : 2;              // packed weight ring
+    static constexpr int kNA = kOneTile ? 4 : 3;              // expanded bf16 A ring
     static constexpr int kNB = 3;                             // token B ring
-    static constexpr int kAccBufs = kDown ? 2 : 1;            // TMEM accumulator buffers
+    static constexpr int kAccBufs = kOneTile ? 2 : 1;         // TMEM accumulator buffers
     static constexpr int kAccCols = kTiles * kBlockT;         // columns per buffer
     static constexpr int kAStageBytes = kTiles * kATileBytes;
     static constexpr int kWStageBytes = packed_block_bytes(kTiles, 32);  // largest (group 32)
     static constexpr int kNibbleBytes = kTiles * 128 * 32;
     static constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
     // transform warp groups; group g expands the chunks it with it % kGroups == g
-    static constexpr int kGroups = kDown ? 2 : 1;
+    static constexpr int kGroups = kOneTile ? 2 : 1;
     static constexpr int kGroupThreads = kTransformThreads / kGroups;
     static constexpr int kTasks = kTiles * 256 / kGroupThreads;  // (row, half) tasks per thread
 
@@ -401,9 +405,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 break;
             }
             tc_fence_after();
-            const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
+            // gate/up: one output tile (gate at column 0, up at kBlockT); down:
+            // kTiles output tiles of 128 features at columns t * kBlockT
+            constexpr int kOutTiles = kDown ? C::kTiles : 1;
 #pragma unroll 1
-            for (int cb = 0; cb < ncb; ++cb) {
+            for (int it = 0; it < kOutTiles * ncb; ++it) {
+                const int t = it / ncb;
+                const int cb = it - t * ncb;
+                const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols +
+                                    t * kBlockT;
                 // p[h][i]: lane half h (features 16h + t/4 (+8)), register i
                 uint32_t p[2][8];
                 if constexpr (kDown) {
@@ -457,8 +467,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 if (c < rows) {
                     const uint4* s4 = reinterpret_cast<const uint4*>(
                         smem + C::kOffEpi + (warp - kWarpEpi0) * C::kEpiWarpBytes + lane * kEpiRowBytes);
-                    uint4* d4 = reinterpret_cast<uint4*>(
-                        a.out + static_cast<size_t>(row0 + c) * a.out_ld + j * 128 + q * 32);
+                    uint4* d4 = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(row0 + c) * a.out_ld +
+                                                         (j * kOutTiles + t) * 128 + q * 32);
                     d4[0] = s4[0];
                     d4[1] = s4[1];
                     d4[2] = s4[2];

@@ -34,6 +34,7 @@ constexpr int kRouteGroupT = 256; // tokens per scatter group (one histogram row
 constexpr int kBlockT = 256;      // block map tile height = largest MMA N
 constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
 constexpr int kDecodeMaxT = 8;    // largest batch the small-batch (decode) path takes
+constexpr int kDownTiles = 1;     // 128-row down-projection tiles per packed block and GEMM unit
 
 // Packed weight block: `tiles` 128-row A tiles of one 64-wide K chunk
 // (gate/up: the gate rows, then the up rows of 128 features; down: 128 rows):

@@ -139,22 +139,32 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
 // Grid: (E / ES) * ctas_per_slice; CTA c serves slice c % (E / ES) and tiles
 // c / (E / ES), c / (E / ES) + ctas_per_slice, ...
 // ---------------------------------------------------------------------------
-constexpr int kRouterTile = 64;   // tokens per tile
-constexpr int kRouterKc = 256;    // K chunk of x held in shared memory
-constexpr int kRouterWarps = 8;
+// Configuration: ES experts per slice, TT tokens per warp, WARPS warps, K
+// chunks of KC.  A tile is TT * WARPS tokens.
+template <int ES_, int TT_, int WARPS_, int KC_>
+struct RouterCfg {
+    static constexpr int ES = ES_, TT = TT_, WARPS = WARPS_, KC = KC_;
+    static constexpr int kTile = TT * WARPS;
+    static constexpr int smem_bytes(int d) { return d * (ES + 4) * 4 + 2 * kTile * KC * 2; }
+};
+using RouterCfg16 = RouterCfg<16, 8, 8, 256>;
+using RouterCfg8 = RouterCfg<8, 8, 16, 128>;
+constexpr int kRouterMinTile = 64;  // smallest tile of the configurations above
 
-__host__ __device__ constexpr int router_smem_bytes(int ES, int d) {
-    return d * (ES + 4) * 4 + 2 * kRouterTile * kRouterKc * 2;
-}
-
-template <int ES>
-__global__ void __launch_bounds__(kRouterWarps * 32, 1)
+template <class RC>
+__global__ void __launch_bounds__(RC::WARPS * 32, 1)
 router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
                           const float* __restrict__ b, float* __restrict__ logits, int T, int d,
                           int E, int32_t* __restrict__ hist, int hist_n,
                           int32_t* __restrict__ status) {
-    constexpr int TT = kRouterTile / kRouterWarps;  // tokens per warp
+    constexpr int ES = RC::ES;
+    constexpr int TT = RC::TT;                      // tokens per warp
+    constexpr int kRouterTile = RC::kTile;
+    constexpr int kRouterKc = RC::KC;
+    constexpr int kRouterWarps = RC::WARPS;
     constexpr int V = TT * ES;                      // values per lane
+    static_assert((kRouterTile * kRouterKc * 2 / 16) % (kRouterWarps * 32) == 0,
+                  "whole 16-byte pieces per thread and chunk");
     constexpr int WS = ES + 4;                      // padded W row (floats)
     static_assert(V % 32 == 0, "reduce-scatter needs a multiple of 32 values");
     extern __shared__ __align__(16) uint8_t rsm[];
@@ -446,7 +456,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
 // ---------------------------------------------------------------------------
 // per-device set-up of the shared-memory router: opt in to large dynamic
 // shared memory once per device and remember the SM count
-template <int ES>
+template <class RC>
 static cudaError_t router_smem_setup(int* num_sms) {
     static std::atomic<int> ready[64];
     static std::atomic<int> sms[64];
@@ -455,7 +465,7 @@ static cudaError_t router_smem_setup(int* num_sms) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (ready[dev].load(std::memory_order_acquire) == 0) {
-        e = cudaFuncSetAttribute(router_logits_smem_kernel<ES>,
+        e = cudaFuncSetAttribute(router_logits_smem_kernel<RC>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         int n = 0;
@@ -468,20 +478,20 @@ static cudaError_t router_smem_setup(int* num_sms) {
     return cudaSuccess;
 }
 
-template <int ES>
+template <class RC>
 static cudaError_t launch_router_smem(const uint16_t* x, const float* W, const float* b,
                                       float* logits, int T, int d, int E, int32_t* hist,
                                       int hist_n, int32_t* status, cudaStream_t st) {
-    const int smem = router_smem_bytes(ES, d);
+    const int smem = RC::smem_bytes(d);
     int num_sms = 0;
-    const cudaError_t e = router_smem_setup<ES>(&num_sms);
+    const cudaError_t e = router_smem_setup<RC>(&num_sms);
     if (e != cudaSuccess) return e;
-    const int nslices = E / ES;
-    const int ntiles = (T + kRouterTile - 1) / kRouterTile;
+    const int nslices = E / RC::ES;
+    const int ntiles = (T + RC::kTile - 1) / RC::kTile;
     int per_slice = num_sms / nslices;
     if (per_slice < 1) per_slice = 1;
     if (per_slice > ntiles) per_slice = ntiles;
-    router_logits_smem_kernel<ES><<<nslices * per_slice, kRouterWarps * 32, smem, st>>>(
+    router_logits_smem_kernel<RC><<<nslices * per_slice, RC::WARPS * 32, smem, st>>>(
         x, W, b, logits, T, d, E, hist, hist_n, status);
     return cudaGetLastError();
 }
@@ -490,11 +500,12 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float*
                                  float* logits, int T, int d, int E, int32_t* hist, int hist_n,
                                  int32_t* status, cudaStream_t st) {
     // batches of at least one tile per SM use the shared-memory kernel
-    if (T >= kRouterTile * 2) {
-        if (E % 16 == 0 && router_smem_bytes(16, d) <= 227 * 1024)
-            return launch_router_smem<16>(x, W, b, logits, T, d, E, hist, hist_n, status, st);
-        if (router_smem_bytes(8, d) <= 227 * 1024)
-            return launch_router_smem<8>(x, W, b, logits, T, d, E, hist, hist_n, status, st);
+    if (T >= kRouterMinTile * 2) {
+        if (E % 16 == 0 && RouterCfg16::smem_bytes(d) <= 227 * 1024)
+            return launch_router_smem<RouterCfg16>(x, W, b, logits, T, d, E, hist, hist_n, status,
+                                                   st);
+        if (RouterCfg8::smem_bytes(d) <= 227 * 1024)
+            return launch_router_smem<RouterCfg8>(x, W, b, logits, T, d, E, hist, hist_n, status, st);
     }
     const int ty = T > 0 ? (T + kLogitTokPerCta - 1) / kLogitTokPerCta : 1;
     if (E % 16 == 0) {
