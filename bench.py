@@ -36,6 +36,7 @@ import moe_inputs as mi  # noqa: E402
 METRIC = "MoE-layer prefill tokens/s (int4 fused grouped GEMM) and % of roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, down GEMM, combine
+KERNELS_PER_STEP_DECODE = 3  # routing cluster, gate/up, down + combine (batches of at most 8 tokens)
 
 
 def load_peaks():
@@ -284,17 +285,19 @@ def run_ours(args, name):
     layer_roof_s = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9))
     tensor_bound = work["flops_gateup"] / (peaks["bf16_tflops_sustained"] * 1e12) >= \
         work["bytes_gateup"] / (peaks["hbm_gbs"] * 1e9)
+    decode = layer.plan.forward_path(s.T) == 1
+    gu_kernel = "decode_gateup_kernel" if decode else "grouped_gemm_kernel<gate/up>"
     if tensor_bound:
         achieved = work["flops_gateup"] / t_gu / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
-                "traffic": TRAFFIC_GATEUP.get(name), "kernel": "grouped_gemm_kernel<gate/up>",
+                "traffic": TRAFFIC_GATEUP.get(name), "kernel": gu_kernel,
                 "peak_kind": "bf16 sustained, %s" % peaks["source"]}
     else:
         achieved = work["bytes_gateup"] / t_gu / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": TRAFFIC_GATEUP.get(name),
-                "kernel": "grouped_gemm_kernel<gate/up>", "peak_kind": "HBM copy, %s" % peaks["source"]}
+                "kernel": gu_kernel, "peak_kind": "HBM copy, %s" % peaks["source"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -318,7 +321,7 @@ def run_ours(args, name):
         "cpu_baseline": cpu,
         "e2e": {"value": world * s.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(s.T * s.d * 2), "d2h_bytes_per_step": int(s.T * s.d * 2)},
-        "gpu_launches": K * KERNELS_PER_STEP,
+        "gpu_launches": K * (KERNELS_PER_STEP_DECODE if decode else KERNELS_PER_STEP),
         "clocks": clk,
     }
     if rank == 0:
@@ -328,9 +331,10 @@ def run_ours(args, name):
         dist.destroy_process_group()
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one gate/up GEMM launch from
-# an ncu capture of the current kernel (profiles/); None until captured.
-TRAFFIC_GATEUP: dict = {}
+# dram__bytes_read.sum + dram__bytes_write.sum (bytes) of one gate/up GEMM
+# launch, from the ncu capture summarised in profiles/kernels_prefill_t8192.md;
+# workloads without a capture of the current kernel report None.
+TRAFFIC_GATEUP: dict = {"prefill_t8192": 584494848}
 
 
 def main():

@@ -257,6 +257,16 @@ MOE_API moe_status_t moe_route_noalloc(const moe_plan_t *plan, int32_t T,
 MOE_API moe_status_t moe_read_status(const void *ws, int32_t *code, int32_t *detail,
                              int32_t clear, void *stream);
 
+/*
+ * Which kernels moe_forward runs at batch T for this plan: 1 for the
+ * small-batch (decode) kernels, which stream the selected experts' weights
+ * (wpnews page "Perplexity Lily: 1.35x Faster Local AI Than MLX on Mac",
+ * section "Why MLX Falls Behind": prefill and decode are separate
+ * workloads), 0 for the batched grouped-GEMM kernels, -1 if plan is NULL or
+ * T is outside 0..T_max.  Host only; launches nothing.
+ */
+MOE_API int moe_forward_path(const moe_plan_t *plan, int32_t T);
+
 #ifdef __cplusplus
 }
 #endif

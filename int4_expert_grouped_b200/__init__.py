@@ -93,6 +93,8 @@ _lib.moe_route_noalloc.argtypes = [_P, ctypes.c_int32, _P, _P, _P, ctypes.POINTE
 _lib.moe_forward_host.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_read_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                  ctypes.c_int32, _P]
+_lib.moe_forward_path.argtypes = [_P, ctypes.c_int32]
+_lib.moe_forward_path.restype = ctypes.c_int
 for _fn in ("moe_plan_create", "moe_plan_info", "moe_prepack_weights", "moe_route",
             "moe_forward", "moe_forward_timed", "moe_forward_host", "moe_read_status",
             "moe_route_noalloc"):
@@ -100,7 +102,8 @@ for _fn in ("moe_plan_create", "moe_plan_info", "moe_prepack_weights", "moe_rout
 
 EXPORTED = ("moe_abi_version", "moe_status_str", "moe_plan_create", "moe_plan_info",
             "moe_plan_destroy", "moe_prepack_weights", "moe_route", "moe_forward",
-            "moe_forward_timed", "moe_forward_host", "moe_read_status", "moe_route_noalloc")
+            "moe_forward_timed", "moe_forward_host", "moe_read_status", "moe_route_noalloc",
+            "moe_forward_path")
 
 
 def abi_version() -> int:
@@ -200,6 +203,10 @@ class Plan:
         _check(_lib.moe_forward_host(self._h, T, ptr(x_host), ptr(w_r), ptr(b_r), ptr(packed_w),
                                      ptr(y_host), ptr(ws), ws.numel() * ws.element_size(),
                                      _stream_ptr(stream)), "moe_forward_host")
+
+    def forward_path(self, T: int) -> int:
+        """1 if moe_forward runs the small-batch kernels at batch T, 0 for the batched ones."""
+        return int(_lib.moe_forward_path(self._h, T))
 
     def read_status(self, ws, clear: bool = True, stream=None):
         code = ctypes.c_int32()

@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe):
     names = declared_functions()
-    assert len(names) == 12
+    assert len(names) == 13
     for n in names:
         assert hasattr(moe.lib(), n), n
     assert set(names) == set(moe.EXPORTED)
@@ -127,3 +127,14 @@ def test_prepack_and_host_checks(moe):
     H = p.info.host_workspace_bytes
     assert lib.moe_forward_host(p.handle, 64, 0x1000, 0x2000, None, 0x3000, 0x4000, 0x5000, H - 1, None) == 4
     assert lib.moe_forward_host(p.handle, 64, None, 0x2000, None, 0x3000, 0x4000, 0x5000, H, None) == 1
+
+
+def test_forward_path_choice(moe):
+    # host-only query: small batches of a supported shape take the decode kernels
+    p = moe.Plan(8192, 2048, 128, 8, 768, 64)
+    assert [p.forward_path(T) for T in (0, 1, 4, 8, 9, 8192)] == [0, 1, 1, 1, 0, 0]
+    assert p.forward_path(-1) == -1 and p.forward_path(8193) == -1
+    tiny = moe.Plan(64, 256, 8, 2, 128, 32)
+    assert tiny.forward_path(3) == 0  # E = 8: too few experts for the 8-CTA routing cluster
+    g32 = moe.Plan(64, 256, 32, 2, 128, 32)
+    assert g32.forward_path(3) == 1 and g32.forward_path(9) == 0
