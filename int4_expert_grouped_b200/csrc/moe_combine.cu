@@ -39,6 +39,8 @@ dispatch_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sort
     const int lane = threadIdx.x & 31;
     const int nv = d >> 3;  // 16-byte vectors per row
     const int warps = gridDim.x * (kThreads / 32);
+    pdl_launch_dependents();
+    pdl_wait();
     const uint4* x4 = reinterpret_cast<const uint4*>(x);
     uint4* xs4 = reinterpret_cast<uint4*>(xs);
     int p = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
@@ -98,6 +100,8 @@ combine_kernel(const uint16_t* __restrict__ o, const int32_t* __restrict__ pos,
     const int nv = d >> 3;
     const int Tk = T * k;
     const uint4* o4 = reinterpret_cast<const uint4*>(o);
+    pdl_launch_dependents();
+    pdl_wait();
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         __syncthreads();  // the previous token's slots are no longer read
         if (threadIdx.x < k) {
@@ -143,8 +147,8 @@ cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int
     const long need = (static_cast<long>(Tk) + kThreads / 32 - 1) / (kThreads / 32);
     const long cap = static_cast<long>(num_sms) * 8;  // 8 CTAs of 8 warps per SM
     const int grid = static_cast<int>(need < cap ? need : cap);
-    dispatch_kernel<<<grid, kThreads, 0, st>>>(x, sorted_assign, Tk, k, d, xs, status);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_kernel, dim3(grid), dim3(kThreads), 0, st, x, sorted_assign, Tk, k, d, xs,
+                      status);
 }
 
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T, int k,
@@ -152,8 +156,8 @@ cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* t
     if (T <= 0) return cudaSuccess;
     const long cap = static_cast<long>(num_sms) * 8;
     const int grid = static_cast<int>(T < cap ? T : cap);
-    combine_kernel<<<grid, kThreads, 0, st>>>(o, pos, topk_w, T, k, d, y, status);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, st, o, pos, topk_w, T, k, d, y,
+                      status);
 }
 
 }  // namespace moe

@@ -271,6 +271,20 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+// Lets the next kernel in the stream be scheduled once every CTA of this one
+// has started (its CTAs then wait in pdl_wait).
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the preceding kernel in the stream has completed and its memory
+// is visible (returns at once when launched without the attribute).  Every
+// kernel calls it before its first access to global data that another kernel
+// of the layer reads or writes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // int4 -> bf16 expansion of the prepacked weights (shared by the grouped GEMM
 // and the small-batch path, so both produce the same bf16 weights)
 // ---------------------------------------------------------------------------

@@ -46,12 +46,6 @@ constexpr int kDnWords = 4;         // nibble words per lane and down row: f <= 
 template <int kT>
 constexpr int dn_block_batch() { return kT <= 4 ? 8 : 4; }
 
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-// Waits until the preceding kernel in the stream has completed and its
-// memory is visible (returns at once when launched without the attribute).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     uint4 v;
@@ -239,8 +233,6 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     float* cs = ws + static_cast<size_t>(d) * (E / kRouteCtas);                  // [t][p][33]
     pdl_launch_dependents();
     const int rank = static_cast<int>(cluster.block_rank());
-    // the status word reports the most recent call: the first kernel clears it
-    if (rank == 0 && threadIdx.x < 2) status[threadIdx.x] = 0;
     const int EC = E / kRouteCtas;
     const int e0 = rank * EC;
     const int nsteps = d >> 5;
@@ -298,6 +290,11 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     }
     cluster.sync();  // all logits are in CTA 0; no CTA touches another's memory after this
     if (rank != 0) return;
+    // everything above reads only the layer's inputs; the outputs below are
+    // read by the previous call's kernels, which must have finished
+    pdl_wait();
+    // the status word reports the most recent call: the first kernel clears it
+    if (threadIdx.x < 2) status[threadIdx.x] = 0;
     route_from_logits(T, E, k, max_blocks, R);
     write_route(R, ro, T * k, E);
 }
@@ -495,21 +492,6 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
     }
 }
 
-template <typename Kern, typename... Args>
-cudaError_t launch_pdl(Kern kernel, dim3 grid, int threads, size_t smem, cudaStream_t st,
-                       Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
 
 constexpr size_t kDecodeSmemLimit = 96 * 1024;
 constexpr size_t kRouteSmemLimit = 200 * 1024;
@@ -582,9 +564,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed,
     const DecodeRouteOut ro{a.topk_idx, a.topk_w,        a.counts,    a.offsets,   a.sorted_assign,
                             a.pos,      a.block_offsets, a.block_map, a.num_blocks};
     const size_t route_smem = route_smem_bytes(s, T);
-    decode_route_kernel<<<kRouteCtas, kRowThreads, route_smem, st>>>(
-        a.x, a.W_r, a.b_r, T, s.d, s.E, s.k, a.max_blocks, ro, a.status);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(decode_route_kernel, dim3(kRouteCtas), dim3(kRowThreads), route_smem, st,
+                               a.x, a.W_r, a.b_r, T, s.d, s.E, s.k, a.max_blocks, ro, a.status);
     if (e != cudaSuccess) return e;
     if (ev_routed && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_routed), st)) != cudaSuccess)
         return e;

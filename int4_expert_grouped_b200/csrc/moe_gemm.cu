@@ -136,6 +136,7 @@ template <bool kDown>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
     using C = Cfg<kDown>;
     extern __shared__ uint8_t smem_raw[];
+    pdl_launch_dependents();
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the block map, the token rows and (down) h come from earlier kernels
 
     const int NT = a.NT;
     const int KC = a.K / kKChunk;
@@ -586,10 +588,10 @@ static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaSt
     if (a.max_units <= 0) return cudaSuccess;
     const int grid = a.max_units < num_sms ? a.max_units : num_sms;
     if (down)
-        grouped_gemm_kernel<true><<<grid, kGemmThreads, Cfg<true>::kSmemBytes, st>>>(a);
-    else
-        grouped_gemm_kernel<false><<<grid, kGemmThreads, Cfg<false>::kSmemBytes, st>>>(a);
-    return cudaGetLastError();
+        return launch_pdl(grouped_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads),
+                          Cfg<true>::kSmemBytes, st, a);
+    return launch_pdl(grouped_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), Cfg<false>::kSmemBytes,
+                      st, a);
 }
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st) {

@@ -28,6 +28,24 @@ struct moe_plan {
 
 namespace moe {
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while its predecessor in the stream finishes, and waits for it in pdl_wait.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr int kMaxExperts = 256;  // experts per layer the routing kernels hold
 constexpr int kMaxTopk = 32;      // one warp lane per selected expert
 constexpr int kRouteGroupT = 256; // tokens per scatter group (one histogram row)

@@ -43,6 +43,8 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
     static_assert(V % 32 == 0, "reduce-scatter needs a multiple of 32 values");
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (blockIdx.x == 0 && blockIdx.y == 0) {
         for (int i = threadIdx.x; i < hist_n; i += blockDim.x) hist[i] = 0;
@@ -178,16 +180,19 @@ router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restric
     const int ctas = gridDim.x / nslices;
     const int e0 = slice * ES;
 
-    if (blockIdx.x == 0) {
-        for (int i = threadIdx.x; i < hist_n; i += blockDim.x) hist[i] = 0;
-        if (threadIdx.x < 2) status[threadIdx.x] = 0;
-    }
-    // the W_r slice, row i -> Ws[i * WS .. + ES)
+    pdl_launch_dependents();
+    // the W_r slice, row i -> Ws[i * WS .. + ES) (an input: loaded while the
+    // previous kernel in the stream finishes)
     for (int idx = threadIdx.x; idx < d * (ES / 4); idx += blockDim.x) {
         const int i = idx / (ES / 4);
         const int q = idx % (ES / 4);
         const float4 v = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) + q);
         *reinterpret_cast<float4*>(Ws + i * WS + 4 * q) = v;
+    }
+    pdl_wait();
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < hist_n; i += blockDim.x) hist[i] = 0;
+        if (threadIdx.x < 2) status[threadIdx.x] = 0;
     }
     __syncthreads();
 
@@ -308,6 +313,8 @@ router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                    int32_t* __restrict__ hist) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    pdl_launch_dependents();
+    pdl_wait();
     const int t = blockIdx.x * kTopkWarps + warp;
     if (t >= T) return;
     int my_id;
@@ -338,6 +345,8 @@ route_scan_kernel(const int32_t* __restrict__ hist, int ng, int E, int BT,
                   int32_t* __restrict__ block_map, int32_t* __restrict__ num_blocks,
                   int max_blocks, int32_t* status) {
     __shared__ int sh_warp[kScanThreads / 32 + 1];
+    pdl_launch_dependents();
+    pdl_wait();
     const int e = threadIdx.x;
     int c = 0;
     if (e < E)
@@ -395,6 +404,8 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
     __shared__ int cnt[kScatterWarps][kMaxExperts];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    pdl_launch_dependents();
+    pdl_wait();
     const int g = blockIdx.x;
     const long total = static_cast<long>(T) * k;
     const long a_begin = static_cast<long>(g) * kRouteGroupT * k;
@@ -491,9 +502,8 @@ static cudaError_t launch_router_smem(const uint16_t* x, const float* W, const f
     int per_slice = num_sms / nslices;
     if (per_slice < 1) per_slice = 1;
     if (per_slice > ntiles) per_slice = ntiles;
-    router_logits_smem_kernel<RC><<<nslices * per_slice, RC::WARPS * 32, smem, st>>>(
-        x, W, b, logits, T, d, E, hist, hist_n, status);
-    return cudaGetLastError();
+    return launch_pdl(router_logits_smem_kernel<RC>, dim3(nslices * per_slice), dim3(RC::WARPS * 32),
+                      smem, st, x, W, b, logits, T, d, E, hist, hist_n, status);
 }
 
 cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float* b,
@@ -508,34 +518,27 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float*
             return launch_router_smem<RouterCfg8>(x, W, b, logits, T, d, E, hist, hist_n, status, st);
     }
     const int ty = T > 0 ? (T + kLogitTokPerCta - 1) / kLogitTokPerCta : 1;
-    if (E % 16 == 0) {
-        dim3 grid(E / 16, ty);
-        router_logits_kernel<16><<<grid, kLogitWarps * 32, 0, st>>>(x, W, b, logits, T, d, E,
-                                                                    hist, hist_n, status);
-    } else {
-        dim3 grid(E / 8, ty);
-        router_logits_kernel<8><<<grid, kLogitWarps * 32, 0, st>>>(x, W, b, logits, T, d, E,
-                                                                   hist, hist_n, status);
-    }
-    return cudaGetLastError();
+    if (E % 16 == 0)
+        return launch_pdl(router_logits_kernel<16>, dim3(E / 16, ty), dim3(kLogitWarps * 32), 0, st,
+                          x, W, b, logits, T, d, E, hist, hist_n, status);
+    return launch_pdl(router_logits_kernel<8>, dim3(E / 8, ty), dim3(kLogitWarps * 32), 0, st, x, W,
+                      b, logits, T, d, E, hist, hist_n, status);
 }
 
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
                                float* topk_w, int32_t* hist, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int grid = (T + kTopkWarps - 1) / kTopkWarps;
-    router_topk_kernel<<<grid, kTopkWarps * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_w, hist);
-    return cudaGetLastError();
+    return launch_pdl(router_topk_kernel, dim3(grid), dim3(kTopkWarps * 32), 0, st, logits, T, E, k,
+                      topk_idx, topk_w, hist);
 }
 
 cudaError_t launch_route_scan(const int32_t* hist, int ng, int E, int BT, int32_t* counts,
                               int32_t* offsets, int32_t* gbase, int32_t* block_offsets,
                               int32_t* block_map, int32_t* num_blocks, int max_blocks,
                               int32_t* status, cudaStream_t st) {
-    route_scan_kernel<<<1, kScanThreads, 0, st>>>(hist, ng, E, BT, counts, offsets, gbase,
-                                                  block_offsets, block_map, num_blocks,
-                                                  max_blocks, status);
-    return cudaGetLastError();
+    return launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, hist, ng, E, BT, counts,
+                      offsets, gbase, block_offsets, block_map, num_blocks, max_blocks, status);
 }
 
 cudaError_t launch_route_scatter(const int32_t* topk_idx, const int32_t* gbase, int T, int k,
@@ -543,9 +546,8 @@ cudaError_t launch_route_scatter(const int32_t* topk_idx, const int32_t* gbase, 
                                  cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int ng = (T + kRouteGroupT - 1) / kRouteGroupT;
-    route_scatter_kernel<<<ng, kScatterWarps * 32, 0, st>>>(topk_idx, gbase, T, k, E, sorted_assign,
-                                                          pos, status);
-    return cudaGetLastError();
+    return launch_pdl(route_scatter_kernel, dim3(ng), dim3(kScatterWarps * 32), 0, st, topk_idx,
+                      gbase, T, k, E, sorted_assign, pos, status);
 }
 
 }  // namespace moe
