@@ -156,8 +156,8 @@ cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* t
     if (T <= 0) return cudaSuccess;
     const long cap = static_cast<long>(num_sms) * 8;
     const int grid = static_cast<int>(T < cap ? T : cap);
-    return launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, st, o, pos, topk_w, T, k, d, y,
-                      status);
+    combine_kernel<<<grid, kThreads, 0, st>>>(o, pos, topk_w, T, k, d, y, status);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -587,11 +587,13 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
 static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaStream_t st) {
     if (a.max_units <= 0) return cudaSuccess;
     const int grid = a.max_units < num_sms ? a.max_units : num_sms;
+    // Plain launches: letting the next kernel's CTAs be scheduled early measured
+    // slower around the GEMMs (their pdl_wait then returns at once).
     if (down)
-        return launch_pdl(grouped_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads),
-                          Cfg<true>::kSmemBytes, st, a);
-    return launch_pdl(grouped_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), Cfg<false>::kSmemBytes,
-                      st, a);
+        grouped_gemm_kernel<true><<<grid, kGemmThreads, Cfg<true>::kSmemBytes, st>>>(a);
+    else
+        grouped_gemm_kernel<false><<<grid, kGemmThreads, Cfg<false>::kSmemBytes, st>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st) {
