@@ -39,8 +39,8 @@ namespace {
 constexpr int kDecodeMaxAssign = kDecodeMaxT * kMaxTopk;
 constexpr int kRouteCtas = 8;       // cluster size of the routing kernel: E/8 experts each
 constexpr int kRowThreads = 512;    // 16 warps, one weight row each
-constexpr int kGuWords = 8;         // nibble words per lane and gate/up row: d <= 2048
-constexpr int kDnWords = 4;         // nibble words per lane and down row: f <= 1024
+constexpr int kGuVecs = 2;          // 16-byte nibble vectors per lane and gate/up row: d <= 2048
+constexpr int kDnVecs = 1;          // 16-byte nibble vectors per lane and down row: f <= 1024
 // experts whose down loads a lane issues together (fewer for larger batches,
 // whose operand loops need the registers)
 template <int kT>
@@ -91,6 +91,35 @@ __device__ __forceinline__ void cta_copy16(void* dst, const void* src, int n) {
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             if (i0 + u * stride < n) d[i0 + u * stride] = v[u];
+    }
+}
+
+// Copy rows of bf16 operands into shared memory with each row's 16-byte
+// pieces reordered: piece v = 4q + w (K 32q + 8w .. + 7) goes to slot
+// w * nvec + q, so the lanes of a warp, which own consecutive vectors q and
+// read piece w of each at the same time, touch consecutive 16-byte slots.
+// nvec = row length / 32; n_rows rows of 4 * nvec pieces.
+__device__ __forceinline__ void cta_copy_rows_by_vector(void* dst, const void* src, int n_rows,
+                                                        int nvec) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    const int per_row = 4 * nvec;
+    const int n = n_rows * per_row;
+    const int stride = blockDim.x;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u * stride < n) v[u] = ld_nc_v4(s + i0 + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * stride;
+            if (i < n) {
+                const int r = i / per_row;
+                const int pv = i - r * per_row;
+                d[r * per_row + (pv & 3) * nvec + (pv >> 2)] = v[u];
+            }
+        }
     }
 }
 
@@ -302,48 +331,54 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
 // ---------------------------------------------------------------------------
 // One packed weight row against kT bf16 operand rows, by one warp.  The row
 // lives in blocks base + c * chunk_stride (one per 64-wide K chunk c) at
-// packed row prow; nibble word w (K 8w .. 8w+7) is word w % 8 of chunk w / 8,
-// its (scale, bias) pair the row's entry for the group holding that half of
-// the chunk.  Lane l owns words l, l + 32, ... (< nw): row_load issues all
-// their loads at once; row_dots expands each word once and dots it with
-// every operand row into the lane's acc[i].
+// packed row prow: 32 bytes of nibbles per chunk, then the (scale, bias)
+// entries.  Vector q (16 bytes, K 32q .. 32q+31) is half q % 2 of chunk q / 2;
+// its (scale, bias) pair is the row's entry for the group holding that half.
+// Lane l owns vectors l, l + 32, ... (< nv): row_load issues all their loads
+// at once; row_dots expands each vector once and dots it with every operand
+// row (stored by cta_copy_rows_by_vector) into the lane's acc[i].
 // ---------------------------------------------------------------------------
-template <int kW>
+template <int kV>
 struct RowLoads {
-    uint32_t nib[kW];
-    uint32_t sb[kW];
+    uint4 nib[kV];
+    uint32_t sb[kV];
 };
 
-template <int kW>
-__device__ __forceinline__ void row_load(RowLoads<kW>& L, const uint8_t* __restrict__ base,
+template <int kV>
+__device__ __forceinline__ void row_load(RowLoads<kV>& L, const uint8_t* __restrict__ base,
                                          size_t chunk_stride, int prow, int nib_bytes, int gpc,
-                                         int nw, int lane) {
+                                         int nv, int lane) {
 #pragma unroll
-    for (int u = 0; u < kW; ++u) {
-        const int w = lane + 32 * u;
-        if (w < nw) {
-            const uint8_t* blk = base + static_cast<size_t>(w >> 3) * chunk_stride;
-            const int wi = w & 7;
-            L.nib[u] = ld_nc_u32(blk + prow * 32 + wi * 4);
-            L.sb[u] = ld_nc_u32(blk + nib_bytes + (prow * gpc + (wi >> 2) * (gpc - 1)) * 4);
+    for (int u = 0; u < kV; ++u) {
+        const int q = lane + 32 * u;
+        if (q < nv) {
+            const uint8_t* blk = base + static_cast<size_t>(q >> 1) * chunk_stride;
+            const int half = q & 1;
+            L.nib[u] = ld_nc_v4(blk + prow * 32 + half * 16);
+            L.sb[u] = ld_nc_u32(blk + nib_bytes + (prow * gpc + half * (gpc - 1)) * 4);
         }
     }
 }
 
-template <int kT, int kW>
-__device__ __forceinline__ void row_dots(const RowLoads<kW>& L, const uint16_t* const* rows, int nw,
+template <int kT, int kV>
+__device__ __forceinline__ void row_dots(const RowLoads<kV>& L, const uint16_t* const* rows, int nv,
                                          int lane, float* acc) {
 #pragma unroll
-    for (int u = 0; u < kW; ++u) {
-        const int w = lane + 32 * u;
-        if (w < nw) {
+    for (int u = 0; u < kV; ++u) {
+        const int q = lane + 32 * u;
+        if (q < nv) {
             BF2 s2, b2;
             s2.u = __byte_perm(L.sb[u], 0, 0x1010);
             b2.u = __byte_perm(L.sb[u], 0, 0x3232);
-            const uint4 wv = expand8(L.nib[u], s2.h, b2.h);
+            const uint32_t words[4] = {L.nib[u].x, L.nib[u].y, L.nib[u].z, L.nib[u].w};
 #pragma unroll
-            for (int i = 0; i < kT; ++i)
-                acc[i] = dot8(wv, *reinterpret_cast<const uint4*>(rows[i] + 8 * w), acc[i]);
+            for (int wi = 0; wi < 4; ++wi) {
+                const uint4 wv = expand8(words[wi], s2.h, b2.h);  // K 32q + 8wi .. + 7
+#pragma unroll
+                for (int i = 0; i < kT; ++i)
+                    acc[i] = dot8(wv, *reinterpret_cast<const uint4*>(rows[i] + 8 * (wi * nv + q)),
+                                  acc[i]);
+            }
         }
     }
 }
@@ -369,7 +404,7 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
     extern __shared__ __align__(16) uint8_t dsm[];
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(dsm);
     pdl_launch_dependents();
-    cta_copy16(dsm, x, kT * d / 8);  // x does not depend on the routing kernel
+    cta_copy_rows_by_vector(dsm, x, kT, d / 32);  // x does not depend on the routing kernel
     pdl_wait();
     const int nq = f / 16;
     const int b = blockIdx.x / nq;
@@ -391,9 +426,9 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
     const int KC = d / kKChunk;
     const int gpc = kKChunk / group;
     const uint8_t* base = wpack + (static_cast<size_t>(sblk[0]) * NT + j) * KC * bb;
-    RowLoads<kGuWords> Lg, Lu;
-    row_load(Lg, base, bb, feat, 2 * 128 * 32, gpc, d / 8, lane);
-    row_load(Lu, base, bb, 128 + feat, 2 * 128 * 32, gpc, d / 8, lane);
+    RowLoads<kGuVecs> Lg, Lu;
+    row_load(Lg, base, bb, feat, 2 * 128 * 32, gpc, d / 32, lane);
+    row_load(Lu, base, bb, 128 + feat, 2 * 128 * 32, gpc, d / 32, lane);
     const uint16_t* rows[kT];
     float ag[kT], au[kT];
 #pragma unroll
@@ -402,8 +437,8 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
         ag[i] = 0.0f;
         au[i] = 0.0f;
     }
-    row_dots<kT>(Lg, rows, d / 8, lane, ag);
-    row_dots<kT>(Lu, rows, d / 8, lane, au);
+    row_dots<kT>(Lg, rows, d / 32, lane, ag);
+    row_dots<kT>(Lu, rows, d / 32, lane, au);
 #pragma unroll
     for (int i = 0; i < kT; ++i) {
         const float gv = warp_sum(ag[i]);
@@ -444,7 +479,7 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
         sw[i] = ro.topk_w[i];
     }
     for (int i = threadIdx.x; i < 3 * nb_max; i += blockDim.x) sbm[i] = ro.block_map[i];
-    cta_copy16(dsm, h, Tk * f / 8);
+    cta_copy_rows_by_vector(dsm, h, Tk, f / 32);
     __syncthreads();
     const int nb = snb;
     const int m = blockIdx.x * 16 + warp;
@@ -452,15 +487,15 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
     const int prow = m % (128 * kDownTiles);
     const int NTd = d / (128 * kDownTiles);
     const int KCd = f / kKChunk;
-    const int nw = f / 8;
+    const int nv = f / 32;  // 16-byte nibble vectors per down row
     constexpr int kDnBlockBatch = dn_block_batch<kT>();
     for (int b0 = 0; b0 < nb; b0 += kDnBlockBatch) {
-        RowLoads<kDnWords> L[kDnBlockBatch];
+        RowLoads<kDnVecs> L[kDnBlockBatch];
 #pragma unroll
         for (int u = 0; u < kDnBlockBatch; ++u)
             if (b0 + u < nb)
                 row_load(L[u], wpack + (static_cast<size_t>(sbm[3 * (b0 + u)]) * NTd + jd) * KCd * bb,
-                         bb, prow, 128 * kDownTiles * 32, kKChunk / group, nw, lane);
+                         bb, prow, 128 * kDownTiles * 32, kKChunk / group, nv, lane);
 #pragma unroll
         for (int u = 0; u < kDnBlockBatch; ++u) {
             if (b0 + u < nb) {
@@ -473,7 +508,7 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
                     rows[i] = hs + static_cast<size_t>(brow0 + min(i, brows - 1)) * f;
                     acc[i] = 0.0f;
                 }
-                row_dots<kT>(L[u], rows, nw, lane, acc);
+                row_dots<kT>(L[u], rows, nv, lane, acc);
 #pragma unroll
                 for (int i = 0; i < kT; ++i) {
                     const float v = warp_sum(acc[i]);
@@ -535,8 +570,8 @@ bool decode_supported(const moe_shape_t& s, int T) {
     if (T * s.k > kDecodeMaxAssign || s.E > kMaxExperts) return false;
     // whole 16-byte vectors of W_r columns per routing CTA
     if (s.E % (4 * kRouteCtas) != 0 || route_smem_bytes(s, T) > kRouteSmemLimit) return false;
-    // nibble words (8 K values each) per lane and row
-    if (s.d > 8 * 32 * kGuWords || s.f > 8 * 32 * kDnWords) return false;
+    // 16-byte nibble vectors (32 K values each) per lane and row
+    if (s.d > 32 * 32 * kGuVecs || s.f > 32 * 32 * kDnVecs) return false;
     const size_t x_bytes = static_cast<size_t>(T) * s.d * 2;
     const size_t h_bytes = static_cast<size_t>(T) * s.k * s.f * 2;
     return x_bytes <= kDecodeSmemLimit && h_bytes <= kDecodeSmemLimit;

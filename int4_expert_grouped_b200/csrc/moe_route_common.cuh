@@ -83,9 +83,14 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, 
 // come before it in the order (logit descending, id ascending).  The experts
 // with slot < k are exactly the ones warp_topk selects, in the same order.
 __device__ __forceinline__ int expert_slot(const float* __restrict__ row, int E, int e) {
-    const Cand me{row[e], e};
+    // better(Cand{u, e2}, Cand{v, e}) for two valid ids, without branches
+    const float v = row[e];
     int r = 0;
-    for (int e2 = 0; e2 < E; ++e2) r += better(Cand{row[e2], e2}, me);
+#pragma unroll 8
+    for (int e2 = 0; e2 < E; ++e2) {
+        const float u = row[e2];
+        r += (u > v) | ((u == v) & (e2 < e));
+    }
     return r;
 }
 
