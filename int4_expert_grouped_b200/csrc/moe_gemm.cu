@@ -435,28 +435,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                             p[h][i] = o.u;
                         }
                 } else {
-                    // gate and up of one lane half per wait (64 registers)
+                    // gate and up of both lane halves in flight before one wait
+                    uint32_t v[2][16], uu[2][16];
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        uint32_t v[16], uu[16];
                         const uint32_t ta = tb + (static_cast<uint32_t>(16 * h) << 16) + cb * 32;
-                        tmem_ld_16x256b_x4(ta, v);
-                        tmem_ld_16x256b_x4(ta + kBlockT, uu);
-                        tmem_ld_wait();
-                        float hv[16];
+                        tmem_ld_16x256b_x4(ta, v[h]);
+                        tmem_ld_16x256b_x4(ta + kBlockT, uu[h]);
+                    }
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float gv = __uint_as_float(v[i]);
-                            const float uv = __uint_as_float(uu[i]);
-                            hv[i] = __fdividef(gv * uv, 1.0f + __expf(-gv));
-                        }
+                    for (int h = 0; h < 2; ++h)
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
+                            float hv[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float gv = __uint_as_float(v[h][2 * i + e]);
+                                const float uv = __uint_as_float(uu[h][2 * i + e]);
+                                hv[e] = __fdividef(gv * uv, 1.0f + __expf(-gv));
+                            }
                             BF2 o;
-                            o.h = __floats2bfloat162_rn(hv[2 * i], hv[2 * i + 1]);
+                            o.h = __floats2bfloat162_rn(hv[0], hv[1]);
                             p[h][i] = o.u;
                         }
-                    }
+                }
+                if (it == kOutTiles * ncb - 1) {
+                    // every TMEM read of this unit has completed: hand the
+                    // accumulator back to the MMA warp before the last stores
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(accempty(buf));
                 }
                 // token group g (8 tokens): matrices (h, octet) = registers
                 // p[h][2g] (features 16h + 0..7) and p[h][2g+1] (16h + 8..15)
@@ -478,9 +487,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 }
                 __syncwarp();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(accempty(buf));
+            if (ncb == 0) {  // a block always has rows; keep the hand-back unconditional
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accempty(buf));
+            }
         }
     }
 
