@@ -14,9 +14,10 @@
 //                          shared memory; CTA 0 then does top-k, counts,
 //                          scan, block map and scatter and writes them out
 //   decode_gateup_kernel   one warp per weight row (8 gate and 8 up rows per
-//                          CTA) streams its int4 row, expands it with the
-//                          GEMM's int4 -> bf16 code and dots it with the
-//                          block's x rows; SwiGLU gives bf16 rows of h
+//                          CTA) streams its int4 row and dots it with the
+//                          block's x rows, group by group (scale and bias
+//                          applied to each group's sum); SwiGLU gives bf16
+//                          rows of h
 //   decode_down_kernel     one warp per output feature (16 per CTA): the down
 //                          row of every selected expert against that expert's
 //                          h rows, each output rounded to bf16, then the
@@ -25,8 +26,11 @@
 // The expert kernels are instantiated per batch size, so their loops over the
 // batch's rows are fully unrolled without dead code.  The weights are read in
 // the prepacked block layout of the batched path, so one packed copy serves
-// both.  Rounding matches the batched path: bf16 weights, fp32 sums, bf16 h,
-// bf16 expert outputs, fp32 slot-order combine.
+// both.  Rounding differs from the batched path only in the weights: there
+// each dequantised weight is rounded to bf16 before the MMA, here the exact
+// codes meet the operands and each group's scale and bias apply to its fp32
+// sum (closer to the unrounded q*s + b).  Both keep fp32 sums, bf16 h, bf16
+// expert outputs and the fp32 slot-order combine.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -360,26 +364,74 @@ __device__ __forceinline__ void row_load(RowLoads<kV>& L, const uint8_t* __restr
     }
 }
 
+// Dot products of one packed row with every operand row, factored by group:
+// with w = q*s + b, sum_k w_k x_k over the vector's 32 K values (one group, or
+// half of a 64-wide group with the same s and b) is s * sum_k q_k x_k +
+// b * sum_k x_k.  The nibbles become fp32 128 + q exactly (q in mantissa
+// bits 16-19 of 128.0), pairs of them meet pairs of operands in packed fp32
+// FMAs, and 128 * sum_k x_k (sums: per row and vector) is taken off at the
+// end.  The weights are not rounded to bf16 on this path.
 template <int kT, int kV>
-__device__ __forceinline__ void row_dots(const RowLoads<kV>& L, const uint16_t* const* rows, int nv,
-                                         int lane, float* acc) {
+__device__ __forceinline__ void row_dots(const RowLoads<kV>& L, const uint16_t* const* rows,
+                                         const float* const* sums, int nv, int lane, float* acc) {
 #pragma unroll
     for (int u = 0; u < kV; ++u) {
         const int q = lane + 32 * u;
         if (q < nv) {
-            BF2 s2, b2;
-            s2.u = __byte_perm(L.sb[u], 0, 0x1010);
-            b2.u = __byte_perm(L.sb[u], 0, 0x3232);
+            const float s = __uint_as_float(L.sb[u] << 16);
+            const float b = __uint_as_float(L.sb[u] & 0xFFFF0000u);
+            float2 a2[kT];
+#pragma unroll
+            for (int t = 0; t < kT; ++t) a2[t] = make_float2(0.0f, 0.0f);
             const uint32_t words[4] = {L.nib[u].x, L.nib[u].y, L.nib[u].z, L.nib[u].w};
 #pragma unroll
             for (int wi = 0; wi < 4; ++wi) {
-                const uint4 wv = expand8(words[wi], s2.h, b2.h);  // K 32q + 8wi .. + 7
+                const uint32_t w = words[wi];  // K 32q + 8wi + 2i (bits 4i), + 2i + 1 (bits 16+4i)
+                float2 wp[4];
 #pragma unroll
-                for (int i = 0; i < kT; ++i)
-                    acc[i] = dot8(wv, *reinterpret_cast<const uint4*>(rows[i] + 8 * (wi * nv + q)),
-                                  acc[i]);
+                for (int i = 0; i < 4; ++i) {
+                    wp[i].x = __uint_as_float(((w << (16 - 4 * i)) & 0x000F0000u) | 0x43000000u);
+                    wp[i].y = __uint_as_float(((w >> (4 * i)) & 0x000F0000u) | 0x43000000u);
+                }
+#pragma unroll
+                for (int t = 0; t < kT; ++t) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(rows[t] + 8 * (wi * nv + q));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 xf = make_float2(__uint_as_float(xw[i] << 16),
+                                                      __uint_as_float(xw[i] & 0xFFFF0000u));
+                        a2[t] = __ffma2_rn(wp[i], xf, a2[t]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < kT; ++t) {
+                const float xs = sums[t][q];
+                acc[t] = fmaf(s, a2[t].x + a2[t].y - 128.0f * xs, fmaf(b, xs, acc[t]));
             }
         }
+    }
+}
+
+// sums[r * nvec + q] = sum of the 32 operand values of vector q of row r
+// (operand rows stored by cta_copy_rows_by_vector)
+__device__ __forceinline__ void cta_vector_sums(const uint16_t* rows, int n_rows, int nvec,
+                                                float* sums) {
+    for (int it = threadIdx.x; it < n_rows * nvec; it += blockDim.x) {
+        const int r = it / nvec;
+        const int q = it - r * nvec;
+        const uint16_t* row = rows + static_cast<size_t>(r) * nvec * 32;
+        float acc = 0.0f;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * (wi * nvec + q));
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc += __uint_as_float(vw[i] << 16) + __uint_as_float(vw[i] & 0xFFFF0000u);
+        }
+        sums[it] = acc;
     }
 }
 
@@ -401,10 +453,14 @@ __global__ void __launch_bounds__(kRowThreads)
 decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wpack, int d,
                      int k, int f, int group, int bb, DecodeRouteOut ro, uint16_t* __restrict__ h) {
     __shared__ int sblk[3 + kT];  // expert, first row, rows, token of each row
+    __shared__ float xsum[kT * 64];  // per token and 32-wide vector (d <= 2048)
     extern __shared__ __align__(16) uint8_t dsm[];
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(dsm);
     pdl_launch_dependents();
-    cta_copy_rows_by_vector(dsm, x, kT, d / 32);  // x does not depend on the routing kernel
+    // x does not depend on the routing kernel
+    cta_copy_rows_by_vector(dsm, x, kT, d / 32);
+    __syncthreads();
+    cta_vector_sums(xs, kT, d / 32, xsum);
     pdl_wait();
     const int nq = f / 16;
     const int b = blockIdx.x / nq;
@@ -430,15 +486,17 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
     row_load(Lg, base, bb, feat, 2 * 128 * 32, gpc, d / 32, lane);
     row_load(Lu, base, bb, 128 + feat, 2 * 128 * 32, gpc, d / 32, lane);
     const uint16_t* rows[kT];
+    const float* sums[kT];
     float ag[kT], au[kT];
 #pragma unroll
     for (int i = 0; i < kT; ++i) {
         rows[i] = xs + static_cast<size_t>(sblk[3 + i]) * d;
+        sums[i] = xsum + sblk[3 + i] * (d / 32);
         ag[i] = 0.0f;
         au[i] = 0.0f;
     }
-    row_dots<kT>(Lg, rows, d / 32, lane, ag);
-    row_dots<kT>(Lu, rows, d / 32, lane, au);
+    row_dots<kT>(Lg, rows, sums, d / 32, lane, ag);
+    row_dots<kT>(Lu, rows, sums, d / 32, lane, au);
 #pragma unroll
     for (int i = 0; i < kT; ++i) {
         const float gv = warp_sum(ag[i]);
@@ -455,7 +513,8 @@ decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__
 // kDownTiles) of down block (16m + r) / (128 * kDownTiles)).  For every block (expert) the warp dots that
 // expert's row with the block's h rows, rounds each sum to bf16 (the expert
 // output o), and after all blocks thread (t, r) sums o over token t's slots
-// in slot order.  Dynamic shared memory: h [kT*k][f] bf16.
+// in slot order.  Dynamic shared memory: h [kT*k][f] bf16, then the fp32 sums
+// of each h row's 32-wide vectors [kT*k][f/32].
 // ---------------------------------------------------------------------------
 template <int kT>
 __global__ void __launch_bounds__(kRowThreads)
@@ -481,6 +540,9 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
     for (int i = threadIdx.x; i < 3 * nb_max; i += blockDim.x) sbm[i] = ro.block_map[i];
     cta_copy_rows_by_vector(dsm, h, Tk, f / 32);
     __syncthreads();
+    float* hsum = reinterpret_cast<float*>(dsm + static_cast<size_t>(Tk) * f * 2);
+    cta_vector_sums(hs, Tk, f / 32, hsum);
+    __syncthreads();
     const int nb = snb;
     const int m = blockIdx.x * 16 + warp;
     const int jd = m / (128 * kDownTiles);
@@ -502,13 +564,16 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
                 const int brow0 = sbm[3 * (b0 + u) + 1];
                 const int brows = min(sbm[3 * (b0 + u) + 2], kT);
                 const uint16_t* rows[kT];
+                const float* sums[kT];
                 float acc[kT];
 #pragma unroll
                 for (int i = 0; i < kT; ++i) {
-                    rows[i] = hs + static_cast<size_t>(brow0 + min(i, brows - 1)) * f;
+                    const int p = brow0 + min(i, brows - 1);
+                    rows[i] = hs + static_cast<size_t>(p) * f;
+                    sums[i] = hsum + p * nv;
                     acc[i] = 0.0f;
                 }
-                row_dots<kT>(L[u], rows, nv, lane, acc);
+                row_dots<kT>(L[u], rows, sums, nv, lane, acc);
 #pragma unroll
                 for (int i = 0; i < kT; ++i) {
                     const float v = warp_sum(acc[i]);
@@ -528,8 +593,14 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
 }
 
 
-constexpr size_t kDecodeSmemLimit = 96 * 1024;
+constexpr size_t kDecodeSmemLimit = 112 * 1024;
 constexpr size_t kRouteSmemLimit = 200 * 1024;
+
+// gate/up: the batch's x rows; down: every assignment's h row and its vector sums
+size_t gateup_smem_bytes(const moe_shape_t& s, int T) { return static_cast<size_t>(T) * s.d * 2; }
+size_t down_smem_bytes(const moe_shape_t& s, int T) {
+    return static_cast<size_t>(T) * s.k * (static_cast<size_t>(s.f) * 2 + (s.f / 32) * 4);
+}
 
 size_t route_smem_bytes(const moe_shape_t& s, int T) {
     return static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(s.d) * (s.E / kRouteCtas) * 4 +
@@ -552,13 +623,13 @@ cudaError_t launch_experts(const DecodeArgs& a, const DecodeRouteOut& ro, cudaSt
     const moe_shape_t& s = a.s;
     const int nb_max = std::min(s.E, kT * s.k);
     cudaError_t e = launch_pdl(decode_gateup_kernel<kT>, dim3(nb_max * (s.f / 16)), kRowThreads,
-                               static_cast<size_t>(kT) * s.d * 2, st, a.x, a.wpack_gu, s.d, s.k,
+                               gateup_smem_bytes(s, kT), st, a.x, a.wpack_gu, s.d, s.k,
                                s.f, s.group, a.gu_block_bytes, ro, a.h);
     if (e != cudaSuccess) return e;
     if (ev_gate_up && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_gate_up), st)) != cudaSuccess)
         return e;
     return launch_pdl(decode_down_kernel<kT>, dim3(s.d / 16), kRowThreads,
-                      static_cast<size_t>(kT) * s.k * s.f * 2, st, a.wpack_dn,
+                      down_smem_bytes(s, kT), st, a.wpack_dn,
                       static_cast<const uint16_t*>(a.h), s.d, s.k, s.f, s.group, a.dn_block_bytes,
                       nb_max, ro, a.y);
 }
@@ -572,9 +643,7 @@ bool decode_supported(const moe_shape_t& s, int T) {
     if (s.E % (4 * kRouteCtas) != 0 || route_smem_bytes(s, T) > kRouteSmemLimit) return false;
     // 16-byte nibble vectors (32 K values each) per lane and row
     if (s.d > 32 * 32 * kGuVecs || s.f > 32 * 32 * kDnVecs) return false;
-    const size_t x_bytes = static_cast<size_t>(T) * s.d * 2;
-    const size_t h_bytes = static_cast<size_t>(T) * s.k * s.f * 2;
-    return x_bytes <= kDecodeSmemLimit && h_bytes <= kDecodeSmemLimit;
+    return gateup_smem_bytes(s, T) <= kDecodeSmemLimit && down_smem_bytes(s, T) <= kDecodeSmemLimit;
 }
 
 cudaError_t prepare_decode_kernels() {
