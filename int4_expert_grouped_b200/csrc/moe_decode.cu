@@ -13,18 +13,19 @@
 //                          butterfly tree and writes the logits into CTA 0's
 //                          shared memory; CTA 0 then does top-k, counts,
 //                          scan, block map and scatter and writes them out
-//   decode_gateup_kernel   one warp per weight row (8 gate and 8 up rows per
-//                          CTA) streams its int4 row and dots it with the
-//                          block's x rows, group by group (scale and bias
-//                          applied to each group's sum); SwiGLU gives bf16
-//                          rows of h
-//   decode_down_kernel     one warp per output feature (16 per CTA): the down
-//                          row of every selected expert against that expert's
-//                          h rows, each output rounded to bf16, then the
+//   decode_gateup_kernel   per (block, 8 features): the gate and up rows as
+//                          one 16-row tile of the warp-level tensor-core MMA
+//                          against the block's x rows (the MMA's 8 columns),
+//                          int4 codes unpacked straight into its registers;
+//                          each 32-wide vector's sum takes its group's scale
+//                          and bias; SwiGLU gives bf16 rows of h
+//   decode_down_kernel     per 16 output features: the same tile MMA for
+//                          every selected expert against that expert's h
+//                          rows, each output rounded to bf16, then the
 //                          routing-weighted sum over a token's slots in order
 //
-// The expert kernels are instantiated per batch size, so their loops over the
-// batch's rows are fully unrolled without dead code.  The weights are read in
+// The MMA's 8 columns hold a block's rows (one per token), so the instruction
+// count does not grow with the batch up to 8 tokens.  The weights are read in
 // the prepacked block layout of the batched path, so one packed copy serves
 // both.  Rounding differs from the batched path only in the weights: there
 // each dequantised weight is rounded to bf16 before the MMA, here the exact
@@ -42,13 +43,7 @@ namespace {
 
 constexpr int kDecodeMaxAssign = kDecodeMaxT * kMaxTopk;
 constexpr int kRouteCtas = 8;       // cluster size of the routing kernel: E/8 experts each
-constexpr int kRowThreads = 512;    // 16 warps, one weight row each
-constexpr int kGuVecs = 2;          // 16-byte nibble vectors per lane and gate/up row: d <= 2048
-constexpr int kDnVecs = 1;          // 16-byte nibble vectors per lane and down row: f <= 1024
-// experts whose down loads a lane issues together (fewer for larger batches,
-// whose operand loops need the registers)
-template <int kT>
-constexpr int dn_block_batch() { return kT <= 4 ? 8 : 4; }
+constexpr int kRowThreads = 512;    // threads of a routing CTA
 
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -62,23 +57,6 @@ __device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
     uint32_t v;
     asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
-}
-
-// sum of the 8 products of bf16 vectors w and x, added to acc
-__device__ __forceinline__ float dot8(const uint4& w, const uint4& x, float acc) {
-    const uint32_t wa[4] = {w.x, w.y, w.z, w.w};
-    const uint32_t xa[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        BF2 a, b;
-        a.u = wa[i];
-        b.u = xa[i];
-        const float2 af = __bfloat1622float2(a.h);
-        const float2 bf = __bfloat1622float2(b.h);
-        acc = fmaf(af.x, bf.x, acc);
-        acc = fmaf(af.y, bf.y, acc);
-    }
-    return acc;
 }
 
 // copy n 16-byte vectors global -> shared by the whole CTA, four loads in
@@ -95,35 +73,6 @@ __device__ __forceinline__ void cta_copy16(void* dst, const void* src, int n) {
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             if (i0 + u * stride < n) d[i0 + u * stride] = v[u];
-    }
-}
-
-// Copy rows of bf16 operands into shared memory with each row's 16-byte
-// pieces reordered: piece v = 4q + w (K 32q + 8w .. + 7) goes to slot
-// w * nvec + q, so the lanes of a warp, which own consecutive vectors q and
-// read piece w of each at the same time, touch consecutive 16-byte slots.
-// nvec = row length / 32; n_rows rows of 4 * nvec pieces.
-__device__ __forceinline__ void cta_copy_rows_by_vector(void* dst, const void* src, int n_rows,
-                                                        int nvec) {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
-    uint4* d = reinterpret_cast<uint4*>(dst);
-    const int per_row = 4 * nvec;
-    const int n = n_rows * per_row;
-    const int stride = blockDim.x;
-    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * stride) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (i0 + u * stride < n) v[u] = ld_nc_v4(s + i0 + u * stride);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * stride;
-            if (i < n) {
-                const int r = i / per_row;
-                const int pv = i - r * per_row;
-                d[r * per_row + (pv & 3) * nvec + (pv >> 2)] = v[u];
-            }
-        }
     }
 }
 
@@ -333,204 +282,242 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
 }
 
 // ---------------------------------------------------------------------------
-// One packed weight row against kT bf16 operand rows, by one warp.  The row
-// lives in blocks base + c * chunk_stride (one per 64-wide K chunk c) at
-// packed row prow: 32 bytes of nibbles per chunk, then the (scale, bias)
-// entries.  Vector q (16 bytes, K 32q .. 32q+31) is half q % 2 of chunk q / 2;
-// its (scale, bias) pair is the row's entry for the group holding that half.
-// Lane l owns vectors l, l + 32, ... (< nv): row_load issues all their loads
-// at once; row_dots expands each vector once and dots it with every operand
-// row (stored by cta_copy_rows_by_vector) into the lane's acc[i].
+// Expert GEMVs on the warp-level tensor-core MMA (m16n8k16, bf16 operands from
+// registers, fp32 accumulators).  A 16-row tile of packed weights is the A
+// operand and up to 8 operand rows (a block's tokens) are the 8 columns of B,
+// so the instruction count does not grow with the batch.
+//
+// Fragments (thread t of the warp: g = t / 4, c = t % 4): A holds rows g and
+// g + 8, logical K pairs c and c + 4; B holds column g, the same K pairs; the
+// accumulator holds rows g, g + 8 x columns 2c, 2c + 1.  Any one-to-one map of
+// the 16 logical K onto the data's K gives the same sum, so thread c takes word
+// c of a 32-wide nibble vector (K 8c .. 8c+7: nibble pair i is K 8c+2i at bits
+// 4i and 8c+2i+1 at bits 16+4i) for both of its rows: pairs 0 and 1 feed the
+// first MMA, pairs 2 and 3 the second, and its operand piece is the 16 bytes of
+// K 8c .. 8c+7 of its column.  A nibble pair becomes two bf16 values 128 + q
+// exactly (q in the mantissa of 128.0), so the MMA gives sum (128 + q) x; with
+// w = q s + b the vector's dot product is s * D + (b - 128 s) * sum x, formed
+// per vector in fp32 with the vector's group scale and bias.  The weights are
+// not rounded to bf16 on this path.
 // ---------------------------------------------------------------------------
-template <int kV>
-struct RowLoads {
-    uint4 nib[kV];
-    uint32_t sb[kV];
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// nibble pair i of a packed word as bf16 (128 + q_lo, 128 + q_hi)
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
+    return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+}
+
+// acc += dot products of one 32-wide vector: wa, wb = word c of the vector in
+// rows g and g + 8; xb = the column's operands K 8c .. 8c+7; sa, sb = the
+// rows' (scale, bias) words; xs0, xs1 = the vector sums of columns 2c, 2c + 1
+__device__ __forceinline__ void vector_mma(float (&acc)[4], uint32_t wa, uint32_t wb,
+                                           const uint4& xb, uint32_t sa, uint32_t sb, float xs0,
+                                           float xs1) {
+    float D[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    mma_16816(D, nib_pair(wa, 0), nib_pair(wb, 0), nib_pair(wa, 1), nib_pair(wb, 1), xb.x, xb.y);
+    mma_16816(D, nib_pair(wa, 2), nib_pair(wb, 2), nib_pair(wa, 3), nib_pair(wb, 3), xb.z, xb.w);
+    const float s0 = __uint_as_float(sa << 16);
+    const float s1 = __uint_as_float(sb << 16);
+    const float c0 = fmaf(-128.0f, s0, __uint_as_float(sa & 0xFFFF0000u));
+    const float c1 = fmaf(-128.0f, s1, __uint_as_float(sb & 0xFFFF0000u));
+    acc[0] = fmaf(s0, D[0], fmaf(c0, xs0, acc[0]));
+    acc[1] = fmaf(s0, D[1], fmaf(c0, xs1, acc[1]));
+    acc[2] = fmaf(s1, D[2], fmaf(c1, xs0, acc[2]));
+    acc[3] = fmaf(s1, D[3], fmaf(c1, xs1, acc[3]));
+}
+
+// Loads of one 16-row tile over a range of 64-wide K chunks: the tile's rows
+// g and g + 8 are packed rows pa and pb of blocks base + ch * bb; per chunk
+// word c of both halves of both rows, and the rows' (scale, bias) words.
+template <int kChunks, int kGpc>
+struct TileLoads {
+    uint32_t w[kChunks][4];         // row a half 0, row a half 1, row b half 0, row b half 1
+    uint32_t sc[kChunks][2 * kGpc];  // row a groups, row b groups
 };
 
-template <int kV>
-__device__ __forceinline__ void row_load(RowLoads<kV>& L, const uint8_t* __restrict__ base,
-                                         size_t chunk_stride, int prow, int nib_bytes, int gpc,
-                                         int nv, int lane) {
+template <int kChunks, int kGpc>
+__device__ __forceinline__ void tile_load(TileLoads<kChunks, kGpc>& L, const uint8_t* base, int bb,
+                                          int nib_bytes, int pa, int pb, int ch0, int ch_step,
+                                          int KC, int c) {
 #pragma unroll
-    for (int u = 0; u < kV; ++u) {
-        const int q = lane + 32 * u;
-        if (q < nv) {
-            const uint8_t* blk = base + static_cast<size_t>(q >> 1) * chunk_stride;
-            const int half = q & 1;
-            L.nib[u] = ld_nc_v4(blk + prow * 32 + half * 16);
-            L.sb[u] = ld_nc_u32(blk + nib_bytes + (prow * gpc + half * (gpc - 1)) * 4);
-        }
-    }
-}
-
-// Dot products of one packed row with every operand row, factored by group:
-// with w = q*s + b, sum_k w_k x_k over the vector's 32 K values (one group, or
-// half of a 64-wide group with the same s and b) is s * sum_k q_k x_k +
-// b * sum_k x_k.  The nibbles become fp32 128 + q exactly (q in mantissa
-// bits 16-19 of 128.0), pairs of them meet pairs of operands in packed fp32
-// FMAs, and 128 * sum_k x_k (sums: per row and vector) is taken off at the
-// end.  The weights are not rounded to bf16 on this path.
-template <int kT, int kV>
-__device__ __forceinline__ void row_dots(const RowLoads<kV>& L, const uint16_t* const* rows,
-                                         const float* const* sums, int nv, int lane, float* acc) {
+    for (int u = 0; u < kChunks; ++u) {
+        const int ch = ch0 + u * ch_step;
+        if (ch < KC) {
+            const uint8_t* blk = base + static_cast<size_t>(ch) * bb;
+            L.w[u][0] = ld_nc_u32(blk + pa * 32 + 4 * c);
+            L.w[u][1] = ld_nc_u32(blk + pa * 32 + 16 + 4 * c);
+            L.w[u][2] = ld_nc_u32(blk + pb * 32 + 4 * c);
+            L.w[u][3] = ld_nc_u32(blk + pb * 32 + 16 + 4 * c);
 #pragma unroll
-    for (int u = 0; u < kV; ++u) {
-        const int q = lane + 32 * u;
-        if (q < nv) {
-            const float s = __uint_as_float(L.sb[u] << 16);
-            const float b = __uint_as_float(L.sb[u] & 0xFFFF0000u);
-            float2 a2[kT];
-#pragma unroll
-            for (int t = 0; t < kT; ++t) a2[t] = make_float2(0.0f, 0.0f);
-            const uint32_t words[4] = {L.nib[u].x, L.nib[u].y, L.nib[u].z, L.nib[u].w};
-#pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-                const uint32_t w = words[wi];  // K 32q + 8wi + 2i (bits 4i), + 2i + 1 (bits 16+4i)
-                float2 wp[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    wp[i].x = __uint_as_float(((w << (16 - 4 * i)) & 0x000F0000u) | 0x43000000u);
-                    wp[i].y = __uint_as_float(((w >> (4 * i)) & 0x000F0000u) | 0x43000000u);
-                }
-#pragma unroll
-                for (int t = 0; t < kT; ++t) {
-                    const uint4 xv = *reinterpret_cast<const uint4*>(rows[t] + 8 * (wi * nv + q));
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 xf = make_float2(__uint_as_float(xw[i] << 16),
-                                                      __uint_as_float(xw[i] & 0xFFFF0000u));
-                        a2[t] = __ffma2_rn(wp[i], xf, a2[t]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < kT; ++t) {
-                const float xs = sums[t][q];
-                acc[t] = fmaf(s, a2[t].x + a2[t].y - 128.0f * xs, fmaf(b, xs, acc[t]));
+            for (int q = 0; q < kGpc; ++q) {
+                L.sc[u][q] = ld_nc_u32(blk + nib_bytes + (pa * kGpc + q) * 4);
+                L.sc[u][kGpc + q] = ld_nc_u32(blk + nib_bytes + (pb * kGpc + q) * 4);
             }
         }
     }
 }
 
-// sums[r * nvec + q] = sum of the 32 operand values of vector q of row r
-// (operand rows stored by cta_copy_rows_by_vector)
-__device__ __forceinline__ void cta_vector_sums(const uint16_t* rows, int n_rows, int nvec,
-                                                float* sums) {
-    for (int it = threadIdx.x; it < n_rows * nvec; it += blockDim.x) {
-        const int r = it / nvec;
-        const int q = it - r * nvec;
-        const uint16_t* row = rows + static_cast<size_t>(r) * nvec * 32;
+// acc += the tile's dot products over the loaded chunks.  xrow: the thread's
+// column in shared memory, advanced to K 8c; xs0, xs1: vector sums of columns
+// 2c and 2c + 1.
+template <int kChunks, int kGpc>
+__device__ __forceinline__ void tile_dots(float (&acc)[4], const TileLoads<kChunks, kGpc>& L,
+                                          const uint16_t* xrow, const float* xs0, const float* xs1,
+                                          int ch0, int ch_step, int KC) {
+#pragma unroll
+    for (int u = 0; u < kChunks; ++u) {
+        const int ch = ch0 + u * ch_step;
+        if (ch < KC) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int v = 2 * ch + hh;
+                const uint4 xb = *reinterpret_cast<const uint4*>(xrow + 32 * v);
+                const int q = kGpc == 2 ? hh : 0;
+                vector_mma(acc, L.w[u][hh], L.w[u][2 + hh], xb, L.sc[u][q], L.sc[u][kGpc + q],
+                           xs0[v], xs1[v]);
+            }
+        }
+    }
+}
+
+// Rows of bf16 operands (n_rows of w elements, row r at src row row_of(r))
+// into shared memory with a row stride of w + 32 elements (64 bytes of pad,
+// so the 8 columns' 16-byte reads fall in distinct banks), and each 32-wide
+// vector's sum (fp32, in K order) into sums [r][w/32].
+template <class RowOf>
+__device__ __forceinline__ void cta_stage_rows(uint16_t* dst, float* sums, const uint16_t* src,
+                                               int n_rows, int w, RowOf row_of) {
+    const int nv = w / 32;
+    for (int it = threadIdx.x; it < n_rows * nv; it += blockDim.x) {
+        const int r = it / nv;
+        const int v = it - r * nv;
+        const uint8_t* s = reinterpret_cast<const uint8_t*>(src + static_cast<size_t>(row_of(r)) * w + 32 * v);
+        uint4 p[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) p[q] = ld_nc_v4(s + 16 * q);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * (w + 32) + 32 * v);
         float acc = 0.0f;
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * (wi * nvec + q));
-            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        for (int q = 0; q < 4; ++q) {
+            d4[q] = p[q];
+            const uint32_t pw[4] = {p[q].x, p[q].y, p[q].z, p[q].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                acc += __uint_as_float(vw[i] << 16) + __uint_as_float(vw[i] & 0xFFFF0000u);
+            for (int i = 0; i < 4; ++i) {
+                acc += __uint_as_float(pw[i] << 16);
+                acc += __uint_as_float(pw[i] & 0xFFFF0000u);
+            }
         }
         sums[it] = acc;
     }
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-    return v;
-}
+constexpr int kGuWarps = 4;   // K split of a gate/up CTA
+constexpr int kGuChunks = 8;  // 64-wide K chunks per warp: d <= 4 * 8 * 64
+constexpr int kGuFeat = 8;    // features per gate/up CTA: 8 gate + 8 up rows, one MMA tile
+constexpr int kDnWarps = 16;  // blocks in flight per down CTA
+template <int kGpc>
+constexpr int dn_chunks() { return kGpc == 1 ? 8 : 6; }  // down K chunks loaded together
 
 // ---------------------------------------------------------------------------
-// Gate/up and SwiGLU for a batch of kT tokens.  Grid: min(E, kT*k) blocks x
-// f/16 feature slices (CTAs past the number of blocks return).  Warp r takes
-// feature 16q' + r of tile j: its gate row and its up row, so SwiGLU needs
-// no exchange between warps.  Rows of the block beyond its count repeat its
-// first row and are not stored.  Dynamic shared memory: x [kT][d].
+// Gate/up and SwiGLU.  Grid: min(E, T*k) blocks x f/8 feature groups (CTAs
+// past the number of blocks return).  The MMA tile's rows g and g + 8 are the
+// gate and up rows of feature 8q + g, so SwiGLU happens in the thread that
+// holds both sums.  The four warps split K; their sums are added in warp
+// order.  Columns beyond the block's rows repeat its last row and are not
+// stored.  Dynamic shared memory: the block's x rows [T][d + 32] bf16, then
+// their vector sums [T][d/32] fp32.
 // ---------------------------------------------------------------------------
-template <int kT>
-__global__ void __launch_bounds__(kRowThreads)
-decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wpack, int d,
-                     int k, int f, int group, int bb, DecodeRouteOut ro, uint16_t* __restrict__ h) {
-    __shared__ int sblk[3 + kT];  // expert, first row, rows, token of each row
-    __shared__ float xsum[kT * 64];  // per token and 32-wide vector (d <= 2048)
+template <int kGpc>
+__global__ void __launch_bounds__(kGuWarps * 32, kGpc == 1 ? 6 : 4)
+decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wpack, int T,
+                     int d, int k, int f, int bb, DecodeRouteOut ro, uint16_t* __restrict__ h) {
     extern __shared__ __align__(16) uint8_t dsm[];
-    const uint16_t* xs = reinterpret_cast<const uint16_t*>(dsm);
+    __shared__ float red[kGuWarps - 1][4][32];
     pdl_launch_dependents();
-    // x does not depend on the routing kernel
-    cta_copy_rows_by_vector(dsm, x, kT, d / 32);
-    __syncthreads();
-    cta_vector_sums(xs, kT, d / 32, xsum);
     pdl_wait();
-    const int nq = f / 16;
-    const int b = blockIdx.x / nq;
-    const int q = blockIdx.x - b * nq;
-    if (b >= min(ro.num_blocks[0], kDecodeMaxAssign)) return;
-    if (threadIdx.x < 3) sblk[threadIdx.x] = ro.block_map[3 * b + threadIdx.x];
-    __syncthreads();
-    const int row0 = sblk[1];
-    const int nrows = min(sblk[2], kT);
-    if (threadIdx.x < kT)
-        sblk[3 + threadIdx.x] =
-            ro.sorted_assign[row0 + min(static_cast<int>(threadIdx.x), nrows - 1)] / k;
-    __syncthreads();
+    const int nfq = f / kGuFeat;
+    const int b = blockIdx.x / nfq;
+    const int fq = blockIdx.x - b * nfq;
+    const int nb = ro.num_blocks[0];
+    const int e = ro.block_map[3 * b];
+    const int row0 = ro.block_map[3 * b + 1];
+    const int cnt = ro.block_map[3 * b + 2];
+    if (b >= min(nb, kDecodeMaxAssign)) return;
+    const int nrows = min(cnt, T);  // a block holds at most one row per token
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int j = q >> 3;
-    const int feat = (q & 7) * 16 + warp;  // feature within tile j
-    const int NT = f / 128;
+    const int g = lane >> 2;
+    const int c = lane & 3;
     const int KC = d / kKChunk;
-    const int gpc = kKChunk / group;
-    const uint8_t* base = wpack + (static_cast<size_t>(sblk[0]) * NT + j) * KC * bb;
-    RowLoads<kGuVecs> Lg, Lu;
-    row_load(Lg, base, bb, feat, 2 * 128 * 32, gpc, d / 32, lane);
-    row_load(Lu, base, bb, 128 + feat, 2 * 128 * 32, gpc, d / 32, lane);
-    const uint16_t* rows[kT];
-    const float* sums[kT];
-    float ag[kT], au[kT];
+    const int j = fq * kGuFeat / 128;
+    const int pa = fq * kGuFeat % 128 + g;  // gate row; the up row is 128 further
+    const uint8_t* base = wpack + (static_cast<size_t>(e) * (f / 128) + j) * KC * bb;
+    TileLoads<kGuChunks, kGpc> L;
+    tile_load(L, base, bb, 2 * 128 * 32, pa, 128 + pa, warp, kGuWarps, KC, c);
+    uint16_t* xsh = reinterpret_cast<uint16_t*>(dsm);
+    float* xss = reinterpret_cast<float*>(dsm + static_cast<size_t>(T) * (d + 32) * 2);
+    const int32_t* sa = ro.sorted_assign + row0;
+    cta_stage_rows(xsh, xss, x, nrows, d, [&](int r) { return sa[r] / k; });
+    __syncthreads();
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const int nv = d / 32;
+    tile_dots(acc, L, xsh + min(g, nrows - 1) * (d + 32) + 8 * c, xss + min(2 * c, nrows - 1) * nv,
+              xss + min(2 * c + 1, nrows - 1) * nv, warp, kGuWarps, KC);
+    if (warp > 0) {
 #pragma unroll
-    for (int i = 0; i < kT; ++i) {
-        rows[i] = xs + static_cast<size_t>(sblk[3 + i]) * d;
-        sums[i] = xsum + sblk[3 + i] * (d / 32);
-        ag[i] = 0.0f;
-        au[i] = 0.0f;
+        for (int i = 0; i < 4; ++i) red[warp - 1][i][lane] = acc[i];
     }
-    row_dots<kT>(Lg, rows, sums, d / 32, lane, ag);
-    row_dots<kT>(Lu, rows, sums, d / 32, lane, au);
+    __syncthreads();
+    if (warp != 0) return;
 #pragma unroll
-    for (int i = 0; i < kT; ++i) {
-        const float gv = warp_sum(ag[i]);
-        const float uv = warp_sum(au[i]);
-        if (lane == 0 && i < nrows)
-            h[static_cast<size_t>(row0 + i) * f + j * 128 + feat] =
+    for (int w = 0; w < kGuWarps - 1; ++w)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += red[w][i][lane];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r = 2 * c + i;
+        if (r < nrows) {
+            const float gv = acc[i];
+            const float uv = acc[2 + i];
+            h[static_cast<size_t>(row0 + r) * f + fq * kGuFeat + g] =
                 bf16_round_bits(__fdividef(gv * uv, 1.0f + __expf(-gv)));
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
-// Down projection and combine for a batch of kT tokens.  Grid: d/16 CTAs;
-// warp r of CTA m owns output feature 16m + r (row (16m + r) % (128 *
-// kDownTiles) of down block (16m + r) / (128 * kDownTiles)).  For every block (expert) the warp dots that
-// expert's row with the block's h rows, rounds each sum to bf16 (the expert
-// output o), and after all blocks thread (t, r) sums o over token t's slots
-// in slot order.  Dynamic shared memory: h [kT*k][f] bf16, then the fp32 sums
-// of each h row's 32-wide vectors [kT*k][f/32].
+// Down projection and combine.  Grid: d/16 CTAs; CTA m owns output features
+// 16m .. 16m+15 (one MMA tile: rows 16m % 128 + g and + 8 of down tile
+// 16m / 128).  The tile against a block's h rows gives each of the block's
+// assignments its 16 outputs.  With at most 8 blocks a pair of warps takes a
+// block, one K half each; otherwise warp w takes blocks w, w + 16, ... over
+// all of K.  The two halves' sums (the second is zero for a whole-K warp) are
+// added and rounded to bf16 (the expert output o), then thread (t, r) sums o
+// over token t's slots in slot order.  Dynamic shared memory: h [T*k][f + 32]
+// bf16, then its vector sums [T*k][f/32] fp32.
 // ---------------------------------------------------------------------------
-template <int kT>
-__global__ void __launch_bounds__(kRowThreads)
-decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict__ h, int d, int k,
-                   int f, int group, int bb, int nb_max, DecodeRouteOut ro,
+template <int kGpc>
+__global__ void __launch_bounds__(kDnWarps * 32, 1)
+decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict__ h, int T,
+                   int d, int k, int f, int bb, int nb_max, DecodeRouteOut ro,
                    uint16_t* __restrict__ y) {
     extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ int spos[kT * kMaxTopk];
-    __shared__ float sw[kT * kMaxTopk];
-    __shared__ int sbm[3 * kT * kMaxTopk];
-    __shared__ float os[kT * kMaxTopk][16];
+    __shared__ int spos[kDecodeMaxAssign];
+    __shared__ float sw[kDecodeMaxAssign];
+    __shared__ int sbm[3 * kDecodeMaxAssign];
+    __shared__ float op[2][kDecodeMaxAssign][16];  // K-half sums of each assignment's outputs
     __shared__ int snb;
-    const int Tk = kT * k;
-    const uint16_t* hs = reinterpret_cast<const uint16_t*>(dsm);
+    const int Tk = T * k;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    const int g = lane >> 2;
+    const int c = lane & 3;
     pdl_wait();  // h and the routing
     if (threadIdx.x == 0) snb = min(ro.num_blocks[0], nb_max);
     for (int i = threadIdx.x; i < Tk; i += blockDim.x) {
@@ -538,100 +525,103 @@ decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict
         sw[i] = ro.topk_w[i];
     }
     for (int i = threadIdx.x; i < 3 * nb_max; i += blockDim.x) sbm[i] = ro.block_map[i];
-    cta_copy_rows_by_vector(dsm, h, Tk, f / 32);
-    __syncthreads();
-    float* hsum = reinterpret_cast<float*>(dsm + static_cast<size_t>(Tk) * f * 2);
-    cta_vector_sums(hs, Tk, f / 32, hsum);
+    uint16_t* hsh = reinterpret_cast<uint16_t*>(dsm);
+    float* hss = reinterpret_cast<float*>(dsm + static_cast<size_t>(Tk) * (f + 32) * 2);
+    cta_stage_rows(hsh, hss, h, Tk, f, [](int r) { return r; });
     __syncthreads();
     const int nb = snb;
-    const int m = blockIdx.x * 16 + warp;
-    const int jd = m / (128 * kDownTiles);
-    const int prow = m % (128 * kDownTiles);
-    const int NTd = d / (128 * kDownTiles);
-    const int KCd = f / kKChunk;
-    const int nv = f / 32;  // 16-byte nibble vectors per down row
-    constexpr int kDnBlockBatch = dn_block_batch<kT>();
-    for (int b0 = 0; b0 < nb; b0 += kDnBlockBatch) {
-        RowLoads<kDnVecs> L[kDnBlockBatch];
+    const int m0 = blockIdx.x * 16;
+    const int jd = m0 / 128;
+    const int pa = m0 % 128 + g;
+    const int KC = f / kKChunk;
+    const int nv = f / 32;
+    constexpr int kCh = dn_chunks<kGpc>();
+    const int split = nb <= kDnWarps / 2 ? 2 : 1;
+    const int part = warp % split;
+    const int kc_part = (KC + split - 1) / split;
+    const int ch_begin = part * kc_part;
+    const int ch_end = min(KC, ch_begin + kc_part);
+    for (int b = warp / split; b < nb; b += kDnWarps / split) {
+        const int brow0 = sbm[3 * b + 1];
+        const int brows = min(sbm[3 * b + 2], T);
+        const uint8_t* base = wpack + (static_cast<size_t>(sbm[3 * b]) * (d / 128) + jd) * KC * bb;
+        const uint16_t* xrow = hsh + (brow0 + min(g, brows - 1)) * (f + 32) + 8 * c;
+        const float* xs0 = hss + (brow0 + min(2 * c, brows - 1)) * nv;
+        const float* xs1 = hss + (brow0 + min(2 * c + 1, brows - 1)) * nv;
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int ch0 = ch_begin; ch0 < ch_end; ch0 += kCh) {
+            TileLoads<kCh, kGpc> L;
+            tile_load(L, base, bb, 128 * 32, pa, pa + 8, ch0, 1, ch_end, c);
+            tile_dots(acc, L, xrow, xs0, xs1, ch0, 1, ch_end);
+        }
 #pragma unroll
-        for (int u = 0; u < kDnBlockBatch; ++u)
-            if (b0 + u < nb)
-                row_load(L[u], wpack + (static_cast<size_t>(sbm[3 * (b0 + u)]) * NTd + jd) * KCd * bb,
-                         bb, prow, 128 * kDownTiles * 32, kKChunk / group, nv, lane);
-#pragma unroll
-        for (int u = 0; u < kDnBlockBatch; ++u) {
-            if (b0 + u < nb) {
-                const int brow0 = sbm[3 * (b0 + u) + 1];
-                const int brows = min(sbm[3 * (b0 + u) + 2], kT);
-                const uint16_t* rows[kT];
-                const float* sums[kT];
-                float acc[kT];
-#pragma unroll
-                for (int i = 0; i < kT; ++i) {
-                    const int p = brow0 + min(i, brows - 1);
-                    rows[i] = hs + static_cast<size_t>(p) * f;
-                    sums[i] = hsum + p * nv;
-                    acc[i] = 0.0f;
-                }
-                row_dots<kT>(L[u], rows, sums, nv, lane, acc);
-#pragma unroll
-                for (int i = 0; i < kT; ++i) {
-                    const float v = warp_sum(acc[i]);
-                    if (lane == 0 && i < brows) os[brow0 + i][warp] = __bfloat162float(__float2bfloat16_rn(v));
-                }
+        for (int i = 0; i < 2; ++i) {
+            const int r = 2 * c + i;
+            if (r < brows) {
+                op[part][brow0 + r][g] = acc[i];
+                op[part][brow0 + r][g + 8] = acc[2 + i];
             }
         }
     }
+    if (split == 1) {  // whole-K sums: the second half is zero (no warp writes op[1])
+        for (int i = threadIdx.x; i < Tk * 16; i += blockDim.x) op[1][i >> 4][i & 15] = 0.0f;
+    }
     __syncthreads();
-    if (threadIdx.x < 16 * kT) {
+    if (threadIdx.x < 16 * T) {
         const int t = threadIdx.x >> 4;
         const int r = threadIdx.x & 15;
         float acc = 0.0f;
-        for (int jj = 0; jj < k; ++jj) acc = fmaf(sw[t * k + jj], os[spos[t * k + jj]][r], acc);
-        y[static_cast<size_t>(t) * d + blockIdx.x * 16 + r] = bf16_round_bits(acc);
+        for (int jj = 0; jj < k; ++jj) {
+            const int pj = spos[t * k + jj];
+            const float o = __bfloat162float(__float2bfloat16_rn(op[0][pj][r] + op[1][pj][r]));
+            acc = fmaf(sw[t * k + jj], o, acc);
+        }
+        y[static_cast<size_t>(t) * d + m0 + r] = bf16_round_bits(acc);
     }
 }
 
-
-constexpr size_t kDecodeSmemLimit = 112 * 1024;
+constexpr size_t kGuSmemLimit = 64 * 1024;
+constexpr size_t kDnSmemLimit = 180 * 1024;
 constexpr size_t kRouteSmemLimit = 200 * 1024;
-
-// gate/up: the batch's x rows; down: every assignment's h row and its vector sums
-size_t gateup_smem_bytes(const moe_shape_t& s, int T) { return static_cast<size_t>(T) * s.d * 2; }
-size_t down_smem_bytes(const moe_shape_t& s, int T) {
-    return static_cast<size_t>(T) * s.k * (static_cast<size_t>(s.f) * 2 + (s.f / 32) * 4);
-}
 
 size_t route_smem_bytes(const moe_shape_t& s, int T) {
     return static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(s.d) * (s.E / kRouteCtas) * 4 +
            static_cast<size_t>(T) * 32 * 33 * 4;
 }
 
-template <int kT>
-cudaError_t set_expert_kernel_smem() {
-    cudaError_t e = cudaFuncSetAttribute(decode_gateup_kernel<kT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kDecodeSmemLimit));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(decode_down_kernel<kT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(kDecodeSmemLimit));
+// gate/up: the block's x rows (at most T) and their vector sums; down: every
+// assignment's h row and its vector sums
+size_t gateup_smem_bytes(const moe_shape_t& s, int T) {
+    return static_cast<size_t>(T) * ((s.d + 32) * 2 + (s.d / 32) * 4);
+}
+size_t down_smem_bytes(const moe_shape_t& s, int T) {
+    return static_cast<size_t>(T) * s.k * ((s.f + 32) * 2 + (s.f / 32) * 4);
 }
 
-template <int kT>
+template <int kGpc>
+cudaError_t set_expert_kernel_smem() {
+    cudaError_t e = cudaFuncSetAttribute(decode_gateup_kernel<kGpc>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kGuSmemLimit));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(decode_down_kernel<kGpc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kDnSmemLimit));
+}
+
+template <int kGpc>
 cudaError_t launch_experts(const DecodeArgs& a, const DecodeRouteOut& ro, cudaStream_t st,
                            void* ev_gate_up) {
     const moe_shape_t& s = a.s;
-    const int nb_max = std::min(s.E, kT * s.k);
-    cudaError_t e = launch_pdl(decode_gateup_kernel<kT>, dim3(nb_max * (s.f / 16)), kRowThreads,
-                               gateup_smem_bytes(s, kT), st, a.x, a.wpack_gu, s.d, s.k,
-                               s.f, s.group, a.gu_block_bytes, ro, a.h);
+    const int nb_max = std::min(s.E, a.T * s.k);
+    cudaError_t e = launch_pdl(decode_gateup_kernel<kGpc>, dim3(nb_max * (s.f / kGuFeat)),
+                               dim3(kGuWarps * 32), gateup_smem_bytes(s, a.T), st, a.x, a.wpack_gu,
+                               a.T, s.d, s.k, s.f, a.gu_block_bytes, ro, a.h);
     if (e != cudaSuccess) return e;
     if (ev_gate_up && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_gate_up), st)) != cudaSuccess)
         return e;
-    return launch_pdl(decode_down_kernel<kT>, dim3(s.d / 16), kRowThreads,
-                      down_smem_bytes(s, kT), st, a.wpack_dn,
-                      static_cast<const uint16_t*>(a.h), s.d, s.k, s.f, s.group, a.dn_block_bytes,
-                      nb_max, ro, a.y);
+    return launch_pdl(decode_down_kernel<kGpc>, dim3(s.d / 16), dim3(kDnWarps * 32),
+                      down_smem_bytes(s, a.T), st, a.wpack_dn, static_cast<const uint16_t*>(a.h),
+                      a.T, s.d, s.k, s.f, a.dn_block_bytes, nb_max, ro, a.y);
 }
 
 }  // namespace
@@ -641,9 +631,10 @@ bool decode_supported(const moe_shape_t& s, int T) {
     if (T * s.k > kDecodeMaxAssign || s.E > kMaxExperts) return false;
     // whole 16-byte vectors of W_r columns per routing CTA
     if (s.E % (4 * kRouteCtas) != 0 || route_smem_bytes(s, T) > kRouteSmemLimit) return false;
-    // 16-byte nibble vectors (32 K values each) per lane and row
-    if (s.d > 32 * 32 * kGuVecs || s.f > 32 * 32 * kDnVecs) return false;
-    return gateup_smem_bytes(s, T) <= kDecodeSmemLimit && down_smem_bytes(s, T) <= kDecodeSmemLimit;
+    // (groups of 32 or 64 and d, f in whole tiles hold for every plan) a
+    // gate/up warp's K chunks fit in its registers
+    if (s.d > kGuWarps * kGuChunks * kKChunk) return false;
+    return gateup_smem_bytes(s, T) <= kGuSmemLimit && down_smem_bytes(s, T) <= kDnSmemLimit;
 }
 
 cudaError_t prepare_decode_kernels() {
@@ -651,15 +642,8 @@ cudaError_t prepare_decode_kernels() {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kRouteSmemLimit));
     if (e != cudaSuccess) return e;
-    static_assert(kDecodeMaxT == 8, "one instantiation per batch size");
     if ((e = set_expert_kernel_smem<1>()) != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<2>()) != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<3>()) != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<4>()) != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<5>()) != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<6>()) != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<7>()) != cudaSuccess) return e;
-    return set_expert_kernel_smem<8>();
+    return set_expert_kernel_smem<2>();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed, void* ev_gate_up) {
@@ -673,17 +657,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed,
     if (e != cudaSuccess) return e;
     if (ev_routed && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_routed), st)) != cudaSuccess)
         return e;
-    switch (T) {
-        case 1: return launch_experts<1>(a, ro, st, ev_gate_up);
-        case 2: return launch_experts<2>(a, ro, st, ev_gate_up);
-        case 3: return launch_experts<3>(a, ro, st, ev_gate_up);
-        case 4: return launch_experts<4>(a, ro, st, ev_gate_up);
-        case 5: return launch_experts<5>(a, ro, st, ev_gate_up);
-        case 6: return launch_experts<6>(a, ro, st, ev_gate_up);
-        case 7: return launch_experts<7>(a, ro, st, ev_gate_up);
-        case 8: return launch_experts<8>(a, ro, st, ev_gate_up);
-    }
-    return cudaErrorInvalidValue;
+    return s.group == 64 ? launch_experts<1>(a, ro, st, ev_gate_up)
+                         : launch_experts<2>(a, ro, st, ev_gate_up);
 }
 
 }  // namespace moe
