@@ -43,6 +43,7 @@ namespace {
 
 constexpr int kDecodeMaxAssign = kDecodeMaxT * kMaxTopk;
 constexpr int kRouteCtas = 8;       // cluster size of the routing kernel: E/8 experts each
+constexpr int kRouteRowsPerLoad = 256;  // W_r rows per tensor load (the box height limit)
 constexpr int kRowThreads = 512;    // threads of a routing CTA
 
 
@@ -103,6 +104,7 @@ struct DecodeRoute {
     int bm[3 * kDecodeMaxAssign];
     int nb;
     int sh_warp[kRowThreads / 32 + 1];
+    int cta_err[kRouteCtas];  // CTA r's copy of its W_r columns timed out (written every call)
 };
 
 __device__ void route_from_logits(int T, int E, int k, int max_blocks, DecodeRoute& R) {
@@ -197,53 +199,49 @@ __device__ void write_route(const DecodeRoute& R, const DecodeRouteOut& o, int T
 // adds chains q and q + m for q < m, m = 16..1), plus the bias.  Item
 // (p, el) of a CTA runs chain p of expert e0 + el for all T tokens: a group
 // of EC lanes reads EC consecutive floats of a W_r row per step, from a copy
-// of the CTA's W_r columns that all threads load with 16-byte vectors first.
-// The logits go to CTA 0's shared memory (distributed shared memory), which
-// then routes.  Dynamic shared memory: x [T][d] bf16, the W_r columns [d][EC]
-// fp32, the chains [T][32][33] fp32.
+// of the CTA's W_r columns that the tensor-memory-access unit brings in, 256
+// rows per load (the load/store units reach a fraction of its rate for this
+// strided copy).  The logits go to CTA 0's shared memory (distributed shared
+// memory), which then routes.  Dynamic shared memory (128-byte aligned): the
+// W_r columns [d][EC] fp32, x [T][d] bf16, the chains [T][32][33] fp32.
 // ---------------------------------------------------------------------------
 __global__ void __cluster_dims__(kRouteCtas, 1, 1) __launch_bounds__(kRowThreads)
-decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
+decode_route_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t* __restrict__ x,
                     const float* __restrict__ bias, int T, int d, int E, int k, int max_blocks,
                     DecodeRouteOut ro, int32_t* __restrict__ status) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ DecodeRoute R;
-    extern __shared__ __align__(16) uint8_t dsm[];
-    const uint16_t* xs = reinterpret_cast<const uint16_t*>(dsm);
-    float* ws = reinterpret_cast<float*>(dsm + static_cast<size_t>(T) * d * 2);  // [i][EC]
-    float* cs = ws + static_cast<size_t>(d) * (E / kRouteCtas);                  // [t][p][33]
+    __shared__ __align__(8) uint64_t wbar;
+    __shared__ int no_abort;
+    extern __shared__ __align__(16) uint8_t dsm_raw[];
+    uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) &
+                                              ~static_cast<uintptr_t>(127));
+    const int EC = E / kRouteCtas;
+    float* ws = reinterpret_cast<float*>(dsm);  // [i][EC]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(dsm + static_cast<size_t>(d) * EC * 4);
+    float* cs = reinterpret_cast<float*>(dsm + static_cast<size_t>(d) * EC * 4 +
+                                         static_cast<size_t>(T) * d * 2);  // [t][p][33]
     pdl_launch_dependents();
     const int rank = static_cast<int>(cluster.block_rank());
-    const int EC = E / kRouteCtas;
     const int e0 = rank * EC;
     const int nsteps = d >> 5;
     const int items = 32 * EC;
-    cta_copy16(dsm, x, T * d / 8);
-    {
-        // W_r[:, e0 .. e0+EC) -> ws: 16-byte vectors (EC % 4 == 0), 16 in
-        // flight per thread before their stores
-        const int nv = d * (EC / 4);
-        const int vrow = EC / 4;
-        for (int v0 = threadIdx.x; v0 < nv; v0 += 16 * kRowThreads) {
-            float4 v[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int vi = v0 + u * kRowThreads;
-                if (vi < nv) {
-                    const int i = vi / vrow;
-                    v[u] = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) +
-                                 (vi - i * vrow));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int vi = v0 + u * kRowThreads;
-                if (vi < nv) reinterpret_cast<float4*>(ws)[vi] = v[u];
-            }
-        }
+    const uint32_t bar = smem_u32(&wbar);
+    if (threadIdx.x == 0) {
+        // W_r[:, e0 .. e0+EC) -> ws in loads of 256 rows (e0 * 4 bytes is a
+        // multiple of 16: EC % 4 == 0)
+        no_abort = 0;
+        mbar_init(bar, 1);
+        fence_mbarrier_init();
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(d) * EC * 4);
+        for (int r0 = 0; r0 < d; r0 += kRouteRowsPerLoad)
+            tma_load_2d(smem_u32(ws + static_cast<size_t>(r0) * EC), &wmap, e0, r0, bar);
     }
-    __syncthreads();
+    cta_copy16(xs, x, T * d / 8);
+    __syncthreads();  // x in place; the barrier initialised
+    const bool w_ok = mbar_wait(bar, 0, &no_abort);
+    if (threadIdx.x == 0) cluster.map_shared_rank(R.cta_err, 0)[rank] = w_ok ? 0 : 1;
     for (int it = threadIdx.x; it < items; it += kRowThreads) {
         const int p = it / EC;
         const int el = it - p * EC;
@@ -277,6 +275,9 @@ decode_route_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     pdl_wait();
     // the status word reports the most recent call: the first kernel clears it
     if (threadIdx.x < 2) status[threadIdx.x] = 0;
+    __syncthreads();
+    if (threadIdx.x < kRouteCtas && R.cta_err[threadIdx.x])
+        report_error(status, MOE_ERR_DEVICE_TIMEOUT, 400 + threadIdx.x);
     route_from_logits(T, E, k, max_blocks, R);
     write_route(R, ro, T * k, E);
 }
@@ -585,8 +586,8 @@ constexpr size_t kDnSmemLimit = 180 * 1024;
 constexpr size_t kRouteSmemLimit = 200 * 1024;
 
 size_t route_smem_bytes(const moe_shape_t& s, int T) {
-    return static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(s.d) * (s.E / kRouteCtas) * 4 +
-           static_cast<size_t>(T) * 32 * 33 * 4;
+    return 128 + static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(s.d) * (s.E / kRouteCtas) * 4 +
+           static_cast<size_t>(T) * 32 * 33 * 4;  // + slack to align the base
 }
 
 // gate/up: the block's x rows (at most T) and their vector sums; down: every
@@ -652,8 +653,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed,
     const DecodeRouteOut ro{a.topk_idx, a.topk_w,        a.counts,    a.offsets,   a.sorted_assign,
                             a.pos,      a.block_offsets, a.block_map, a.num_blocks};
     const size_t route_smem = route_smem_bytes(s, T);
-    cudaError_t e = launch_pdl(decode_route_kernel, dim3(kRouteCtas), dim3(kRowThreads), route_smem, st,
-                               a.x, a.W_r, a.b_r, T, s.d, s.E, s.k, a.max_blocks, ro, a.status);
+    CUtensorMap wmap;
+    cudaError_t e = encode_f32_cols_map(&wmap, a.W_r, s.d, s.E, s.E / kRouteCtas, kRouteRowsPerLoad);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(decode_route_kernel, dim3(kRouteCtas), dim3(kRowThreads), route_smem, st, wmap, a.x,
+                   a.b_r, T, s.d, s.E, s.k, a.max_blocks, ro, a.status);
     if (e != cudaSuccess) return e;
     if (ev_routed && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_routed), st)) != cudaSuccess)
         return e;

@@ -563,8 +563,7 @@ cudaError_t prepare_gemm_kernels() {
                                 Cfg<true>::kSmemBytes);
 }
 
-cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                                 uint32_t box_rows) {
+static cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (encode == nullptr) {
         cudaDriverEntryPointQueryResult q;
@@ -574,6 +573,31 @@ cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t ro
             return e != cudaSuccess ? e : cudaErrorInvalidValue;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    *out = encode;
+    return cudaSuccess;
+}
+
+cudaError_t encode_f32_cols_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
+                                uint32_t box_cols, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    const cudaError_t e = tensor_map_encoder(&encode);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                                 uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    const cudaError_t e = tensor_map_encoder(&encode);
+    if (e != cudaSuccess) return e;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(kKChunk), box_rows};

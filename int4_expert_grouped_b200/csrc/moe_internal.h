@@ -111,6 +111,10 @@ struct GemmArgs {
     int block_bytes;
     int max_units;                 // upper bound of num_blocks * NT
 };
+// Encode the tensor map of a row-major fp32 matrix [rows, cols] read in boxes
+// of box_cols columns x box_rows rows, unswizzled.
+cudaError_t encode_f32_cols_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
+                                uint32_t box_cols, uint32_t box_rows);
 // Encode the tensor map of a row-major bf16 matrix [rows, cols] read in boxes
 // of 64 columns x box_rows rows with the 128-byte swizzle.
 cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
