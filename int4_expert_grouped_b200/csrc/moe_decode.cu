@@ -297,9 +297,9 @@ decode_route_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t* __
 // first MMA, pairs 2 and 3 the second, and its operand piece is the 16 bytes of
 // K 8c .. 8c+7 of its column.  A nibble pair becomes two bf16 values 128 + q
 // exactly (q in the mantissa of 128.0), so the MMA gives sum (128 + q) x; with
-// w = q s + b the vector's dot product is s * D + (b - 128 s) * sum x, formed
-// per vector in fp32 with the vector's group scale and bias.  The weights are
-// not rounded to bf16 on this path.
+// w = q s + b a group's dot product is s * D + (b - 128 s) * sum x, formed in
+// fp32 once per group (the MMAs of a 64-wide group accumulate together).  The
+// weights are not rounded to bf16 on this path.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -314,15 +314,18 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
     return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
 }
 
-// acc += dot products of one 32-wide vector: wa, wb = word c of the vector in
-// rows g and g + 8; xb = the column's operands K 8c .. 8c+7; sa, sb = the
-// rows' (scale, bias) words; xs0, xs1 = the vector sums of columns 2c, 2c + 1
-__device__ __forceinline__ void vector_mma(float (&acc)[4], uint32_t wa, uint32_t wb,
-                                           const uint4& xb, uint32_t sa, uint32_t sb, float xs0,
-                                           float xs1) {
-    float D[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+// D += sum (128 + q) x over one 32-wide vector: wa, wb = word c of the vector
+// in rows g and g + 8; xb = the column's operands K 8c .. 8c+7
+__device__ __forceinline__ void vector_mma(float (&D)[4], uint32_t wa, uint32_t wb, const uint4& xb) {
     mma_16816(D, nib_pair(wa, 0), nib_pair(wb, 0), nib_pair(wa, 1), nib_pair(wb, 1), xb.x, xb.y);
     mma_16816(D, nib_pair(wa, 2), nib_pair(wb, 2), nib_pair(wa, 3), nib_pair(wb, 3), xb.z, xb.w);
+}
+
+// acc += s * D + (b - 128 s) * sum x for one group: sa, sb = the (scale,
+// bias) words of rows g and g + 8; xs0, xs1 = the group's operand sums of
+// columns 2c, 2c + 1
+__device__ __forceinline__ void group_fold(float (&acc)[4], const float (&D)[4], uint32_t sa,
+                                           uint32_t sb, float xs0, float xs1) {
     const float s0 = __uint_as_float(sa << 16);
     const float s1 = __uint_as_float(sb << 16);
     const float c0 = fmaf(-128.0f, s0, __uint_as_float(sa & 0xFFFF0000u));
@@ -375,13 +378,19 @@ __device__ __forceinline__ void tile_dots(float (&acc)[4], const TileLoads<kChun
     for (int u = 0; u < kChunks; ++u) {
         const int ch = ch0 + u * ch_step;
         if (ch < KC) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int v = 2 * ch + hh;
-                const uint4 xb = *reinterpret_cast<const uint4*>(xrow + 32 * v);
-                const int q = kGpc == 2 ? hh : 0;
-                vector_mma(acc, L.w[u][hh], L.w[u][2 + hh], xb, L.sc[u][q], L.sc[u][kGpc + q],
-                           xs0[v], xs1[v]);
+            const int v = 2 * ch;
+            const uint4 xb0 = *reinterpret_cast<const uint4*>(xrow + 32 * v);
+            const uint4 xb1 = *reinterpret_cast<const uint4*>(xrow + 32 * v + 32);
+            float D[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            vector_mma(D, L.w[u][0], L.w[u][2], xb0);
+            if (kGpc == 2) {  // a group per vector
+                group_fold(acc, D, L.sc[u][0], L.sc[u][2], xs0[v], xs1[v]);
+                D[0] = D[1] = D[2] = D[3] = 0.0f;
+                vector_mma(D, L.w[u][1], L.w[u][3], xb1);
+                group_fold(acc, D, L.sc[u][1], L.sc[u][3], xs0[v + 1], xs1[v + 1]);
+            } else {  // one group for the chunk: its four MMAs share the fold
+                vector_mma(D, L.w[u][1], L.w[u][3], xb1);
+                group_fold(acc, D, L.sc[u][0], L.sc[u][1], xs0[v] + xs0[v + 1], xs1[v] + xs1[v + 1]);
             }
         }
     }
