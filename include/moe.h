@@ -182,7 +182,10 @@ MOE_API moe_status_t moe_route(const moe_plan_t *plan, int32_t T, const uint16_t
  * nibble*scale+bias), products accumulate in fp32, the SwiGLU output is
  * rounded to bf16 before the down projection, each expert's down output is
  * rounded to bf16, the k weighted outputs of a token are summed in fp32 in
- * slot order j = 0..k-1 and y is rounded to bf16.
+ * slot order j = 0..k-1 and y is rounded to bf16.  The small-batch kernels
+ * (moe_forward_path == 1) do not round the weights: each group's fp32 sum of
+ * nibble * x takes the group's scale and bias (scale * sum + bias * sum x);
+ * the later roundings are the same.
  */
 MOE_API moe_status_t moe_forward(const moe_plan_t *plan, int32_t T, const uint16_t *x,
                          const float *W_r, const float *b_r,
