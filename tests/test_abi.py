@@ -138,3 +138,9 @@ def test_forward_path_choice(moe):
     assert tiny.forward_path(3) == 0  # E = 8: too few experts for the 8-CTA routing cluster
     g32 = moe.Plan(64, 256, 32, 2, 128, 32)
     assert g32.forward_path(3) == 1 and g32.forward_path(9) == 0
+    # d = 4096: a gate/up warp's K chunks no longer fit its registers
+    assert moe.Plan(64, 4096, 128, 8, 768, 64).forward_path(1) == 0
+    # f = 1024 at T = 8: 64 h rows and their sums still fit the down kernel's shared memory
+    assert moe.Plan(64, 2048, 128, 8, 1024, 64).forward_path(8) == 1
+    # E = 256 at d = 2048: a routing CTA's 32 W_r columns (256 KB) exceed its shared memory
+    assert moe.Plan(64, 2048, 256, 8, 768, 64).forward_path(1) == 0
