@@ -223,6 +223,32 @@ def check_block_map(orc, seed=13):
         assert np.all(np.diff(bm[:, 1]) > 0) if nb > 1 else True
 
 
+# Block maps worked out by hand: expert e with c_e rows gets ceil(c_e / BT)
+# tiles in ascending expert order; tile i starts at offsets[e] + i * BT and
+# holds min(BT, c_e - i * BT) rows, so only an expert's last tile is ragged
+# and experts without rows get no tile.
+BLOCK_MAP_CASES = [
+    # (counts, BT, expected (expert, first row, rows) entries, block_offsets)
+    ((300, 0, 256, 1), 128,
+     [(0, 0, 128), (0, 128, 128), (0, 256, 44), (2, 300, 128), (2, 428, 128), (3, 556, 1)],
+     (0, 3, 3, 5, 6)),
+    ((513, 255, 0, 256), 256,
+     [(0, 0, 256), (0, 256, 256), (0, 512, 1), (1, 513, 255), (3, 768, 256)],
+     (0, 3, 4, 4, 5)),
+    ((0, 0, 7), 4, [(2, 0, 4), (2, 4, 3)], (0, 0, 0, 2)),
+]
+
+
+def check_block_map_hand(orc):
+    for counts, BT, entries, bo_ref in BLOCK_MAP_CASES:
+        counts = np.array(counts, np.int32)
+        offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        bo, bm, nb = orc.block_map(counts, offsets, BT)
+        assert nb == len(entries), (counts, nb)
+        assert [tuple(int(v) for v in row) for row in bm] == entries, (counts, bm)
+        assert tuple(int(v) for v in bo) == bo_ref, (counts, bo)
+
+
 # ----------------------------------------------------------------------------
 # dequantisation
 # ----------------------------------------------------------------------------
@@ -361,6 +387,7 @@ ALL_CHECKS = [
     check_topk_weights,
     check_scan_scatter,
     check_block_map,
+    check_block_map_hand,
     check_dequant_hand,
     check_dequant_all_nibbles,
     check_single_expert_is_dense_mlp,

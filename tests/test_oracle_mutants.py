@@ -27,6 +27,24 @@ MUTANTS = {
                            "offsets[e + 1] = offsets[e] + counts[e] + (e == 0);"),
     "scatter_stores_token": ("sorted_assign[p] = (int32_t)a;", "sorted_assign[p] = (int32_t)(a / k);"),
     "block_rows_not_clipped": ("? counts[e] - i * BT : BT", "? BT : BT"),
+    # an expert's rows split evenly over its tiles (300 rows at BT 128: 100/100/100)
+    "block_even_split": (
+        "const int64_t rows = counts[e] - i * BT < BT ? counts[e] - i * BT : BT;\n"
+        "            block_map[3 * nb + 0] = (int32_t)e;\n"
+        "            block_map[3 * nb + 1] = (int32_t)(offsets[e] + i * BT);",
+        "const int64_t per = (counts[e] + tiles - 1) / tiles;\n"
+        "            const int64_t rows = i == tiles - 1 ? counts[e] - per * (tiles - 1) : per;\n"
+        "            block_map[3 * nb + 0] = (int32_t)e;\n"
+        "            block_map[3 * nb + 1] = (int32_t)(offsets[e] + i * per);"),
+    # the ragged tile first (300 rows at BT 128: 44/128/128)
+    "block_ragged_first": (
+        "const int64_t rows = counts[e] - i * BT < BT ? counts[e] - i * BT : BT;\n"
+        "            block_map[3 * nb + 0] = (int32_t)e;\n"
+        "            block_map[3 * nb + 1] = (int32_t)(offsets[e] + i * BT);",
+        "const int64_t rag = counts[e] - (tiles - 1) * BT;\n"
+        "            const int64_t rows = i == 0 ? rag : BT;\n"
+        "            block_map[3 * nb + 0] = (int32_t)e;\n"
+        "            block_map[3 * nb + 1] = (int32_t)(offsets[e] + (i == 0 ? 0 : rag + (i - 1) * BT));"),
     "nibble_order_swapped": ("(4 * (kk % 2))", "(4 * (1 - kk % 2))"),
     "group_index_wrong": ("scale[n * (K / G) + kk / G]", "scale[n * (K / G) + kk / (2 * G)]"),
     "silu_sign": ("return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
