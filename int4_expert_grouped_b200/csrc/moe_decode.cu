@@ -238,6 +238,10 @@ decode_route_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t* __
         for (int r0 = 0; r0 < d; r0 += kRouteRowsPerLoad)
             tma_load_2d(smem_u32(ws + static_cast<size_t>(r0) * EC), &wmap, e0, r0, bar);
     }
+    // x may be the output of the previous kernel in the stream (for example
+    // y of the previous call), so it is read only after that kernel has
+    // completed; W_r and the bias are never written by this library
+    pdl_wait();
     cta_copy16(xs, x, T * d / 8);
     __syncthreads();  // x in place; the barrier initialised
     const bool w_ok = mbar_wait(bar, 0, &no_abort);
@@ -270,9 +274,6 @@ decode_route_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t* __
     }
     cluster.sync();  // all logits are in CTA 0; no CTA touches another's memory after this
     if (rank != 0) return;
-    // everything above reads only the layer's inputs; the outputs below are
-    // read by the previous call's kernels, which must have finished
-    pdl_wait();
     // the status word reports the most recent call: the first kernel clears it
     if (threadIdx.x < 2) status[threadIdx.x] = 0;
     __syncthreads();

@@ -4,9 +4,10 @@ Integer outputs (top-k indices, counts, offsets, scatter order, inverse
 positions, block map) must match bit for bit; routing weights within 1e-6
 relative; the layer output within |y - ref| <= 2e-2 * (1 + |ref|) with the
 relative RMS error also reported and bounded.  Small workloads are checked in
-full; the 8K- and 32K-token prefill workloads have their routing checked in
-full and their outputs on sampled tokens (the oracle computes those one
-token at a time).
+full; the 8K-token prefill layer has every token's output checked, and the
+32K-token Zipf layer the outputs of the first and last token of every
+block-map entry and of every token of its most and least loaded experts (the
+oracle computes those one token at a time).
 """
 import numpy as np
 import pytest
@@ -98,9 +99,10 @@ def test_layer_full(moe, name):
     check_y(y[:s.T], ref["y"], name)
 
 
-@pytest.mark.parametrize("name", ["prefill_t8192", "prefill_t32768_zipf"])
-def test_layer_large_sampled(moe, name):
-    inp = workload(name)
+def test_layer_t8192_every_token(moe):
+    # the 8192-token prefill layer: routing in full and the output of every
+    # token against the oracle (about 9 s of CPU on 16 cores)
+    inp = workload("prefill_t8192")
     s = inp.shape
     layer = moe.MoeLayer.from_inputs(inp)
     x = moe.bf16_tensor(inp.x, "cuda")
@@ -110,15 +112,47 @@ def test_layer_large_sampled(moe, name):
     assert layer.read_status() == (0, 0)
     rref = oracle_route(inp)
     check_route(bufs, rref, s.T, s.k)
-    # sampled tokens: both ends, a spread, and tokens of the most loaded expert
-    rng = np.random.default_rng(1234)
-    hot = int(np.argmax(rref["counts"]))
-    hot_tokens = rref["sorted_assign"][rref["offsets"][hot]:rref["offsets"][hot + 1]] // s.k
-    toks = np.unique(np.concatenate([[0, 1, s.T - 1], rng.choice(s.T, 40, replace=False),
-                                     rng.choice(hot_tokens, 8, replace=False)]))
-    yref, idx, w = oracle.token_outputs(inp, toks)
+    toks = np.arange(s.T)
+    yref, idx, _ = oracle.token_outputs(inp, toks)
+    assert np.array_equal(idx, rref["topk_idx"])
+    check_y(y[:s.T], yref, "prefill_t8192, every token")
+
+
+def block_entry_tokens(rref, k):
+    """Tokens of the first and the last row of every block-map entry."""
+    bm = rref["block_map"]
+    sa = rref["sorted_assign"]
+    first = sa[bm[:, 1]] // k
+    last = sa[bm[:, 1] + bm[:, 2] - 1] // k
+    return np.unique(np.concatenate([first, last]))
+
+
+def test_layer_t32768_zipf_every_block(moe):
+    # the Zipf-skewed 32768-token layer: routing in full; the output of at
+    # least one token of every block-map entry (its first and last rows), and
+    # of every token of the most and of the least loaded non-empty expert
+    inp = workload("prefill_t32768_zipf")
+    s = inp.shape
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bufs = layer.route_buffers(s.T)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    assert layer.read_status() == (0, 0)
+    rref = oracle_route(inp)
+    check_route(bufs, rref, s.T, s.k)
+    counts, offsets, sa = rref["counts"], rref["offsets"], rref["sorted_assign"]
+    nonempty = np.flatnonzero(counts)
+    hot = int(nonempty[np.argmax(counts[nonempty])])
+    cold = int(nonempty[np.argmin(counts[nonempty])])
+    expert_tokens = lambda e: sa[offsets[e]:offsets[e + 1]] // s.k
+    toks = np.unique(np.concatenate([block_entry_tokens(rref, s.k), expert_tokens(hot),
+                                     expert_tokens(cold)]))
+    print("checking %d of %d tokens (%d block-map entries; expert %d has %d rows, expert %d has %d)"
+          % (len(toks), s.T, rref["num_blocks"], hot, counts[hot], cold, counts[cold]))
+    yref, idx, _ = oracle.token_outputs(inp, toks)
     assert np.array_equal(idx, rref["topk_idx"][toks])
-    check_y(y[torch.from_numpy(toks).cuda()], yref, name)
+    check_y(y[torch.from_numpy(toks).cuda()], yref, "prefill_t32768_zipf, every block")
 
 
 def test_route_entry_point_matches_forward(moe):
@@ -278,3 +312,33 @@ def test_decode_path_wide_layer(moe, T):
     assert layer.plan.forward_path(T) == 1
     check_route(bufs, oracle_route(inp), T, 8)
     check_y(y[:T], oracle.forward(inp)["y"], "decode wide T=%d" % T)
+
+
+def test_chained_calls_read_previous_output(moe):
+    # The next call's x is the previous call's y, with no synchronisation in
+    # between: a batched call then a small-batch call, then a small-batch call
+    # on that output.  Kernels chained by programmatic dependent launch may
+    # start early, so each must read x only after its predecessor completed.
+    inp = workload("prefill_t512")
+    s = inp.shape
+    layer = moe.MoeLayer.from_inputs(inp)
+    assert layer.plan.forward_path(512) == 0 and layer.plan.forward_path(1) == 1
+    x = moe.bf16_tensor(inp.x, "cuda")
+    y1 = layer.forward(x)
+    b2 = layer.route_buffers(1)
+    y2 = layer.forward(y1[:1], route_out=b2)
+    b3 = layer.route_buffers(4)
+    y3 = layer.forward(torch.cat([y2[:1]] * 4), route_out=b3)  # torch's copy sits in between
+    y4 = layer.forward(y3[:2])
+    torch.cuda.synchronize()
+    assert layer.read_status() == (0, 0)
+    check_y(y1[:512], oracle.forward(inp)["y"], "batched call")
+    bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    for xin, yout, bufs in ((y1[:1], y2, b2), (torch.cat([y2[:1]] * 4), y3, b3), (y3[:2], y4, None)):
+        T = xin.shape[0]
+        sub = mi.Inputs(mi.Shape(T, s.d, s.E, s.k, s.f, s.group), inp.seed, bits(xin), inp.w_r,
+                        inp.b_r, inp.gate, inp.up, inp.down)
+        if bufs is not None:
+            check_route(bufs, oracle_route(sub), T, s.k)
+        check_y(yout[:T], oracle.forward(sub)["y"], "chained T=%d" % T)
+
