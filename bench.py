@@ -35,8 +35,8 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer prefill tokens/s (int4 fused grouped GEMM) and % of roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
-KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, down GEMM, combine
-KERNELS_PER_STEP_DECODE = 3  # routing cluster, gate/up, down + combine (batches of at most 8 tokens)
+KERNELS_PER_STEP = 7  # logits, top-k, scan, scatter, gate/up GEMM (row gather), down GEMM, combine
+KERNELS_PER_STEP_DECODE = 1  # one persistent kernel (batches of at most 8 tokens)
 
 
 def load_peaks():
@@ -212,7 +212,7 @@ def time_layer(layer, x, y, K, repeats, flush, stream, world=1):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             total = float(t.item())
         stages = {
-            "routing_and_dispatch": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
+            "routing": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
             "gate_up_gemm": float(np.mean([r[1].elapsed_time(r[2]) for r in evs])),
             "down_gemm": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
             "combine": float(np.mean([r[3].elapsed_time(r[4]) for r in evs])),

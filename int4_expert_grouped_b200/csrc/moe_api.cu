@@ -169,6 +169,8 @@ moe_status_t moe_plan_create(const moe_shape_t* shape, moe_plan_t** plan, moe_pl
         return r;
     };
     p->o_status = take(256);
+    p->o_dsync = take(moe::kDecodeSyncBytes);  // offset 256: flags of the small-batch kernel
+    p->o_dscr = take(moe::decode_workspace_bytes(s, s.T_max));
     p->o_logits = take(T * E * 4);
     p->o_hist = take(static_cast<size_t>(p->ng_max) * E * 4);
     p->o_gbase = take(static_cast<size_t>(p->ng_max) * E * 4);
@@ -181,7 +183,7 @@ moe_status_t moe_plan_create(const moe_shape_t* shape, moe_plan_t** plan, moe_pl
     p->o_sa = take(T * k * 4);
     p->o_pos = take(T * k * 4);
     p->o_bm = take(static_cast<size_t>(p->max_blocks) * 12);
-    p->o_xs = take(T * k * s.d * 2);  // x rows in expert order, later the down outputs o
+    p->o_o = take(T * k * s.d * 2);   // down outputs o, one bf16 row per assignment
     p->o_h = take(T * k * s.f * 2);
     p->ws_bytes = o;
     p->o_xstage = take(T * s.d * 2);
@@ -276,7 +278,7 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     const moe_shape_t& s = plan->s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const RoutePtrs r = route_ptrs(plan, ws, route_out);
-    uint16_t* xs = at<uint16_t>(ws, plan->o_xs);
+    uint16_t* o = at<uint16_t>(ws, plan->o_o);
     uint16_t* h = at<uint16_t>(ws, plan->o_h);
     int32_t* status = at<int32_t>(ws, plan->o_status);
     auto mark = [&](void* e) -> bool {
@@ -284,7 +286,8 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     };
     if (ev && !mark(ev->start)) return MOE_ERR_CUDA;
     if (moe::decode_supported(s, T)) {
-        // a few tokens: three launches bound by reading the selected experts' weights
+        // a few tokens: one persistent kernel bound by reading the selected
+        // experts' weights
         const uint8_t* wp = static_cast<const uint8_t*>(packed_w);
         moe::DecodeArgs da{};
         da.s = s;
@@ -296,7 +299,6 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
         da.wpack_dn = wp + align_up(plan->gu_packed, 256);
         da.gu_block_bytes = plan->group_bytes;
         da.dn_block_bytes = plan->down_block_bytes;
-        da.max_blocks = plan->max_blocks;
         da.topk_idx = r.idx;
         da.topk_w = r.w;
         da.counts = r.counts;
@@ -309,8 +311,12 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
         da.h = h;
         da.y = y;
         da.status = status;
-        MOE_CUDA(moe::launch_decode(da, st, ev ? ev->routed : nullptr, ev ? ev->gate_up : nullptr));
-        if (ev && !(mark(ev->down) && mark(ev->end))) return MOE_ERR_CUDA;
+        da.sync = at<int32_t>(ws, plan->o_dsync);
+        da.scratch = at<uint8_t>(ws, plan->o_dscr);
+        MOE_CUDA(moe::launch_decode(da, num_sms, st));
+        // one kernel: the stage events all mark its end
+        if (ev && !(mark(ev->routed) && mark(ev->gate_up) && mark(ev->down) && mark(ev->end)))
+            return MOE_ERR_CUDA;
         return MOE_OK;
     }
     moe_status_t rs = run_route(plan, T, x, W_r, b_r, r, ws, st);
@@ -321,8 +327,6 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
         return MOE_OK;
     }
     const int Tk = T * s.k;
-    // step 5 (dispatch): token rows into expert order
-    MOE_CUDA(moe::launch_dispatch(x, r.sa, Tk, s.k, s.d, xs, status, num_sms, st));
     if (ev && !mark(ev->routed)) return MOE_ERR_CUDA;
 
     const int mb = max_blocks_for(s, T);
@@ -339,13 +343,17 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.group = s.group;
     g.block_bytes = plan->group_bytes;
     g.max_units = mb * g.NT;
-    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT));
+    // the token operand is gathered from x by row: no copy of x in expert order
+    g.sorted_assign = r.sa;
+    g.k = s.k;
+    g.T = T;
+    MOE_CUDA(moe::encode_bf16_gather_map(&g.bmap, x, static_cast<uint64_t>(T), s.d));
     MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
     if (ev && !mark(ev->gate_up)) return MOE_ERR_CUDA;
 
-    // the down outputs o reuse the storage of xs, which gate/up has finished reading
     g.wpack = wp + align_up(plan->gu_packed, 256);
-    g.out = xs;
+    g.out = o;
+    g.sorted_assign = nullptr;
     g.K = s.f;
     g.NT = s.d / (128 * moe::kDownTiles);
     g.out_ld = s.d;
@@ -354,7 +362,7 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;
-    MOE_CUDA(moe::launch_combine(xs, r.pos, r.w, T, s.k, s.d, y, status, num_sms, st));
+    MOE_CUDA(moe::launch_combine(o, r.pos, r.w, T, s.k, s.d, y, status, num_sms, st));
     if (ev && !mark(ev->end)) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -1,39 +1,53 @@
 // Small-batch (decode) path of the MoE layer: the same operation as the
 // batched path (inblix article "Perplexity's Lily engine beats MLX by 35% on
 // M5 Max, no PyTorch needed", paragraph 3: routing, prefix scan, scatter,
-// block map, dequantisation-fused expert GEMMs, weighted combine) for a few
-// tokens, where the layer is bound by reading the selected experts' int4
-// weights from HBM.  Three launches chained with programmatic dependent
-// launch, so each one's start-up overlaps the previous one's tail:
+// block map, dequantisation-fused expert GEMMs, weighted combine) for at most
+// eight tokens, where the layer is bound by reading the selected experts'
+// int4 weights from HBM (wpnews page "Perplexity Lily: 1.35x Faster Local AI
+// Than MLX on Mac", section "Why MLX Falls Behind": prefill and decode are
+// separate workloads).
 //
-//   decode_route_kernel    one cluster of 8 CTAs: each CTA runs the 32 fp32
-//                          fused-multiply-add chains of its E/8 experts
-//                          (lanes over experts, so W_r is read in row
-//                          segments), combines them with the router's fixed
-//                          butterfly tree and writes the logits into CTA 0's
-//                          shared memory; CTA 0 then does top-k, counts,
-//                          scan, block map and scatter and writes them out
-//   decode_gateup_kernel   per (block, 8 features): the gate and up rows as
-//                          one 16-row tile of the warp-level tensor-core MMA
-//                          against the block's x rows (the MMA's 8 columns),
-//                          int4 codes unpacked straight into its registers;
-//                          each 32-wide vector's sum takes its group's scale
-//                          and bias; SwiGLU gives bf16 rows of h
-//   decode_down_kernel     per 16 output features: the same tile MMA for
-//                          every selected expert against that expert's h
-//                          rows, each output rounded to bf16, then the
-//                          routing-weighted sum over a token's slots in order
+// One persistent kernel, one CTA per SM, in four phases separated by flags in
+// the workspace (no host round trip, no second launch):
 //
-// The MMA's 8 columns hold a block's rows (one per token), so the instruction
-// count does not grow with the batch up to 8 tokens.  The weights are read in
-// the prepacked block layout of the batched path, so one packed copy serves
-// both.  Rounding differs from the batched path only in the weights: there
-// each dequantised weight is rounded to bf16 before the MMA, here the exact
-// codes meet the operands and each group's scale and bias apply to its fp32
-// sum (closer to the unrounded q*s + b).  Both keep fp32 sums, bf16 h, bf16
-// expert outputs and the fp32 slot-order combine.
-#include <cooperative_groups.h>
-
+//   1. router partials  CTA c owns routing item c (8 experts x one residue
+//                       class r of the 32 fp32 chains): it brings its W_r
+//                       piece in by one tensor load, runs the chains
+//                       p = r, r+8, r+16, r+24 over all tokens and combines
+//                       them by the first two levels of the router's
+//                       butterfly; the partial u_r goes to the workspace
+//   2. routing          every CTA, once all items are in: the last three
+//                       butterfly levels and the bias give the logits; top-k,
+//                       weights, counts, offsets, block map and scatter are
+//                       computed in every CTA identically (CTA 0 writes them)
+//   3. experts          the units (gate/up: expert, 128-feature tile, two
+//                       64-wide K chunks; down: expert, 128-output tile, half
+//                       of K) are dealt round robin to the CTAs, gate/up units
+//                       first.  A producer warp streams each unit's packed
+//                       blocks into a shared-memory ring with bulk copies, as
+//                       far ahead as the ring allows, so every SM keeps its
+//                       share of the weights in flight; eight warps multiply
+//                       them on the warp-level tensor-core MMA.  Partial sums
+//                       go to the workspace; the last unit of a tile (an
+//                       atomic count) adds them in a fixed order: SwiGLU into
+//                       h for gate/up, and for down the weighted sum of each
+//                       token's expert outputs in slot order into y
+//   4. exit             the last CTA to leave resets the flags for the next
+//                       call
+//
+// MMA form (m16n8k16, bf16 operands from registers, fp32 accumulators): a
+// 16-row tile of packed weights is A, the rows of one expert's block (at most
+// eight tokens) are the eight columns of B.  A nibble pair becomes two bf16
+// values 128 + q exactly, so the MMA gives sum (128 + q) x; with
+// w = q s + b a group's dot product is s * D + (b - 128 s) * sum x, formed in
+// fp32 once per group.  The weights are not rounded to bf16 on this path
+// (closer to the unrounded q s + b than the batched path's rounding); h and
+// each expert output are rounded to bf16 and a token's slots are summed in
+// slot order, as in the batched path.
+//
+// Every wait is bounded (%globaltimer): a CTA that gives up records
+// MOE_ERR_DEVICE_TIMEOUT, raises an abort flag the others poll, and still
+// takes part in the exit count.
 #include <algorithm>
 
 #include "moe_route_common.cuh"
@@ -41,267 +55,80 @@
 namespace moe {
 namespace {
 
-constexpr int kDecodeMaxAssign = kDecodeMaxT * kMaxTopk;
-constexpr int kRouteCtas = 8;       // cluster size of the routing kernel: E/8 experts each
-constexpr int kRouteRowsPerLoad = 256;  // W_r rows per tensor load (the box height limit)
-constexpr int kRowThreads = 512;    // threads of a routing CTA
+constexpr int kDecComputeWarps = 8;
+constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;  // + one producer warp
+constexpr int kDecProducerWarp = kDecComputeWarps;
+constexpr int kDecComputeThreads = kDecComputeWarps * 32;
+constexpr int kDecStages = 16;
+constexpr int kDecStageBytes = packed_block_bytes(2, 32);  // a gate/up block (group 32: largest)
+constexpr int kDecMaxAssign = 64;                          // T * k the path takes
+constexpr int kDecGuChunks = 2;                            // 64-wide K chunks per gate/up unit
+constexpr int kDecMaxNT = 16;                              // f / 128
+constexpr int kDecMaxNTd = 64;                             // d / 128
+constexpr int kDecWRows = 256;                             // W_r rows per tensor load (box limit)
+constexpr uint32_t kDecMagic0 = 0x4D6F4544u, kDecMagic1 = 0x53796E63u;
 
+// Flags in the workspace's decode region (int32 offsets).
+constexpr int kSyncMagic = 0;     // two words: the region has been initialised
+constexpr int kSyncRoute = 2;     // routing items published
+constexpr int kSyncExit = 3;      // CTAs that have finished
+constexpr int kSyncAbort = 4;     // a CTA gave up waiting
+constexpr int kSyncHReady = 16;   // [kDecMaxAssign] gate/up tiles done per block
+constexpr int kSyncDn = kSyncHReady + kDecMaxAssign;  // [kDecMaxNTd] down units done per tile
+constexpr int kSyncGu = kSyncDn + kDecMaxNTd;         // [kDecMaxAssign * kDecMaxNT] per (block, tile)
+constexpr int kSyncInts = kSyncGu + kDecMaxAssign * kDecMaxNT;
+static_assert(kSyncInts * 4 <= kDecodeSyncBytes, "decode flags fit their workspace region");
 
-__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
     uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
 }
-__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+__device__ __forceinline__ float ld_cg_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
 }
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int atom_acq_rel_add(int* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// barrier of the eight compute warps (the producer warp does not take part)
+__device__ __forceinline__ void compute_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeThreads) : "memory");
+}
 
-// copy n 16-byte vectors global -> shared by the whole CTA, four loads in
-// flight per thread before their stores
-__device__ __forceinline__ void cta_copy16(void* dst, const void* src, int n) {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
-    uint4* d = reinterpret_cast<uint4*>(dst);
-    const int stride = blockDim.x;
-    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * stride) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (i0 + u * stride < n) v[u] = ld_nc_v4(s + i0 + u * stride);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (i0 + u * stride < n) d[i0 + u * stride] = v[u];
-    }
+// 3-D tensor load (TMA): coordinates c0 (innermost), c1, c2.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
 }
 
 __device__ __forceinline__ uint16_t bf16_round_bits(float v) {
     const __nv_bfloat16 b = __float2bfloat16_rn(v);
     return *reinterpret_cast<const uint16_t*>(&b);
 }
-
-// ---------------------------------------------------------------------------
-// Routing of the few tokens in shared memory (CTA 0 of the routing cluster,
-// kRowThreads threads) from the logits lg [T][E]: top-k (each (token, expert)
-// pair finds its slot in parallel; the warp of a token then forms the
-// weights), counts (integer atomics), offsets (exclusive scan), block map
-// (ceil(count / kBlockT) tiles per expert in ascending expert order), and the
-// stable scatter (the rank of assignment a within its expert is the number of
-// earlier assignments to that expert).
-// ---------------------------------------------------------------------------
-struct DecodeRoute {
-    float lg[kDecodeMaxT * kMaxExperts];
-    float sel[kDecodeMaxAssign];  // logit of each selected slot
-    int idx[kDecodeMaxAssign];
-    float w[kDecodeMaxAssign];
-    int sa[kDecodeMaxAssign];
-    int pos[kDecodeMaxAssign];
-    int cnt[kMaxExperts];
-    int off[kMaxExperts + 1];
-    int bo[kMaxExperts + 1];
-    int bm[3 * kDecodeMaxAssign];
-    int nb;
-    int sh_warp[kRowThreads / 32 + 1];
-    int cta_err[kRouteCtas];  // CTA r's copy of its W_r columns timed out (written every call)
-};
-
-__device__ void route_from_logits(int T, int E, int k, int max_blocks, DecodeRoute& R) {
-    static_assert(kRowThreads >= kMaxExperts, "one thread per expert");
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int tid = threadIdx.x;
-    const int Tk = T * k;
-    if (tid < E) R.cnt[tid] = 0;
-    for (int it = tid; it < T * E; it += kRowThreads) {
-        const int t = it / E;
-        const int e = it - t * E;
-        const int slot = expert_slot(R.lg + t * E, E, e);
-        if (slot < k) {
-            R.idx[t * k + slot] = e;
-            R.sel[t * k + slot] = R.lg[it];
-        }
-    }
-    __syncthreads();
-    for (int t = warp; t < T; t += kRowThreads / 32) {
-        const float wt = warp_slot_weights(lane < k ? R.sel[t * k + lane] : 0.0f, k, lane);
-        if (lane < k) R.w[t * k + lane] = wt;
-    }
-    __syncthreads();
-    for (int a = tid; a < Tk; a += kRowThreads) atomicAdd(&R.cnt[R.idx[a]], 1);
-    __syncthreads();
-    const int c = tid < E ? R.cnt[tid] : 0;
-    int total = 0;
-    const int off = block_exclusive_scan<kRowThreads>(c, R.sh_warp, &total);
-    if (tid < E) R.off[tid] = off;
-    if (tid == 0) R.off[E] = total;
-    const int nt = (c + kBlockT - 1) / kBlockT;
-    int nb_total = 0;
-    const int bo = block_exclusive_scan<kRowThreads>(tid < E ? nt : 0, R.sh_warp, &nb_total);
-    if (tid < E) {
-        R.bo[tid] = bo;
-        for (int i = 0; i < nt && bo + i < max_blocks && bo + i < kDecodeMaxAssign; ++i) {
-            R.bm[3 * (bo + i) + 0] = tid;
-            R.bm[3 * (bo + i) + 1] = off + i * kBlockT;
-            R.bm[3 * (bo + i) + 2] = min(kBlockT, c - i * kBlockT);
-        }
-    }
-    if (tid == 0) {
-        R.bo[E] = nb_total;
-        R.nb = min(min(nb_total, max_blocks), kDecodeMaxAssign);
-    }
-    for (int a = tid; a < Tk; a += kRowThreads) {
-        const int e = R.idx[a];
-        int rank = 0;
-        for (int a2 = 0; a2 < a; ++a2) rank += R.idx[a2] == e;
-        const int p = R.off[e] + rank;
-        R.sa[p] = a;
-        R.pos[a] = p;
-    }
-    __syncthreads();
+__device__ __forceinline__ float bf16_round(float v) {
+    return __bfloat162float(__float2bfloat16_rn(v));
 }
 
-struct DecodeRouteOut {
-    int32_t* topk_idx;
-    float* topk_w;
-    int32_t* counts;
-    int32_t* offsets;
-    int32_t* sorted_assign;
-    int32_t* pos;
-    int32_t* block_offsets;
-    int32_t* block_map;
-    int32_t* num_blocks;
-};
-
-__device__ void write_route(const DecodeRoute& R, const DecodeRouteOut& o, int Tk, int E) {
-    for (int a = threadIdx.x; a < Tk; a += blockDim.x) {
-        o.topk_idx[a] = R.idx[a];
-        o.topk_w[a] = R.w[a];
-        o.sorted_assign[a] = R.sa[a];
-        o.pos[a] = R.pos[a];
-    }
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-        if (e < E) o.counts[e] = R.cnt[e];
-        o.offsets[e] = R.off[e];
-        o.block_offsets[e] = R.bo[e];
-    }
-    for (int i = threadIdx.x; i < 3 * R.nb; i += blockDim.x) o.block_map[i] = R.bm[i];
-    if (threadIdx.x == 0) o.num_blocks[0] = R.nb;
-}
-
-// ---------------------------------------------------------------------------
-// Routing.  One cluster of kRouteCtas CTAs; CTA c owns experts
-// [c*EC, (c+1)*EC), EC = E / kRouteCtas <= 32.  The logit of (t, e) is 32
-// chains, chain p taking i = p, p+32, ... in ascending i with fused
-// multiply-add from 0, combined by the xor butterfly m = 16..1 (the value
-// lane p holds after step m is v_p + v_{p^m}, so the result is the tree that
-// adds chains q and q + m for q < m, m = 16..1), plus the bias.  Item
-// (p, el) of a CTA runs chain p of expert e0 + el for all T tokens: a group
-// of EC lanes reads EC consecutive floats of a W_r row per step, from a copy
-// of the CTA's W_r columns that the tensor-memory-access unit brings in, 256
-// rows per load (the load/store units reach a fraction of its rate for this
-// strided copy).  The logits go to CTA 0's shared memory (distributed shared
-// memory), which then routes.  Dynamic shared memory (128-byte aligned): the
-// W_r columns [d][EC] fp32, x [T][d] bf16, the chains [T][32][33] fp32.
-// ---------------------------------------------------------------------------
-__global__ void __cluster_dims__(kRouteCtas, 1, 1) __launch_bounds__(kRowThreads)
-decode_route_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t* __restrict__ x,
-                    const float* __restrict__ bias, int T, int d, int E, int k, int max_blocks,
-                    DecodeRouteOut ro, int32_t* __restrict__ status) {
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    __shared__ DecodeRoute R;
-    __shared__ __align__(8) uint64_t wbar;
-    __shared__ int no_abort;
-    extern __shared__ __align__(16) uint8_t dsm_raw[];
-    uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) &
-                                              ~static_cast<uintptr_t>(127));
-    const int EC = E / kRouteCtas;
-    float* ws = reinterpret_cast<float*>(dsm);  // [i][EC]
-    uint16_t* xs = reinterpret_cast<uint16_t*>(dsm + static_cast<size_t>(d) * EC * 4);
-    float* cs = reinterpret_cast<float*>(dsm + static_cast<size_t>(d) * EC * 4 +
-                                         static_cast<size_t>(T) * d * 2);  // [t][p][33]
-    pdl_launch_dependents();
-    const int rank = static_cast<int>(cluster.block_rank());
-    const int e0 = rank * EC;
-    const int nsteps = d >> 5;
-    const int items = 32 * EC;
-    const uint32_t bar = smem_u32(&wbar);
-    if (threadIdx.x == 0) {
-        // W_r[:, e0 .. e0+EC) -> ws in loads of 256 rows (e0 * 4 bytes is a
-        // multiple of 16: EC % 4 == 0)
-        no_abort = 0;
-        mbar_init(bar, 1);
-        fence_mbarrier_init();
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(d) * EC * 4);
-        for (int r0 = 0; r0 < d; r0 += kRouteRowsPerLoad)
-            tma_load_2d(smem_u32(ws + static_cast<size_t>(r0) * EC), &wmap, e0, r0, bar);
-    }
-    // x may be the output of the previous kernel in the stream (for example
-    // y of the previous call), so it is read only after that kernel has
-    // completed; W_r and the bias are never written by this library
-    pdl_wait();
-    cta_copy16(xs, x, T * d / 8);
-    __syncthreads();  // x in place; the barrier initialised
-    const bool w_ok = mbar_wait(bar, 0, &no_abort);
-    if (threadIdx.x == 0) cluster.map_shared_rank(R.cta_err, 0)[rank] = w_ok ? 0 : 1;
-    for (int it = threadIdx.x; it < items; it += kRowThreads) {
-        const int p = it / EC;
-        const int el = it - p * EC;
-#pragma unroll 1
-        for (int t = 0; t < T; ++t) {
-            float a = 0.0f;
-#pragma unroll 16
-            for (int s = 0; s < nsteps; ++s)
-                a = __fmaf_rn(bf16_bits_to_float(xs[t * d + 32 * s + p]), ws[(32 * s + p) * EC + el], a);
-            cs[(t * 32 + p) * 33 + el] = a;
-        }
-    }
-    __syncthreads();
-    float* lg0 = cluster.map_shared_rank(R.lg, 0);
-    for (int it = threadIdx.x; it < T * EC; it += kRowThreads) {
-        const int t = it / EC;
-        const int el = it - t * EC;
-        float v[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = cs[(t * 32 + q) * 33 + el];
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1)
-#pragma unroll
-            for (int q = 0; q < m; ++q) v[q] = __fadd_rn(v[q], v[q + m]);
-        lg0[t * E + e0 + el] = bias ? __fadd_rn(v[0], bias[e0 + el]) : v[0];
-    }
-    cluster.sync();  // all logits are in CTA 0; no CTA touches another's memory after this
-    if (rank != 0) return;
-    // the status word reports the most recent call: the first kernel clears it
-    if (threadIdx.x < 2) status[threadIdx.x] = 0;
-    __syncthreads();
-    if (threadIdx.x < kRouteCtas && R.cta_err[threadIdx.x])
-        report_error(status, MOE_ERR_DEVICE_TIMEOUT, 400 + threadIdx.x);
-    route_from_logits(T, E, k, max_blocks, R);
-    write_route(R, ro, T * k, E);
-}
-
-// ---------------------------------------------------------------------------
-// Expert GEMVs on the warp-level tensor-core MMA (m16n8k16, bf16 operands from
-// registers, fp32 accumulators).  A 16-row tile of packed weights is the A
-// operand and up to 8 operand rows (a block's tokens) are the 8 columns of B,
-// so the instruction count does not grow with the batch.
-//
-// Fragments (thread t of the warp: g = t / 4, c = t % 4): A holds rows g and
-// g + 8, logical K pairs c and c + 4; B holds column g, the same K pairs; the
-// accumulator holds rows g, g + 8 x columns 2c, 2c + 1.  Any one-to-one map of
-// the 16 logical K onto the data's K gives the same sum, so thread c takes word
-// c of a 32-wide nibble vector (K 8c .. 8c+7: nibble pair i is K 8c+2i at bits
-// 4i and 8c+2i+1 at bits 16+4i) for both of its rows: pairs 0 and 1 feed the
-// first MMA, pairs 2 and 3 the second, and its operand piece is the 16 bytes of
-// K 8c .. 8c+7 of its column.  A nibble pair becomes two bf16 values 128 + q
-// exactly (q in the mantissa of 128.0), so the MMA gives sum (128 + q) x; with
-// w = q s + b a group's dot product is s * D + (b - 128 s) * sum x, formed in
-// fp32 once per group (the MMAs of a 64-wide group accumulate together).  The
-// weights are not rounded to bf16 on this path.
-// ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
@@ -337,81 +164,57 @@ __device__ __forceinline__ void group_fold(float (&acc)[4], const float (&D)[4],
     acc[3] = fmaf(s1, D[3], fmaf(c1, xs1, acc[3]));
 }
 
-// Loads of one 16-row tile over a range of 64-wide K chunks: the tile's rows
-// g and g + 8 are packed rows pa and pb of blocks base + ch * bb; per chunk
-// word c of both halves of both rows, and the rows' (scale, bias) words.
-template <int kChunks, int kGpc>
-struct TileLoads {
-    uint32_t w[kChunks][4];         // row a half 0, row a half 1, row b half 0, row b half 1
-    uint32_t sc[kChunks][2 * kGpc];  // row a groups, row b groups
-};
+__device__ __forceinline__ uint32_t lds_u32(const uint8_t* p) {
+    return *reinterpret_cast<const uint32_t*>(p);
+}
 
-template <int kChunks, int kGpc>
-__device__ __forceinline__ void tile_load(TileLoads<kChunks, kGpc>& L, const uint8_t* base, int bb,
-                                          int nib_bytes, int pa, int pb, int ch0, int ch_step,
-                                          int KC, int c) {
-#pragma unroll
-    for (int u = 0; u < kChunks; ++u) {
-        const int ch = ch0 + u * ch_step;
-        if (ch < KC) {
-            const uint8_t* blk = base + static_cast<size_t>(ch) * bb;
-            L.w[u][0] = ld_nc_u32(blk + pa * 32 + 4 * c);
-            L.w[u][1] = ld_nc_u32(blk + pa * 32 + 16 + 4 * c);
-            L.w[u][2] = ld_nc_u32(blk + pb * 32 + 4 * c);
-            L.w[u][3] = ld_nc_u32(blk + pb * 32 + 16 + 4 * c);
-#pragma unroll
-            for (int q = 0; q < kGpc; ++q) {
-                L.sc[u][q] = ld_nc_u32(blk + nib_bytes + (pa * kGpc + q) * 4);
-                L.sc[u][kGpc + q] = ld_nc_u32(blk + nib_bytes + (pb * kGpc + q) * 4);
-            }
-        }
+// One 64-wide K chunk of a 16-row tile held in shared memory: blk = the
+// packed block (rows x 32 bytes of nibbles, then per row and group a (scale,
+// bias) word), rows ra and ra + 8; xrow = the thread's B column at K 8c of
+// this chunk; xs0, xs1 = the 32-wide vector sums of columns 2c, 2c + 1 at
+// this chunk's first vector.
+template <int kGpc>
+__device__ __forceinline__ void chunk_mma(float (&acc)[4], const uint8_t* blk, int nib_bytes, int ra,
+                                          int c, const uint16_t* xrow, const float* xs0,
+                                          const float* xs1) {
+    const int rb = ra + 8;
+    const uint32_t wa0 = lds_u32(blk + ra * 32 + 4 * c);
+    const uint32_t wa1 = lds_u32(blk + ra * 32 + 16 + 4 * c);
+    const uint32_t wb0 = lds_u32(blk + rb * 32 + 4 * c);
+    const uint32_t wb1 = lds_u32(blk + rb * 32 + 16 + 4 * c);
+    const uint4 xb0 = *reinterpret_cast<const uint4*>(xrow);
+    const uint4 xb1 = *reinterpret_cast<const uint4*>(xrow + 32);
+    float D[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    vector_mma(D, wa0, wb0, xb0);
+    if constexpr (kGpc == 2) {  // a group per 32-wide vector
+        group_fold(acc, D, lds_u32(blk + nib_bytes + (ra * 2) * 4), lds_u32(blk + nib_bytes + (rb * 2) * 4),
+                   xs0[0], xs1[0]);
+        D[0] = D[1] = D[2] = D[3] = 0.0f;
+        vector_mma(D, wa1, wb1, xb1);
+        group_fold(acc, D, lds_u32(blk + nib_bytes + (ra * 2 + 1) * 4),
+                   lds_u32(blk + nib_bytes + (rb * 2 + 1) * 4), xs0[1], xs1[1]);
+    } else {  // one group for the chunk: its four MMAs share the fold
+        vector_mma(D, wa1, wb1, xb1);
+        group_fold(acc, D, lds_u32(blk + nib_bytes + ra * 4), lds_u32(blk + nib_bytes + rb * 4),
+                   xs0[0] + xs0[1], xs1[0] + xs1[1]);
     }
 }
 
-// acc += the tile's dot products over the loaded chunks.  xrow: the thread's
-// column in shared memory, advanced to K 8c; xs0, xs1: vector sums of columns
-// 2c and 2c + 1.
-template <int kChunks, int kGpc>
-__device__ __forceinline__ void tile_dots(float (&acc)[4], const TileLoads<kChunks, kGpc>& L,
-                                          const uint16_t* xrow, const float* xs0, const float* xs1,
-                                          int ch0, int ch_step, int KC) {
-#pragma unroll
-    for (int u = 0; u < kChunks; ++u) {
-        const int ch = ch0 + u * ch_step;
-        if (ch < KC) {
-            const int v = 2 * ch;
-            const uint4 xb0 = *reinterpret_cast<const uint4*>(xrow + 32 * v);
-            const uint4 xb1 = *reinterpret_cast<const uint4*>(xrow + 32 * v + 32);
-            float D[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            vector_mma(D, L.w[u][0], L.w[u][2], xb0);
-            if (kGpc == 2) {  // a group per vector
-                group_fold(acc, D, L.sc[u][0], L.sc[u][2], xs0[v], xs1[v]);
-                D[0] = D[1] = D[2] = D[3] = 0.0f;
-                vector_mma(D, L.w[u][1], L.w[u][3], xb1);
-                group_fold(acc, D, L.sc[u][1], L.sc[u][3], xs0[v + 1], xs1[v + 1]);
-            } else {  // one group for the chunk: its four MMAs share the fold
-                vector_mma(D, L.w[u][1], L.w[u][3], xb1);
-                group_fold(acc, D, L.sc[u][0], L.sc[u][1], xs0[v] + xs0[v + 1], xs1[v] + xs1[v + 1]);
-            }
-        }
-    }
-}
-
-// Rows of bf16 operands (n_rows of w elements, row r at src row row_of(r))
-// into shared memory with a row stride of w + 32 elements (64 bytes of pad,
-// so the 8 columns' 16-byte reads fall in distinct banks), and each 32-wide
-// vector's sum (fp32, in K order) into sums [r][w/32].
+// Rows of bf16 operands into shared memory with a row stride of w + 32
+// elements (the eight columns' 16-byte reads then fall in distinct banks),
+// and each 32-wide vector's fp32 sum in K order into sums[r][w / 32].
+// Reads through L2 (the rows may have been written by other CTAs).
 template <class RowOf>
-__device__ __forceinline__ void cta_stage_rows(uint16_t* dst, float* sums, const uint16_t* src,
-                                               int n_rows, int w, RowOf row_of) {
+__device__ __forceinline__ void stage_rows(uint16_t* dst, float* sums, const uint16_t* src, int n_rows,
+                                           int w, RowOf row_of, int tid, int nthreads) {
     const int nv = w / 32;
-    for (int it = threadIdx.x; it < n_rows * nv; it += blockDim.x) {
+    for (int it = tid; it < n_rows * nv; it += nthreads) {
         const int r = it / nv;
         const int v = it - r * nv;
         const uint8_t* s = reinterpret_cast<const uint8_t*>(src + static_cast<size_t>(row_of(r)) * w + 32 * v);
         uint4 p[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) p[q] = ld_nc_v4(s + 16 * q);
+        for (int q = 0; q < 4; ++q) p[q] = ld_cg_v4(s + 16 * q);
         uint4* d4 = reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * (w + 32) + 32 * v);
         float acc = 0.0f;
 #pragma unroll
@@ -428,251 +231,640 @@ __device__ __forceinline__ void cta_stage_rows(uint16_t* dst, float* sums, const
     }
 }
 
-constexpr int kGuWarps = 4;   // K split of a gate/up CTA
-constexpr int kGuChunks = 8;  // 64-wide K chunks per warp: d <= 4 * 8 * 64
-constexpr int kGuFeat = 8;    // features per gate/up CTA: 8 gate + 8 up rows, one MMA tile
-constexpr int kDnWarps = 16;  // blocks in flight per down CTA
-template <int kGpc>
-constexpr int dn_chunks() { return kGpc == 1 ? 8 : 6; }  // down K chunks loaded together
+// Routing of the few tokens, in shared memory (identical in every CTA).
+struct DecRoute {
+    float sel[kDecMaxAssign];  // logit of each selected slot
+    int idx[kDecMaxAssign];
+    float w[kDecMaxAssign];
+    int sa[kDecMaxAssign];
+    int pos[kDecMaxAssign];
+    int cnt[kMaxExperts];
+    int off[kMaxExperts + 1];
+    int bo[kMaxExperts + 1];
+    int blk_e[kDecMaxAssign];  // block b: expert, first row, rows (one block per selected expert)
+    int blk_row0[kDecMaxAssign];
+    int blk_n[kDecMaxAssign];
+    int nb;
+    int sh_warp[kDecThreads / 32 + 1];
+    int flag;                  // broadcast of a thread-0 decision to the compute warps
+    int hok;                   // the h rows of a block became ready
+    int fail;                  // a compute warp gave up on the current unit
+    int abort_local;           // this CTA gave up
+};
 
-// ---------------------------------------------------------------------------
-// Gate/up and SwiGLU.  Grid: min(E, T*k) blocks x f/8 feature groups (CTAs
-// past the number of blocks return).  The MMA tile's rows g and g + 8 are the
-// gate and up rows of feature 8q + g, so SwiGLU happens in the thread that
-// holds both sums.  The four warps split K; their sums are added in warp
-// order.  Columns beyond the block's rows repeat its last row and are not
-// stored.  Dynamic shared memory: the block's x rows [T][d + 32] bf16, then
-// their vector sums [T][d/32] fp32.
-// ---------------------------------------------------------------------------
-template <int kGpc>
-__global__ void __launch_bounds__(kGuWarps * 32, kGpc == 1 ? 6 : 4)
-decode_gateup_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wpack, int T,
-                     int d, int k, int f, int bb, DecodeRouteOut ro, uint16_t* __restrict__ h) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ float red[kGuWarps - 1][4][32];
-    pdl_launch_dependents();
-    pdl_wait();
-    const int nfq = f / kGuFeat;
-    const int b = blockIdx.x / nfq;
-    const int fq = blockIdx.x - b * nfq;
-    const int nb = ro.num_blocks[0];
-    const int e = ro.block_map[3 * b];
-    const int row0 = ro.block_map[3 * b + 1];
-    const int cnt = ro.block_map[3 * b + 2];
-    if (b >= min(nb, kDecodeMaxAssign)) return;
-    const int nrows = min(cnt, T);  // a block holds at most one row per token
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int g = lane >> 2;
-    const int c = lane & 3;
-    const int KC = d / kKChunk;
-    const int j = fq * kGuFeat / 128;
-    const int pa = fq * kGuFeat % 128 + g;  // gate row; the up row is 128 further
-    const uint8_t* base = wpack + (static_cast<size_t>(e) * (f / 128) + j) * KC * bb;
-    TileLoads<kGuChunks, kGpc> L;
-    tile_load(L, base, bb, 2 * 128 * 32, pa, 128 + pa, warp, kGuWarps, KC, c);
-    uint16_t* xsh = reinterpret_cast<uint16_t*>(dsm);
-    float* xss = reinterpret_cast<float*>(dsm + static_cast<size_t>(T) * (d + 32) * 2);
-    const int32_t* sa = ro.sorted_assign + row0;
-    cta_stage_rows(xsh, xss, x, nrows, d, [&](int r) { return sa[r] / k; });
-    __syncthreads();
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const int nv = d / 32;
-    tile_dots(acc, L, xsh + min(g, nrows - 1) * (d + 32) + 8 * c, xss + min(2 * c, nrows - 1) * nv,
-              xss + min(2 * c + 1, nrows - 1) * nv, warp, kGuWarps, KC);
-    if (warp > 0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) red[warp - 1][i][lane] = acc[i];
+// top-k (each (token, expert) pair finds its slot; ties go to the lower id),
+// the softmax weights over the k slots, counts (integer atomics), offsets
+// (exclusive scan), one block per expert with rows (ascending expert), and
+// the stable scatter (rank of assignment a = number of earlier assignments
+// to its expert).  All kDecThreads threads.
+__device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int Tk = T * k;
+    if (tid < E) R.cnt[tid] = 0;
+    for (int it = tid; it < T * E; it += kDecThreads) {
+        const int t = it / E;
+        const int e = it - t * E;
+        const int slot = expert_slot(lg + t * E, E, e);
+        if (slot < k) {
+            R.idx[t * k + slot] = e;
+            R.sel[t * k + slot] = lg[it];
+        }
     }
     __syncthreads();
-    if (warp != 0) return;
-#pragma unroll
-    for (int w = 0; w < kGuWarps - 1; ++w)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += red[w][i][lane];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int r = 2 * c + i;
-        if (r < nrows) {
-            const float gv = acc[i];
-            const float uv = acc[2 + i];
-            h[static_cast<size_t>(row0 + r) * f + fq * kGuFeat + g] =
-                bf16_round_bits(__fdividef(gv * uv, 1.0f + __expf(-gv)));
+    for (int t = warp; t < T; t += kDecThreads / 32) {
+        const float wt = warp_slot_weights(lane < k ? R.sel[t * k + lane] : 0.0f, k, lane);
+        if (lane < k) R.w[t * k + lane] = wt;
+    }
+    for (int a = tid; a < Tk; a += kDecThreads) atomicAdd(&R.cnt[R.idx[a]], 1);
+    __syncthreads();
+    const int c = tid < E ? R.cnt[tid] : 0;
+    int total = 0;
+    const int off = block_exclusive_scan<kDecThreads>(c, R.sh_warp, &total);
+    if (tid < E) R.off[tid] = off;
+    if (tid == 0) R.off[E] = total;
+    // at most T <= 8 rows per expert: one block of the block map each
+    const int nt = c > 0 ? 1 : 0;
+    int nb = 0;
+    const int bo = block_exclusive_scan<kDecThreads>(nt, R.sh_warp, &nb);
+    if (tid < E) {
+        R.bo[tid] = bo;
+        if (nt) {
+            R.blk_e[bo] = tid;
+            R.blk_row0[bo] = off;
+            R.blk_n[bo] = c;
         }
+    }
+    if (tid == 0) {
+        R.bo[E] = nb;
+        R.nb = nb;
+    }
+    __syncthreads();
+    for (int a = tid; a < Tk; a += kDecThreads) {
+        const int e = R.idx[a];
+        int rank = 0;
+        for (int a2 = 0; a2 < a; ++a2) rank += R.idx[a2] == e;
+        const int p = R.off[e] + rank;
+        R.sa[p] = a;
+        R.pos[a] = p;
+    }
+    __syncthreads();
+}
+
+// Layout of the dynamic shared memory (byte offsets; the base is 1024-aligned).
+struct DecSmem {
+    int ring, x, xsum, h, hsum, lg, route, bars, total;
+};
+__host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
+    DecSmem L;
+    int o = 0;
+    auto take = [&](int bytes) {
+        const int r = o;
+        o = (o + bytes + 127) / 128 * 128;
+        return r;
+    };
+    L.ring = take(kDecStages * kDecStageBytes);
+    L.x = take(T * (d + 32) * 2);
+    L.xsum = take(T * (d / 32) * 4);
+    L.h = take(kDecodeMaxT * (f + 32) * 2);
+    L.hsum = take(kDecodeMaxT * (f / 32) * 4);
+    L.lg = take(T * E * 4);
+    L.route = take(static_cast<int>(sizeof(DecRoute)));
+    L.bars = take((2 * kDecStages + 1) * 8);
+    L.total = o + 1024;  // + slack to align the base
+    return L;
+}
+
+struct DecParams {
+    int T, d, E, k, f;
+    const uint16_t* x;
+    const float* b_r;
+    const uint8_t* wgu;   // packed gate/up blocks [E][f/128][d/64][bb_gu]
+    const uint8_t* wdn;   // packed down blocks [E][d/128][f/64][bb_dn]
+    int bb_gu, bb_dn;
+    int32_t *topk_idx, *counts, *offsets, *sorted_assign, *pos, *block_offsets, *block_map,
+        *num_blocks;
+    float* topk_w;
+    float* U;             // router partials [T][E][8]
+    float* pgu;           // gate/up partial sums [T*k][f/128][KS][256]
+    float* pdn;           // down partial sums [T*k][d/128][DS][128]
+    uint16_t* h;          // [T*k][f]
+    uint16_t* y;          // [T][d]
+    int32_t* status;
+    int32_t* sync;        // the decode flags
+};
+
+// Wait until *flag >= target (thread-level, bounded; also gives up when the
+// call's abort flag is raised).  Returns false on giving up.
+__device__ __forceinline__ bool wait_flag(const int* flag, int target, const int* abort) {
+    if (ld_acquire(flag) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t n = 1;; ++n) {
+        if (ld_acquire(flag) >= target) return true;
+        if ((n & 15u) == 0) {
+            if (ld_acquire(abort) != 0) return false;
+            if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+        }
+        __nanosleep(32);
     }
 }
 
-// ---------------------------------------------------------------------------
-// Down projection and combine.  Grid: d/16 CTAs; CTA m owns output features
-// 16m .. 16m+15 (one MMA tile: rows 16m % 128 + g and + 8 of down tile
-// 16m / 128).  The tile against a block's h rows gives each of the block's
-// assignments its 16 outputs.  With at most 8 blocks a pair of warps takes a
-// block, one K half each; otherwise warp w takes blocks w, w + 16, ... over
-// all of K.  The two halves' sums (the second is zero for a whole-K warp) are
-// added and rounded to bf16 (the expert output o), then thread (t, r) sums o
-// over token t's slots in slot order.  Dynamic shared memory: h [T*k][f + 32]
-// bf16, then its vector sums [T*k][f/32] fp32.
-// ---------------------------------------------------------------------------
-template <int kGpc>
-__global__ void __launch_bounds__(kDnWarps * 32, 1)
-decode_down_kernel(const uint8_t* __restrict__ wpack, const uint16_t* __restrict__ h, int T,
-                   int d, int k, int f, int bb, int nb_max, DecodeRouteOut ro,
-                   uint16_t* __restrict__ y) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ int spos[kDecodeMaxAssign];
-    __shared__ float sw[kDecodeMaxAssign];
-    __shared__ int sbm[3 * kDecodeMaxAssign];
-    __shared__ float op[2][kDecodeMaxAssign][16];  // K-half sums of each assignment's outputs
-    __shared__ int snb;
-    const int Tk = T * k;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int g = lane >> 2;
-    const int c = lane & 3;
-    pdl_wait();  // h and the routing
-    if (threadIdx.x == 0) snb = min(ro.num_blocks[0], nb_max);
-    for (int i = threadIdx.x; i < Tk; i += blockDim.x) {
-        spos[i] = ro.pos[i];
-        sw[i] = ro.topk_w[i];
-    }
-    for (int i = threadIdx.x; i < 3 * nb_max; i += blockDim.x) sbm[i] = ro.block_map[i];
-    uint16_t* hsh = reinterpret_cast<uint16_t*>(dsm);
-    float* hss = reinterpret_cast<float*>(dsm + static_cast<size_t>(Tk) * (f + 32) * 2);
-    cta_stage_rows(hsh, hss, h, Tk, f, [](int r) { return r; });
-    __syncthreads();
-    const int nb = snb;
-    const int m0 = blockIdx.x * 16;
-    const int jd = m0 / 128;
-    const int pa = m0 % 128 + g;
-    const int KC = f / kKChunk;
-    const int nv = f / 32;
-    constexpr int kCh = dn_chunks<kGpc>();
-    const int split = nb <= kDnWarps / 2 ? 2 : 1;
-    const int part = warp % split;
-    const int kc_part = (KC + split - 1) / split;
-    const int ch_begin = part * kc_part;
-    const int ch_end = min(KC, ch_begin + kc_part);
-    for (int b = warp / split; b < nb; b += kDnWarps / split) {
-        const int brow0 = sbm[3 * b + 1];
-        const int brows = min(sbm[3 * b + 2], T);
-        const uint8_t* base = wpack + (static_cast<size_t>(sbm[3 * b]) * (d / 128) + jd) * KC * bb;
-        const uint16_t* xrow = hsh + (brow0 + min(g, brows - 1)) * (f + 32) + 8 * c;
-        const float* xs0 = hss + (brow0 + min(2 * c, brows - 1)) * nv;
-        const float* xs1 = hss + (brow0 + min(2 * c + 1, brows - 1)) * nv;
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int ch0 = ch_begin; ch0 < ch_end; ch0 += kCh) {
-            TileLoads<kCh, kGpc> L;
-            tile_load(L, base, bb, 128 * 32, pa, pa + 8, ch0, 1, ch_end, c);
-            tile_dots(acc, L, xrow, xs0, xs1, ch0, 1, ch_end);
+// Wait until the flags region carries both magic words (CTA 0 writes them
+// after zeroing the region, the second one last, with release order).
+__device__ __forceinline__ bool wait_magic(const int* sync, const int* abort) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t n = 0;; ++n) {
+        if (static_cast<uint32_t>(ld_acquire(sync + kSyncMagic + 1)) == kDecMagic1 &&
+            static_cast<uint32_t>(ld_acquire(sync + kSyncMagic)) == kDecMagic0)
+            return true;
+        if ((n & 15u) == 15u) {
+            if (ld_acquire(abort) != 0) return false;
+            if (globaltimer() - t0 > kWaitTimeoutNs) return false;
         }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = 2 * c + i;
-            if (r < brows) {
-                op[part][brow0 + r][g] = acc[i];
-                op[part][brow0 + r][g + 8] = acc[2 + i];
+        __nanosleep(32);
+    }
+}
+
+__device__ __forceinline__ int vload(const int& v) { return *reinterpret_cast<const volatile int*>(&v); }
+
+// the thread that gives up: record the error and stop every CTA of the call
+__device__ __forceinline__ void dec_fail(const DecParams& p, DecRoute& R, int detail) {
+    report_error(p.status, MOE_ERR_DEVICE_TIMEOUT, detail);
+    st_release(p.sync + kSyncAbort, 1);
+    R.abort_local = 1;
+}
+
+template <int kGpc>
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ DecParams p) {
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    pdl_launch_dependents();
+    const int T = p.T, d = p.d, E = p.E, k = p.k, f = p.f;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int G = gridDim.x;
+    const int cta = blockIdx.x;
+    const DecSmem L = dec_smem_layout(T, d, E, f);
+    uint8_t* ring = smem + L.ring;
+    uint16_t* xsh = reinterpret_cast<uint16_t*>(smem + L.x);
+    float* xsum = reinterpret_cast<float*>(smem + L.xsum);
+    uint16_t* hsh = reinterpret_cast<uint16_t*>(smem + L.h);
+    float* hsum = reinterpret_cast<float*>(smem + L.hsum);
+    float* lg = reinterpret_cast<float*>(smem + L.lg);
+    DecRoute& R = *reinterpret_cast<DecRoute*>(smem + L.route);
+    const uint32_t bar0 = smem_u32(smem + L.bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (kDecStages + s); };
+    const uint32_t wbar = bar0 + 8u * (2 * kDecStages);
+    int32_t* sync = p.sync;
+    const int* abort_g = sync + kSyncAbort;
+
+    // routing items of this CTA: item i = (octet i >> 3, residue i & 7)
+    const int my_items = cta < E ? (E - 1 - cta) / G + 1 : 0;
+    const int item_bytes = (d / 8) * 32;
+    if (tid == 0) {
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), kDecComputeWarps);
+        }
+        mbar_init(wbar, 1);
+        R.abort_local = 0;
+        fence_mbarrier_init();
+        // W_r pieces (model weights, never written by this library: loaded
+        // before waiting for the previous kernel): rows i = 8j + r, j < d/8,
+        // of the item's 8 experts, [j][8] fp32
+        if (my_items > 0) {
+            mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(my_items * item_bytes));
+            for (int ii = 0; ii < my_items; ++ii) {
+                const int item = cta + ii * G;
+                for (int j0 = 0; j0 < d / 8; j0 += kDecWRows)
+                    tma_load_3d(smem_u32(ring + ii * item_bytes + j0 * 32), &wmap, 8 * (item >> 3), item & 7,
+                                j0, wbar);
             }
         }
     }
-    if (split == 1) {  // whole-K sums: the second half is zero (no warp writes op[1])
-        for (int i = threadIdx.x; i < Tk * 16; i += blockDim.x) op[1][i >> 4][i & 15] = 0.0f;
+    // x may be the output of the previous kernel in the stream (for example
+    // y of the previous call): read it, and the workspace, only after that
+    // kernel has completed
+    pdl_wait();
+    stage_rows(xsh, xsum, p.x, T, d, [](int r) { return r; }, tid, kDecThreads);
+    if (cta == 0 && tid == 0) {
+        // the status word reports the most recent call; the flags region is
+        // zeroed on first use (and reset by the last CTA of every call)
+        p.status[0] = 0;
+        p.status[1] = 0;
+        R.flag = !(static_cast<uint32_t>(sync[kSyncMagic]) == kDecMagic0 &&
+                   static_cast<uint32_t>(sync[kSyncMagic + 1]) == kDecMagic1);
     }
     __syncthreads();
-    if (threadIdx.x < 16 * T) {
-        const int t = threadIdx.x >> 4;
-        const int r = threadIdx.x & 15;
-        float acc = 0.0f;
-        for (int jj = 0; jj < k; ++jj) {
-            const int pj = spos[t * k + jj];
-            const float o = __bfloat162float(__float2bfloat16_rn(op[0][pj][r] + op[1][pj][r]));
-            acc = fmaf(sw[t * k + jj], o, acc);
+    if (cta == 0 && vload(R.flag)) {
+        for (int i = tid + 2; i < kSyncInts; i += kDecThreads) sync[i] = 0;
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            sync[kSyncMagic] = static_cast<int>(kDecMagic0);
+            __threadfence();
+            st_release(sync + kSyncMagic + 1, static_cast<int>(kDecMagic1));
         }
-        y[static_cast<size_t>(t) * d + m0 + r] = bf16_round_bits(acc);
+    }
+
+    // ---- phase 1: router partials ----------------------------------------
+    // chain p = r + 8q (q < 4) of expert 8o + el and token t runs
+    // i = p, p + 32, ... with fused multiply-add from 0; lanes 4m .. 4m + 3
+    // hold q = 0..3 of one (t, el), and u_r = (c_r + c_{r+16}) + (c_{r+8} + c_{r+24})
+    // is the value the router's butterfly holds at chain r after its levels
+    // 16 and 8
+    if (my_items > 0) {
+        // every thread waits; the outcome is made uniform before any shuffle
+        const bool w_ok = __syncthreads_and(mbar_wait(wbar, 0, &R.abort_local)) != 0;
+        if (!w_ok && tid == 0) dec_fail(p, R, 500);
+        if (w_ok) {
+            for (int ii = 0; ii < my_items; ++ii) {
+                const int item = cta + ii * G;
+                const int o = item >> 3;
+                const int r = item & 7;
+                const float* wsl = reinterpret_cast<const float*>(ring + ii * item_bytes);
+                for (int ch = tid; ch < T * 32; ch += kDecThreads) {  // T * 32 <= 256: one pass
+                    const int q = ch & 3;
+                    const int el = (ch >> 2) & 7;
+                    const int t = ch >> 5;
+                    const uint16_t* xr = xsh + t * (d + 32) + r + 8 * q;
+                    const float* wr = wsl + q * 8 + el;
+                    float acc = 0.0f;
+#pragma unroll 8
+                    for (int m = 0; m < d / 32; ++m)
+                        acc = __fmaf_rn(bf16_bits_to_float(xr[32 * m]), wr[32 * m], acc);
+                    const float s02 = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
+                    const float u = __fadd_rn(s02, __shfl_xor_sync(0xffffffffu, s02, 1));
+                    if (q == 0) p.U[(static_cast<size_t>(t) * E + 8 * o + el) * 8 + r] = u;
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        bool ok = !vload(R.abort_local);
+        if (ok && !wait_magic(sync, abort_g)) {
+            dec_fail(p, R, 501);
+            ok = false;
+        }
+        if (my_items > 0) red_release_add(sync + kSyncRoute, my_items);  // counted even on failure
+        if (ok && !wait_flag(sync + kSyncRoute, E, abort_g)) dec_fail(p, R, 502);
+    }
+    __syncthreads();
+
+    // ---- phase 2: routing (every CTA) ---------------------------------------
+    if (!vload(R.abort_local)) {
+        for (int it = tid; it < T * E; it += kDecThreads) {
+            const uint4 ua = ld_cg_v4(p.U + static_cast<size_t>(it) * 8);
+            const uint4 ub = ld_cg_v4(p.U + static_cast<size_t>(it) * 8 + 4);
+            const float4 a = make_float4(__uint_as_float(ua.x), __uint_as_float(ua.y),
+                                         __uint_as_float(ua.z), __uint_as_float(ua.w));
+            const float4 b = make_float4(__uint_as_float(ub.x), __uint_as_float(ub.y),
+                                         __uint_as_float(ub.z), __uint_as_float(ub.w));
+            // levels 4, 2, 1 of the butterfly: ((u0+u4) + (u2+u6)) + ((u1+u5) + (u3+u7))
+            const float S = __fadd_rn(__fadd_rn(__fadd_rn(a.x, b.x), __fadd_rn(a.z, b.z)),
+                                      __fadd_rn(__fadd_rn(a.y, b.y), __fadd_rn(a.w, b.w)));
+            lg[it] = p.b_r != nullptr ? __fadd_rn(S, __ldg(p.b_r + (it % E))) : S;
+        }
+    }
+    __syncthreads();
+    const bool routed = !vload(R.abort_local);
+    if (routed) route_small(lg, T, E, k, R);
+    const int nb = routed ? R.nb : 0;
+    const int Tk = T * k;
+    if (cta == 0 && routed) {
+        for (int a = tid; a < Tk; a += kDecThreads) {
+            p.topk_idx[a] = R.idx[a];
+            p.topk_w[a] = R.w[a];
+            p.sorted_assign[a] = R.sa[a];
+            p.pos[a] = R.pos[a];
+        }
+        for (int e = tid; e <= E; e += kDecThreads) {
+            if (e < E) p.counts[e] = R.cnt[e];
+            p.offsets[e] = R.off[e];
+            p.block_offsets[e] = R.bo[e];
+        }
+        for (int b = tid; b < nb; b += kDecThreads) {
+            p.block_map[3 * b + 0] = R.blk_e[b];
+            p.block_map[3 * b + 1] = R.blk_row0[b];
+            p.block_map[3 * b + 2] = R.blk_n[b];
+        }
+        if (tid == 0) p.num_blocks[0] = nb;
+    }
+
+    // ---- phase 3: expert units ------------------------------------------------
+    const int NT = f / 128, KC = d / kKChunk, KS = KC / kDecGuChunks;
+    const int NTd = d / 128, KCd = f / kKChunk;
+    const int DS = (KCd % 4 == 0) ? 2 : 1;  // K halves of a down unit
+    const int dn_chunks = KCd / DS;         // chunks per down unit (even)
+    const int u_gu = nb * NT * KS;
+    const int u_total = u_gu + nb * NTd * DS;
+
+    if (warp == kDecProducerWarp) {
+        // the whole warp runs the loop; one elected lane issues the copies
+        uint32_t q = 0;
+        bool ok = true;
+        for (int i = cta; ok && i < u_total; i += G) {
+            const uint8_t* src;
+            int nst;
+            if (i < u_gu) {
+                const int b = i / (NT * KS);
+                const int j = (i / KS) % NT;
+                const int s = i % KS;
+                src = p.wgu + ((static_cast<size_t>(R.blk_e[b]) * NT + j) * KC + s * kDecGuChunks) * p.bb_gu;
+                nst = kDecGuChunks;
+            } else {
+                const int v = i - u_gu;
+                const int b = v / (NTd * DS);
+                const int jd = (v / DS) % NTd;
+                const int s2 = v % DS;
+                src = p.wdn + ((static_cast<size_t>(R.blk_e[b]) * NTd + jd) * KCd + s2 * dn_chunks) * p.bb_dn;
+                nst = dn_chunks / 2;
+            }
+            // one stage = one gate/up block = two consecutive down blocks (same bytes)
+            for (int st = 0; st < nst; ++st, ++q) {
+                const int slot = q % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(empty(slot), ((q / kDecStages) & 1) ^ 1, &R.abort_local))) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(p.bb_gu));
+                    bulk_copy_g2s(smem_u32(ring + slot * kDecStageBytes), src + static_cast<size_t>(st) * p.bb_gu,
+                                  static_cast<uint32_t>(p.bb_gu), full(slot));
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok && lane == 0) {
+            if (!vload(R.abort_local)) dec_fail(p, R, 503);
+            // let the copies already issued land before the CTA exits
+            const uint32_t first = q > kDecStages ? q - kDecStages : 0;
+            for (uint32_t i = first; i < q; ++i) {
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(full(i % kDecStages), (i / kDecStages) & 1))
+                    if (globaltimer() - t0 > 200000000ull) break;
+            }
+        }
+    } else {
+        // compute warps: MMA fragment coordinates
+        const int g = lane >> 2;
+        const int c = lane & 3;
+        uint32_t q = 0;
+        int h_block = -1;  // block whose h rows are staged in hsh
+        const int nvd = d / 32, nvf = f / 32;
+        for (int i = cta; i < u_total; i += G) {
+            const bool gu = i < u_gu;
+            int b, j, s;
+            if (gu) {
+                b = i / (NT * KS);
+                j = (i / KS) % NT;
+                s = i % KS;
+            } else {
+                const int v = i - u_gu;
+                b = v / (NTd * DS);
+                j = (v / DS) % NTd;
+                s = v % DS;
+            }
+            const int row0 = R.blk_row0[b];
+            const int n = R.blk_n[b];
+            if (!gu && h_block != b) {
+                // h rows of this block: wait until all its gate/up tiles are in
+                if (tid == 0) {
+                    R.hok = 1;
+                    if (!wait_flag(sync + kSyncHReady + b, NT, abort_g)) {
+                        dec_fail(p, R, 504);
+                        R.hok = 0;
+                    }
+                }
+                compute_sync();  // also: every warp is done with the previous h rows
+                if (!vload(R.hok)) break;
+                stage_rows(hsh, hsum, p.h + static_cast<size_t>(row0) * f, n, f, [](int r) { return r; }, tid,
+                           kDecComputeThreads);
+                compute_sync();
+                h_block = b;
+            }
+            // B columns: column g is row min(g, n-1) of the block; the
+            // accumulator's columns 2c, 2c + 1 need their vector sums
+            const int cg = min(g, n - 1), c0 = min(2 * c, n - 1), c1 = min(2 * c + 1, n - 1);
+            const uint16_t* brow;
+            const float *bs0, *bs1;
+            if (gu) {
+                brow = xsh + (R.sa[row0 + cg] / k) * (d + 32) + 8 * c;
+                bs0 = xsum + (R.sa[row0 + c0] / k) * nvd;
+                bs1 = xsum + (R.sa[row0 + c1] / k) * nvd;
+            } else {
+                brow = hsh + cg * (f + 32) + 8 * c;
+                bs0 = hsum + c0 * nvf;
+                bs1 = hsum + c1 * nvf;
+            }
+            // gate/up: warp w takes rows 32w .. 32w + 31 of the 256-row block
+            // (two 16-row tiles); down: rows 16w .. 16w + 15 of the 128-row tile
+            float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+            const int nst = gu ? kDecGuChunks : dn_chunks / 2;
+            if (tid == 0) R.fail = 0;
+            compute_sync();
+            for (int st = 0; st < nst; ++st, ++q) {
+                const int slot = q % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
+                    // give up on this unit; the others learn of it at the
+                    // barrier below, so every compute warp leaves together
+                    if (lane == 0) {
+                        R.fail = 1;
+                        if (!vload(R.abort_local)) dec_fail(p, R, 505);
+                    }
+                    continue;
+                }
+                const uint8_t* stage = ring + slot * kDecStageBytes;
+                if (gu) {
+                    const int kc = s * kDecGuChunks + st;  // K chunk of d
+                    const uint16_t* xr = brow + kKChunk * kc;
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt)
+                        chunk_mma<kGpc>(acc[tt], stage, 256 * 32, 32 * warp + 16 * tt + g, c, xr,
+                                        bs0 + 2 * kc, bs1 + 2 * kc);
+                } else {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int kc = s * dn_chunks + 2 * st + half;  // K chunk of f
+                        chunk_mma<kGpc>(acc[0], stage + half * p.bb_dn, 128 * 32, 16 * warp + g, c,
+                                        brow + kKChunk * kc, bs0 + 2 * kc, bs1 + 2 * kc);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty(slot));
+            }
+            compute_sync();
+            if (vload(R.fail)) break;
+            // partial sums of this unit -> workspace, then count the unit
+            if (gu) {
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    const int ra = 32 * warp + 16 * tt + g;
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int col = 2 * c + e2;
+                        if (col < n) {
+                            float* dst = p.pgu + ((static_cast<size_t>(row0 + col) * NT + j) * KS + s) * 256;
+                            dst[ra] = acc[tt][e2];
+                            dst[ra + 8] = acc[tt][2 + e2];
+                        }
+                    }
+                }
+            } else {
+                const int ra = 16 * warp + g;
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int col = 2 * c + e2;
+                    if (col < n) {
+                        float* dst = p.pdn + ((static_cast<size_t>(row0 + col) * NTd + j) * DS + s) * 128;
+                        dst[ra] = acc[0][e2];
+                        dst[ra + 8] = acc[0][2 + e2];
+                    }
+                }
+            }
+            __threadfence();
+            compute_sync();
+            if (tid == 0) {
+                int* cnt = gu ? sync + kSyncGu + b * NT + j : sync + kSyncDn + j;
+                const int last = gu ? KS - 1 : nb * DS - 1;
+                R.flag = atom_acq_rel_add(cnt, 1) == last;
+            }
+            compute_sync();
+            if (vload(R.flag)) {
+                if (gu) {
+                    // the block's h for this tile: sum the K parts in order,
+                    // SwiGLU, round to bf16
+                    for (int it = tid; it < 128 * n; it += kDecComputeThreads) {
+                        const int r = it & 127;
+                        const int col = it >> 7;
+                        const float* src = p.pgu + (static_cast<size_t>(row0 + col) * NT + j) * KS * 256;
+                        float gs = 0.0f, us = 0.0f;
+                        for (int s2 = 0; s2 < KS; ++s2) {
+                            gs += ld_cg_f32(src + s2 * 256 + r);
+                            us += ld_cg_f32(src + s2 * 256 + 128 + r);
+                        }
+                        p.h[static_cast<size_t>(row0 + col) * f + j * 128 + r] =
+                            bf16_round_bits(__fdividef(gs * us, 1.0f + __expf(-gs)));
+                    }
+                    __threadfence();
+                    compute_sync();
+                    if (tid == 0) red_release_add(sync + kSyncHReady + b, 1);
+                } else {
+                    // output tile j of every token: each expert output is the sum
+                    // of its K halves rounded to bf16; the token's slots are
+                    // summed in slot order
+                    for (int it = tid; it < 128 * T; it += kDecComputeThreads) {
+                        const int m = it & 127;
+                        const int t = it >> 7;
+                        float yv = 0.0f;
+                        for (int jj = 0; jj < k; ++jj) {
+                            const int pr = R.pos[t * k + jj];
+                            const float* src = p.pdn + (static_cast<size_t>(pr) * NTd + j) * DS * 128 + m;
+                            float o = ld_cg_f32(src);
+                            for (int s2 = 1; s2 < DS; ++s2) o += ld_cg_f32(src + s2 * 128);
+                            yv = fmaf(R.w[t * k + jj], bf16_round(o), yv);
+                        }
+                        p.y[static_cast<size_t>(t) * d + j * 128 + m] = bf16_round_bits(yv);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- phase 4: exit; the last CTA resets the flags ----------------------
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        R.flag = atom_acq_rel_add(sync + kSyncExit, 1) == G - 1;
+    }
+    __syncthreads();
+    if (vload(R.flag)) {
+        for (int i = tid + 2; i < kSyncInts; i += kDecThreads) sync[i] = 0;
+        __threadfence();
     }
 }
 
-constexpr size_t kGuSmemLimit = 64 * 1024;
-constexpr size_t kDnSmemLimit = 180 * 1024;
-constexpr size_t kRouteSmemLimit = 200 * 1024;
-
-size_t route_smem_bytes(const moe_shape_t& s, int T) {
-    return 128 + static_cast<size_t>(T) * s.d * 2 + static_cast<size_t>(s.d) * (s.E / kRouteCtas) * 4 +
-           static_cast<size_t>(T) * 32 * 33 * 4;  // + slack to align the base
-}
-
-// gate/up: the block's x rows (at most T) and their vector sums; down: every
-// assignment's h row and its vector sums
-size_t gateup_smem_bytes(const moe_shape_t& s, int T) {
-    return static_cast<size_t>(T) * ((s.d + 32) * 2 + (s.d / 32) * 4);
-}
-size_t down_smem_bytes(const moe_shape_t& s, int T) {
-    return static_cast<size_t>(T) * s.k * ((s.f + 32) * 2 + (s.f / 32) * 4);
-}
-
-template <int kGpc>
-cudaError_t set_expert_kernel_smem() {
-    cudaError_t e = cudaFuncSetAttribute(decode_gateup_kernel<kGpc>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kGuSmemLimit));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(decode_down_kernel<kGpc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(kDnSmemLimit));
-}
-
-template <int kGpc>
-cudaError_t launch_experts(const DecodeArgs& a, const DecodeRouteOut& ro, cudaStream_t st,
-                           void* ev_gate_up) {
-    const moe_shape_t& s = a.s;
-    const int nb_max = std::min(s.E, a.T * s.k);
-    cudaError_t e = launch_pdl(decode_gateup_kernel<kGpc>, dim3(nb_max * (s.f / kGuFeat)),
-                               dim3(kGuWarps * 32), gateup_smem_bytes(s, a.T), st, a.x, a.wpack_gu,
-                               a.T, s.d, s.k, s.f, a.gu_block_bytes, ro, a.h);
-    if (e != cudaSuccess) return e;
-    if (ev_gate_up && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_gate_up), st)) != cudaSuccess)
-        return e;
-    return launch_pdl(decode_down_kernel<kGpc>, dim3(s.d / 16), dim3(kDnWarps * 32),
-                      down_smem_bytes(s, a.T), st, a.wpack_dn, static_cast<const uint16_t*>(a.h),
-                      a.T, s.d, s.k, s.f, a.dn_block_bytes, nb_max, ro, a.y);
-}
+constexpr int kDecSmemLimit = 227 * 1024;
 
 }  // namespace
 
 bool decode_supported(const moe_shape_t& s, int T) {
     if (T < 1 || T > kDecodeMaxT) return false;
-    if (T * s.k > kDecodeMaxAssign || s.E > kMaxExperts) return false;
-    // whole 16-byte vectors of W_r columns per routing CTA
-    if (s.E % (4 * kRouteCtas) != 0 || route_smem_bytes(s, T) > kRouteSmemLimit) return false;
-    // (groups of 32 or 64 and d, f in whole tiles hold for every plan) a
-    // gate/up warp's K chunks fit in its registers
-    if (s.d > kGuWarps * kGuChunks * kKChunk) return false;
-    return gateup_smem_bytes(s, T) <= kGuSmemLimit && down_smem_bytes(s, T) <= kDnSmemLimit;
+    if (T * s.k > kDecMaxAssign || s.E > kMaxExperts || s.E % 8 != 0) return false;
+    if (s.f / 128 > kDecMaxNT || s.d / 128 > kDecMaxNTd) return false;
+    return dec_smem_layout(T, s.d, s.E, s.f).total <= kDecSmemLimit;
+}
+
+size_t decode_workspace_bytes(const moe_shape_t& s, int T_max) {
+    const size_t T = static_cast<size_t>(std::min(T_max, kDecodeMaxT));
+    const size_t Tk = T * s.k;
+    const size_t KS = (s.d / kKChunk) / kDecGuChunks;
+    const size_t DS = ((s.f / kKChunk) % 4 == 0) ? 2 : 1;
+    const size_t u = T * s.E * 8 * 4;
+    const size_t gu = Tk * (s.f / 128) * KS * 256 * 4;
+    const size_t dn = Tk * (s.d / 128) * DS * 128 * 4;
+    auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
+    return r256(u) + r256(gu) + r256(dn);
 }
 
 cudaError_t prepare_decode_kernels() {
-    cudaError_t e = cudaFuncSetAttribute(decode_route_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kRouteSmemLimit));
+    cudaError_t e = cudaFuncSetAttribute(decode_layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDecSmemLimit);
     if (e != cudaSuccess) return e;
-    if ((e = set_expert_kernel_smem<1>()) != cudaSuccess) return e;
-    return set_expert_kernel_smem<2>();
+    return cudaFuncSetAttribute(decode_layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kDecSmemLimit);
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed, void* ev_gate_up) {
+cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t st) {
     const moe_shape_t& s = a.s;
-    const int T = a.T;
-    const DecodeRouteOut ro{a.topk_idx, a.topk_w,        a.counts,    a.offsets,   a.sorted_assign,
-                            a.pos,      a.block_offsets, a.block_map, a.num_blocks};
-    const size_t route_smem = route_smem_bytes(s, T);
     CUtensorMap wmap;
-    cudaError_t e = encode_f32_cols_map(&wmap, a.W_r, s.d, s.E, s.E / kRouteCtas, kRouteRowsPerLoad);
+    cudaError_t e = encode_f32_3d_map(&wmap, a.W_r, static_cast<uint64_t>(s.E), 8, static_cast<uint64_t>(s.d / 8),
+                                      8, 1, static_cast<uint32_t>(std::min(s.d / 8, kDecWRows)));
     if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_route_kernel, dim3(kRouteCtas), dim3(kRowThreads), route_smem, st, wmap, a.x,
-                   a.b_r, T, s.d, s.E, s.k, a.max_blocks, ro, a.status);
-    if (e != cudaSuccess) return e;
-    if (ev_routed && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_routed), st)) != cudaSuccess)
-        return e;
-    return s.group == 64 ? launch_experts<1>(a, ro, st, ev_gate_up)
-                         : launch_experts<2>(a, ro, st, ev_gate_up);
+    DecParams p{};
+    p.T = a.T;
+    p.d = s.d;
+    p.E = s.E;
+    p.k = s.k;
+    p.f = s.f;
+    p.x = a.x;
+    p.b_r = a.b_r;
+    p.wgu = a.wpack_gu;
+    p.wdn = a.wpack_dn;
+    p.bb_gu = a.gu_block_bytes;
+    p.bb_dn = a.dn_block_bytes;
+    p.topk_idx = a.topk_idx;
+    p.counts = a.counts;
+    p.offsets = a.offsets;
+    p.sorted_assign = a.sorted_assign;
+    p.pos = a.pos;
+    p.block_offsets = a.block_offsets;
+    p.block_map = a.block_map;
+    p.num_blocks = a.num_blocks;
+    p.topk_w = a.topk_w;
+    const size_t T = static_cast<size_t>(a.T);
+    const size_t Tk = T * s.k;
+    const size_t KS = (s.d / kKChunk) / kDecGuChunks;
+    auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
+    uint8_t* scratch = a.scratch;
+    p.U = reinterpret_cast<float*>(scratch);
+    p.pgu = reinterpret_cast<float*>(scratch + r256(T * s.E * 8 * 4));
+    p.pdn = reinterpret_cast<float*>(scratch + r256(T * s.E * 8 * 4) + r256(Tk * (s.f / 128) * KS * 256 * 4));
+    p.h = a.h;
+    p.y = a.y;
+    p.status = a.status;
+    p.sync = a.sync;
+    const int smem = dec_smem_layout(a.T, s.d, s.E, s.f).total;
+    if (s.group == 64)
+        return launch_pdl(decode_layer_kernel<1>, dim3(num_sms), dim3(kDecThreads), smem, st, wmap, p);
+    return launch_pdl(decode_layer_kernel<2>, dim3(num_sms), dim3(kDecThreads), smem, st, wmap, p);
 }
 
 }  // namespace moe

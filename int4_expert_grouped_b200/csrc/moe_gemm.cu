@@ -6,7 +6,8 @@
 //   prepack_kernel        logical nibbles/scales -> per (expert, tile, K chunk)
 //                         contiguous blocks in the order the GEMM reads them
 //   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
-//       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order,
+//       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order
+//                (xs[p] = x[sorted_assign[p] / k], gathered on load),
 //                epilogue h = silu(D0) * D1 -> bf16 h rows
 //       down:    D = kDownTiles 128-row tiles of Wd times h^T, epilogue
 //                o = bf16(D) rows
@@ -30,8 +31,9 @@
 //   warp 0       bulk-copies packed weight blocks into the W ring (TMA engine)
 //   warp 1       allocates TMEM; runs the MMA loop, one elected lane issues
 //                tcgen05.mma and tcgen05.commit
-//   warp 2       loads 2-D TMA tiles of the token rows (xs or h) into the
-//                B ring (128-byte swizzle); warp 3 has no role
+//   warp 2       loads the token rows into the B ring (128-byte swizzle):
+//                gate/up gathers them from x by TMA row gathers (four rows
+//                per copy), down loads 2-D TMA tiles of h; warp 3 has no role
 //   warps 4-11   expand int4 -> bf16 from the W ring into the A ring, in two
 //                groups that take alternate K chunks
 //   warps 12-15  epilogue: TMEM -> registers -> bf16 rows of h or o
@@ -296,13 +298,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             mbar_wait_drain(drain_bar, 0);
         }
     } else if (warp == kWarpLoader) {
-        // one 2-D TMA tile of kBlockT token rows per stage (rows past the block
-        // belong to the next expert or lie past the end and are zero-filled;
-        // the MMA ignores columns >= N and the epilogue columns >= rows)
+        // Down: one 2-D TMA tile of kBlockT rows of h per stage (rows past the
+        // block belong to the next expert or lie past the end and are
+        // zero-filled; the MMA ignores columns >= N and the epilogue columns
+        // >= rows).  Gate/up: the block's token rows gathered from x, four per
+        // copy, only the N rows the MMA reads (rows >= the block's rows repeat
+        // its last token); lane l issues row groups l and l + 32.
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-            const int row0 = a.block_map[3 * (u / NT) + 1];
+            const int b = u / NT;
+            const int row0 = a.block_map[3 * b + 1];
+            const int rows = max(a.block_map[3 * b + 2], 1);
+            int tok[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+            int ngroups = 0;
+            uint32_t bytes = kBStageBytes;
+            if constexpr (!kDown) {
+                const int N = (rows + 15) & ~15;
+                ngroups = N >> 2;
+                bytes = static_cast<uint32_t>(N) * (kKChunk * 2);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int p = min(4 * (lane + 32 * h) + r, rows - 1);
+                        int t = a.sorted_assign[row0 + p] / a.k;
+                        if (static_cast<unsigned>(t) >= static_cast<unsigned>(a.T)) {
+                            report_error(a.status, MOE_ERR_DEVICE_BOUNDS, 110);
+                            t = 0;
+                        }
+                        tok[h][r] = t;
+                    }
+            }
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNB;
                 if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
@@ -310,9 +337,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     ok = false;
                     break;
                 }
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(bfull(s), kBStageBytes);
-                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
+                const uint32_t dst = sbase + C::kOffB + s * kBStageBytes;
+                if constexpr (kDown) {
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(bfull(s), bytes);
+                        tma_load_2d(dst, &a.bmap, c * kKChunk, row0, bfull(s));
+                    }
+                } else {
+                    if (elect_one()) mbar_arrive_expect_tx(bfull(s), bytes);
+                    __syncwarp();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int g = lane + 32 * h;
+                        if (g < ngroups)
+                            tma_gather4(dst + g * 4 * (kKChunk * 2), &a.bmap, c * kKChunk, tok[h][0],
+                                        tok[h][1], tok[h][2], tok[h][3], bfull(s));
+                    }
                 }
                 __syncwarp();
             }
@@ -587,6 +627,22 @@ cudaError_t encode_f32_cols_map(CUtensorMap* map, const float* base, uint64_t ro
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t encode_f32_3d_map(CUtensorMap* map, const float* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                              uint32_t b0, uint32_t b1, uint32_t b2) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    const cudaError_t e = tensor_map_encoder(&encode);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 4, d0 * d1 * 4};
+    const cuuint32_t box[3] = {b0, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims,
                               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

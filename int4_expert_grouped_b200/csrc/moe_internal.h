@@ -21,8 +21,8 @@ struct moe_plan {
     size_t dn_packed;
     size_t packed_bytes;
     // workspace offsets
-    size_t o_status, o_logits, o_hist, o_gbase, o_idx, o_w, o_counts, o_offsets, o_bo, o_nb,
-        o_sa, o_pos, o_bm, o_xs, o_h, ws_bytes;
+    size_t o_status, o_dsync, o_dscr, o_logits, o_hist, o_gbase, o_idx, o_w, o_counts, o_offsets, o_bo, o_nb,
+        o_sa, o_pos, o_bm, o_o, o_h, ws_bytes;
     size_t o_xstage, o_ystage, host_ws_bytes;
 };
 
@@ -53,6 +53,7 @@ constexpr int kBlockT = 256;      // block map tile height = largest MMA N
 constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
 constexpr int kDecodeMaxT = 8;    // largest batch the small-batch (decode) path takes
 constexpr int kDownTiles = 1;     // 128-row down-projection tiles per packed block and GEMM unit
+constexpr int kDecodeSyncBytes = 8192;  // flags of the small-batch kernel (workspace bytes 256 ..)
 
 // Packed weight block: `tiles` 128-row A tiles of one 64-wide K chunk
 // (gate/up: the gate rows, then the up rows of 128 features; down: 128 rows):
@@ -95,10 +96,15 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
                            cudaStream_t st);
 
 struct GemmArgs {
-    // B operand (token rows in expert order) for 2-D TMA tiles of 64 columns x
-    // kBlockT rows with the 128-byte swizzle, the K-major layout the MMA
-    // reads: gate/up reads xs [T*k, d], down reads h [T*k, f].
+    // B operand: token rows in expert order, 64 columns per K chunk, in the
+    // K-major 128-byte-swizzled layout the MMA reads.  Gate/up gathers the
+    // rows from x [T, d] four at a time (map box: 64 columns x 1 row), the
+    // token of expert-ordered row p being sorted_assign[p] / k; down loads
+    // 2-D tiles of kBlockT rows of h [T*k, f] (box: 64 columns x kBlockT rows).
     CUtensorMap bmap;
+    const int32_t* sorted_assign;  // [T*k] (gate/up only)
+    int k;                         // experts per token (gate/up only)
+    int T;                         // tokens, rows of x (gate/up only)
     const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
     const int32_t* block_map;      // [num_blocks, 3]
     const int32_t* num_blocks;     // [1], device
@@ -115,18 +121,24 @@ struct GemmArgs {
 // of box_cols columns x box_rows rows, unswizzled.
 cudaError_t encode_f32_cols_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
                                 uint32_t box_cols, uint32_t box_rows);
+// Encode the tensor map of a 3-D fp32 tensor with dims d0 (innermost,
+// contiguous) x d1 x d2, read in unswizzled boxes b0 x b1 x b2.
+cudaError_t encode_f32_3d_map(CUtensorMap* map, const float* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                              uint32_t b0, uint32_t b1, uint32_t b2);
 // Encode the tensor map of a row-major bf16 matrix [rows, cols] read in boxes
 // of 64 columns x box_rows rows with the 128-byte swizzle.
 cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                                  uint32_t box_rows);
+// The same map with a box of one row, for four-row gathers.
+inline cudaError_t encode_bf16_gather_map(CUtensorMap* map, const void* base, uint64_t rows,
+                                          uint64_t cols) {
+    return encode_bf16_rows_map(map, base, rows, cols, 1);
+}
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t prepare_gemm_kernels();
 
-// ---- dispatch and combine (moe_combine.cu) ----
-// xs[p] = x[sorted_assign[p] / k] for p < T*k
-cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
-                            uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st);
+// ---- combine (moe_combine.cu) ----
 // y[t] = bf16(sum_i topk_w[t*k+i] * o[pos[t*k+i]])
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T,
                            int k, int d, uint16_t* y, int32_t* status, int num_sms,
@@ -143,20 +155,21 @@ struct DecodeArgs {
     const uint8_t* wpack_dn;     // packed down blocks
     int gu_block_bytes;
     int dn_block_bytes;
-    int max_blocks;
     int32_t *topk_idx, *counts, *offsets, *sorted_assign, *pos, *block_offsets, *block_map,
         *num_blocks;
     float* topk_w;
     uint16_t* h;                 // workspace [T*k, f]
     uint16_t* y;                 // [T, d]
     int32_t* status;
+    int32_t* sync;               // workspace flags (kDecodeSyncBytes, zero or left by this kernel)
+    uint8_t* scratch;            // workspace, decode_workspace_bytes
 };
-// Whether the small-batch kernels take this shape at batch T (otherwise the
+// Whether the small-batch kernel takes this shape at batch T (otherwise the
 // batched path runs).
 bool decode_supported(const moe_shape_t& s, int T);
+// Workspace bytes of the small-batch kernel's partial sums for batches up to T_max.
+size_t decode_workspace_bytes(const moe_shape_t& s, int T_max);
 cudaError_t prepare_decode_kernels();
-// Records ev_routed after the routing kernel and ev_gate_up after the gate/up
-// kernel when they are not null.
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* ev_routed, void* ev_gate_up);
+cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t st);
 
 }  // namespace moe

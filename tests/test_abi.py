@@ -130,17 +130,23 @@ def test_prepack_and_host_checks(moe):
 
 
 def test_forward_path_choice(moe):
-    # host-only query: small batches of a supported shape take the decode kernels
+    # host-only query: small batches of a supported shape take the decode kernel
     p = moe.Plan(8192, 2048, 128, 8, 768, 64)
     assert [p.forward_path(T) for T in (0, 1, 4, 8, 9, 8192)] == [0, 1, 1, 1, 0, 0]
     assert p.forward_path(-1) == -1 and p.forward_path(8193) == -1
     tiny = moe.Plan(64, 256, 8, 2, 128, 32)
-    assert tiny.forward_path(3) == 0  # E = 8: too few experts for the 8-CTA routing cluster
+    assert tiny.forward_path(3) == 1 and tiny.forward_path(9) == 0
     g32 = moe.Plan(64, 256, 32, 2, 128, 32)
     assert g32.forward_path(3) == 1 and g32.forward_path(9) == 0
-    # d = 4096: a gate/up warp's K chunks no longer fit its registers
-    assert moe.Plan(64, 4096, 128, 8, 768, 64).forward_path(1) == 0
-    # f = 1024 at T = 8: 64 h rows and their sums still fit the down kernel's shared memory
+    # d = 4096: the x rows of 8 tokens no longer fit beside the weight ring
+    wide = moe.Plan(64, 4096, 128, 8, 768, 64)
+    assert wide.forward_path(4) == 1 and wide.forward_path(8) == 0
+    # f = 1024 at T = 8: 8 h rows and their sums still fit
     assert moe.Plan(64, 2048, 128, 8, 1024, 64).forward_path(8) == 1
-    # E = 256 at d = 2048: a routing CTA's 32 W_r columns (256 KB) exceed its shared memory
-    assert moe.Plan(64, 2048, 256, 8, 768, 64).forward_path(1) == 0
+    # f = 4096: more than 16 feature tiles per expert
+    assert moe.Plan(64, 2048, 128, 8, 4096, 64).forward_path(1) == 0
+    # E = 256: two routing items per CTA on 148 SMs, still one kernel
+    assert moe.Plan(64, 2048, 256, 8, 768, 64).forward_path(1) == 1
+    # at most 64 assignments per call: k = 16 takes batches of up to 4 tokens
+    k16 = moe.Plan(64, 2048, 128, 16, 768, 64)
+    assert k16.forward_path(4) == 1 and k16.forward_path(5) == 0
