@@ -35,7 +35,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer prefill tokens/s (int4 fused grouped GEMM) and % of roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
-KERNELS_PER_STEP = 7  # logits, top-k, scan, scatter, gate/up GEMM (row gather), down GEMM, combine
+KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, down GEMM, combine
 KERNELS_PER_STEP_DECODE = 1  # one persistent kernel (batches of at most 8 tokens)
 
 

@@ -1,13 +1,17 @@
-// Combine after the grouped GEMMs (inblix article "Perplexity's Lily engine
-// beats MLX by 35% on M5 Max, no PyTorch needed", paragraph 3: the
-// routing-weighted sum of the expert outputs):
+// Dispatch and combine around the grouped GEMMs (inblix article "Perplexity's
+// Lily engine beats MLX by 35% on M5 Max, no PyTorch needed", paragraph 3:
+// scatter of the routed tokens into expert-contiguous order, and the
+// routing-weighted sum of the expert outputs).
 //
+//   dispatch_kernel   xs[p] = x[sorted_assign[p] / k]        p < T*k
 //   combine_kernel    y[t]  = bf16( sum_{j<k} w[t,j] * o[pos[t,j]] )
 //
-// Bound by HBM bandwidth; it moves 16-byte vectors, consecutive threads on
-// consecutive vectors of a row.  The down GEMM writes one output row per
-// assignment, so the sum over a token's experts runs in a fixed order with
-// no atomics.
+// Both are bound by HBM bandwidth and move 16-byte vectors, consecutive
+// threads on consecutive vectors of a row.  Copying the token rows into
+// expert order once lets both grouped GEMMs read their token operand as dense
+// 2-D TMA tiles (a gather of single rows runs at a small fraction of that
+// rate), and writing the down outputs per assignment lets the sum over a
+// token's experts run in a fixed order with no atomics.
 #include "moe_internal.h"
 
 namespace moe {
@@ -21,6 +25,49 @@ __device__ __forceinline__ uint4 ld_nc_v4(const uint4* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+// One warp per row (grid-stride): lane l moves 16-byte vectors l, l + 32, ...
+// of the row, up to kDispatchVecs of them loaded before the first store (all
+// of a row for d <= 2048), with the next row's source index read before the
+// stores.
+constexpr int kDispatchVecs = 8;
+
+__global__ void __launch_bounds__(kThreads)
+dispatch_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_assign, int Tk,
+                int k, int d, uint16_t* __restrict__ xs, int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int nv = d >> 3;  // 16-byte vectors per row
+    const int warps = gridDim.x * (kThreads / 32);
+    pdl_launch_dependents();
+    pdl_wait();
+    const uint4* x4 = reinterpret_cast<const uint4*>(x);
+    uint4* xs4 = reinterpret_cast<uint4*>(xs);
+    int p = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    int a = p < Tk ? sorted_assign[p] : 0;
+    for (; p < Tk; p += warps) {
+        const int a_next = p + warps < Tk ? sorted_assign[p + warps] : 0;
+        if (static_cast<unsigned>(a) >= static_cast<unsigned>(Tk)) {
+            if (lane == 0) report_error(status, MOE_ERR_DEVICE_BOUNDS, 300);
+            a = 0;
+        }
+        const uint4* src = x4 + static_cast<size_t>(a / k) * nv;
+        uint4* dst = xs4 + static_cast<size_t>(p) * nv;
+        for (int i0 = 0; i0 < nv; i0 += 32 * kDispatchVecs) {
+            uint4 v[kDispatchVecs];
+#pragma unroll
+            for (int u = 0; u < kDispatchVecs; ++u) {
+                const int i = i0 + 32 * u + lane;
+                v[u] = i < nv ? ld_nc_v4(src + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kDispatchVecs; ++u) {
+                const int i = i0 + 32 * u + lane;
+                if (i < nv) dst[i] = v[u];
+            }
+        }
+        a = a_next;
+    }
 }
 
 union BF8 {
@@ -93,6 +140,16 @@ combine_kernel(const uint16_t* __restrict__ o, const int32_t* __restrict__ pos,
 }
 
 }  // namespace
+
+cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
+                            uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st) {
+    if (Tk <= 0) return cudaSuccess;
+    const long need = (static_cast<long>(Tk) + kThreads / 32 - 1) / (kThreads / 32);
+    const long cap = static_cast<long>(num_sms) * 8;  // 8 CTAs of 8 warps per SM
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    return launch_pdl(dispatch_kernel, dim3(grid), dim3(kThreads), 0, st, x, sorted_assign, Tk, k, d, xs,
+                      status);
+}
 
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T, int k,
                            int d, uint16_t* y, int32_t* status, int num_sms, cudaStream_t st) {

@@ -120,20 +120,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
         : "memory");
 }
 
-// Four rows (r0..r3) of a 2-D tensor, columns c0 .. c0 + box - 1, into shared
-// memory as four consecutive rows of the map's box (TMA row gather; the
-// map's box is one row high).  With the 128-byte swizzle the rows land in the
-// swizzled positions of the shared-memory address they are written to.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int c0, int r0, int r1,
-                                            int r2, int r3, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(r0), "r"(r1),
-          "r"(r2), "r"(r3)
-        : "memory");
-}
-
 // 16-byte copy global -> shared; src_bytes = 0 writes zeros and reads nothing.
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),

@@ -6,8 +6,7 @@
 //   prepack_kernel        logical nibbles/scales -> per (expert, tile, K chunk)
 //                         contiguous blocks in the order the GEMM reads them
 //   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
-//       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order
-//                (xs[p] = x[sorted_assign[p] / k], gathered on load),
+//       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order,
 //                epilogue h = silu(D0) * D1 -> bf16 h rows
 //       down:    D = kDownTiles 128-row tiles of Wd times h^T, epilogue
 //                o = bf16(D) rows
@@ -31,9 +30,8 @@
 //   warp 0       bulk-copies packed weight blocks into the W ring (TMA engine)
 //   warp 1       allocates TMEM; runs the MMA loop, one elected lane issues
 //                tcgen05.mma and tcgen05.commit
-//   warp 2       loads the token rows into the B ring (128-byte swizzle):
-//                gate/up gathers them from x by TMA row gathers (four rows
-//                per copy), down loads 2-D TMA tiles of h; warp 3 has no role
+//   warp 2       loads 2-D TMA tiles of the token rows (xs or h) into the
+//                B ring (128-byte swizzle); warp 3 has no role
 //   warps 4-11   expand int4 -> bf16 from the W ring into the A ring, in two
 //                groups that take alternate K chunks
 //   warps 12-15  epilogue: TMEM -> registers -> bf16 rows of h or o
@@ -298,38 +296,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             mbar_wait_drain(drain_bar, 0);
         }
     } else if (warp == kWarpLoader) {
-        // Down: one 2-D TMA tile of kBlockT rows of h per stage (rows past the
-        // block belong to the next expert or lie past the end and are
-        // zero-filled; the MMA ignores columns >= N and the epilogue columns
-        // >= rows).  Gate/up: the block's token rows gathered from x, four per
-        // copy, only the N rows the MMA reads (rows >= the block's rows repeat
-        // its last token); lane l issues row groups l and l + 32.
+        // one 2-D TMA tile of kBlockT token rows per stage (rows past the block
+        // belong to the next expert or lie past the end and are zero-filled;
+        // the MMA ignores columns >= N and the epilogue columns >= rows)
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-            const int b = u / NT;
-            const int row0 = a.block_map[3 * b + 1];
-            const int rows = max(a.block_map[3 * b + 2], 1);
-            int tok[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-            int ngroups = 0;
-            uint32_t bytes = kBStageBytes;
-            if constexpr (!kDown) {
-                const int N = (rows + 15) & ~15;
-                ngroups = N >> 2;
-                bytes = static_cast<uint32_t>(N) * (kKChunk * 2);
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int p = min(4 * (lane + 32 * h) + r, rows - 1);
-                        int t = a.sorted_assign[row0 + p] / a.k;
-                        if (static_cast<unsigned>(t) >= static_cast<unsigned>(a.T)) {
-                            report_error(a.status, MOE_ERR_DEVICE_BOUNDS, 110);
-                            t = 0;
-                        }
-                        tok[h][r] = t;
-                    }
-            }
+            const int row0 = a.block_map[3 * (u / NT) + 1];
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNB;
                 if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
@@ -337,22 +310,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     ok = false;
                     break;
                 }
-                const uint32_t dst = sbase + C::kOffB + s * kBStageBytes;
-                if constexpr (kDown) {
-                    if (elect_one()) {
-                        mbar_arrive_expect_tx(bfull(s), bytes);
-                        tma_load_2d(dst, &a.bmap, c * kKChunk, row0, bfull(s));
-                    }
-                } else {
-                    if (elect_one()) mbar_arrive_expect_tx(bfull(s), bytes);
-                    __syncwarp();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int g = lane + 32 * h;
-                        if (g < ngroups)
-                            tma_gather4(dst + g * 4 * (kKChunk * 2), &a.bmap, c * kKChunk, tok[h][0],
-                                        tok[h][1], tok[h][2], tok[h][3], bfull(s));
-                    }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(bfull(s), kBStageBytes);
+                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
                 }
                 __syncwarp();
             }

@@ -22,7 +22,7 @@ struct moe_plan {
     size_t packed_bytes;
     // workspace offsets
     size_t o_status, o_dsync, o_dscr, o_logits, o_hist, o_gbase, o_idx, o_w, o_counts, o_offsets, o_bo, o_nb,
-        o_sa, o_pos, o_bm, o_o, o_h, ws_bytes;
+        o_sa, o_pos, o_bm, o_xs, o_h, ws_bytes;
     size_t o_xstage, o_ystage, host_ws_bytes;
 };
 
@@ -96,15 +96,10 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
                            cudaStream_t st);
 
 struct GemmArgs {
-    // B operand: token rows in expert order, 64 columns per K chunk, in the
-    // K-major 128-byte-swizzled layout the MMA reads.  Gate/up gathers the
-    // rows from x [T, d] four at a time (map box: 64 columns x 1 row), the
-    // token of expert-ordered row p being sorted_assign[p] / k; down loads
-    // 2-D tiles of kBlockT rows of h [T*k, f] (box: 64 columns x kBlockT rows).
+    // B operand (token rows in expert order) for 2-D TMA tiles of 64 columns x
+    // kBlockT rows with the 128-byte swizzle, the K-major layout the MMA
+    // reads: gate/up reads xs [T*k, d], down reads h [T*k, f].
     CUtensorMap bmap;
-    const int32_t* sorted_assign;  // [T*k] (gate/up only)
-    int k;                         // experts per token (gate/up only)
-    int T;                         // tokens, rows of x (gate/up only)
     const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
     const int32_t* block_map;      // [num_blocks, 3]
     const int32_t* num_blocks;     // [1], device
@@ -129,16 +124,15 @@ cudaError_t encode_f32_3d_map(CUtensorMap* map, const float* base, uint64_t d0, 
 // of 64 columns x box_rows rows with the 128-byte swizzle.
 cudaError_t encode_bf16_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                                  uint32_t box_rows);
-// The same map with a box of one row, for four-row gathers.
-inline cudaError_t encode_bf16_gather_map(CUtensorMap* map, const void* base, uint64_t rows,
-                                          uint64_t cols) {
-    return encode_bf16_rows_map(map, base, rows, cols, 1);
-}
+
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down(const GemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t prepare_gemm_kernels();
 
-// ---- combine (moe_combine.cu) ----
+// ---- dispatch and combine (moe_combine.cu) ----
+// xs[p] = x[sorted_assign[p] / k] for p < T*k
+cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
+                            uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st);
 // y[t] = bf16(sum_i topk_w[t*k+i] * o[pos[t*k+i]])
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T,
                            int k, int d, uint16_t* y, int32_t* status, int num_sms,
