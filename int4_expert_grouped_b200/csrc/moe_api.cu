@@ -47,6 +47,7 @@ moe_status_t device_setup(int* num_sms) {
     if (c.prepared.load() == 0) {
         if (moe::prepare_gemm_kernels() != cudaSuccess) return MOE_ERR_CUDA;
         if (moe::prepare_decode_kernels() != cudaSuccess) return MOE_ERR_CUDA;
+        if (moe::prepare_router_fast() != cudaSuccess) return MOE_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -105,10 +106,19 @@ moe_status_t run_route(const moe_plan* p, int T, const uint16_t* x, const float*
     int32_t* status = at<int32_t>(ws, p->o_status);
     int32_t* hist = at<int32_t>(ws, p->o_hist);
     const int ng = (T + kRouteGroupT - 1) / kRouteGroupT;
-    MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, at<float>(ws, p->o_logits), T, s.d, s.E, hist,
-                                       std::max(ng, 1) * s.E, status, st));
-    MOE_CUDA(moe::launch_router_topk(at<float>(ws, p->o_logits), T, s.E, s.k, r.idx, r.w, hist,
-                                     st));
+    if (moe::router_fast_supported(T, s.d, s.E)) {
+        // int8 tensor-core logits with a proven error bound; the fixed-order
+        // fp32 logits only for the pairs the bound cannot settle
+        const moe::RouterFastWs fw = moe::router_fast_ws(at<uint8_t>(ws, p->o_rfast),
+                                                         at<float>(ws, p->o_logits), T, s.d, s.E);
+        MOE_CUDA(moe::launch_router_fast(x, W_r, b_r, T, s.d, s.E, s.k, fw, r.idx, r.w, hist,
+                                         std::max(ng, 1) * s.E, status, st));
+    } else {
+        MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, at<float>(ws, p->o_logits), T, s.d, s.E, hist,
+                                           std::max(ng, 1) * s.E, status, st));
+        MOE_CUDA(moe::launch_router_topk(at<float>(ws, p->o_logits), T, s.E, s.k, r.idx, r.w, hist,
+                                         st));
+    }
     MOE_CUDA(moe::launch_route_scan(hist, ng, s.E, p->block_t, r.counts, r.offsets,
                                     at<int32_t>(ws, p->o_gbase), r.bo, r.bm, r.nb, p->max_blocks,
                                     status, st));
@@ -185,6 +195,9 @@ moe_status_t moe_plan_create(const moe_shape_t* shape, moe_plan_t** plan, moe_pl
     p->o_bm = take(static_cast<size_t>(p->max_blocks) * 12);
     p->o_xs = take(T * k * s.d * 2);  // x rows in expert order, later the down outputs o
     p->o_h = take(T * k * s.f * 2);
+    p->o_rfast = take(moe::router_fast_supported(s.T_max, s.d, s.E)
+                          ? moe::router_fast_ws_bytes(s.T_max, s.d, s.E)
+                          : 0);
     p->ws_bytes = o;
     p->o_xstage = take(T * s.d * 2);
     p->o_ystage = take(T * s.d * 2);

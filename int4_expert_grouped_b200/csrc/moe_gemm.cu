@@ -593,6 +593,21 @@ cudaError_t encode_f32_cols_map(CUtensorMap* map, const float* base, uint64_t ro
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_u8_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                               uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    const cudaError_t e = tensor_map_encoder(&encode);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {128, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t encode_f32_3d_map(CUtensorMap* map, const float* base, uint64_t d0, uint64_t d1, uint64_t d2,
                               uint32_t b0, uint32_t b1, uint32_t b2) {
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;

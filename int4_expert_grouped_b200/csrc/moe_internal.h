@@ -22,7 +22,7 @@ struct moe_plan {
     size_t packed_bytes;
     // workspace offsets
     size_t o_status, o_dsync, o_dscr, o_logits, o_hist, o_gbase, o_idx, o_w, o_counts, o_offsets, o_bo, o_nb,
-        o_sa, o_pos, o_bm, o_xs, o_h, ws_bytes;
+        o_sa, o_pos, o_bm, o_xs, o_h, o_rfast, ws_bytes;
     size_t o_xstage, o_ystage, host_ws_bytes;
 };
 
@@ -77,6 +77,28 @@ cudaError_t launch_route_scatter(const int32_t* topk_idx, const int32_t* gbase, 
                                  int E, int32_t* sorted_assign, int32_t* pos, int32_t* status,
                                  cudaStream_t st);
 
+// ---- router with exact near-tie recheck (moe_router_fast.cu) ----
+constexpr int kFastRouterMinT = 1024;  // smallest batch the int8 tensor-core router takes
+struct RouterFastWs {
+    int8_t *xa, *xb;            // token digits [T][d]
+    int8_t *wc, *wd;            // expert digits [E][d]
+    float *s_t, *E_t, *A_t, *N_t, *theta;  // per token: scale, remainder max, sum |x'|, ||x||, threshold
+    float *u_e, *F_e, *B_e, *Wn_e;         // per expert: scale, remainder max, sum |w|, ||w||
+    float* L;                   // [T][E] approximate logits with the bias
+    float* exact;               // [T][E] fixed-order logits of the candidate pairs
+};
+bool router_fast_supported(int T, int d, int E);
+size_t router_fast_ws_bytes(int T, int d, int E);
+// Carve the router's scratch out of `base` (router_fast_ws_bytes); L is the
+// [T][E] logits buffer.
+RouterFastWs router_fast_ws(uint8_t* base, float* L, int T, int d, int E);
+cudaError_t prepare_router_fast();
+// Top-k indices and weights and the per-group histograms (cleared here, as is
+// the status word) for T >= kFastRouterMinT tokens.
+cudaError_t launch_router_fast(const uint16_t* x, const float* W, const float* b, int T, int d, int E,
+                               int k, const RouterFastWs& ws, int32_t* topk_idx, float* topk_w,
+                               int32_t* hist, int hist_n, int32_t* status, cudaStream_t st);
+
 // ---- weights and GEMM (moe_gemm.cu) ----
 struct PrepackSource {
     const uint8_t* q0;   // A0 rows come from this projection
@@ -116,6 +138,10 @@ struct GemmArgs {
 // of box_cols columns x box_rows rows, unswizzled.
 cudaError_t encode_f32_cols_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
                                 uint32_t box_cols, uint32_t box_rows);
+// Encode the tensor map of a row-major int8 matrix [rows, cols] read in boxes
+// of 128 columns (bytes) x box_rows rows with the 128-byte swizzle.
+cudaError_t encode_u8_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                               uint32_t box_rows);
 // Encode the tensor map of a 3-D fp32 tensor with dims d0 (innermost,
 // contiguous) x d1 x d2, read in unswizzled boxes b0 x b1 x b2.
 cudaError_t encode_f32_3d_map(CUtensorMap* map, const float* base, uint64_t d0, uint64_t d1, uint64_t d2,

@@ -342,3 +342,62 @@ def test_chained_calls_read_previous_output(moe):
             check_route(bufs, oracle_route(sub), T, s.k)
         check_y(yout[:T], oracle.forward(sub)["y"], "chained T=%d" % T)
 
+
+
+# ---------------------------------------------------------------------------
+# The int8 tensor-core router (batches of 1024 tokens and more): exact ties,
+# near ties and all-tied rows, where the fixed-order recheck decides.  Routing
+# only (moe_route), compared bit for bit with the oracle.
+# ---------------------------------------------------------------------------
+def route_only(moe, T, d, E, k, x_bits, w_r, b_r):
+    plan = moe.Plan(T, d, E, k, 128, 64)
+    ws = torch.empty(plan.info.workspace_bytes, dtype=torch.uint8, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    out = {"topk_idx": torch.empty((T, k), **i32),
+           "topk_w": torch.empty((T, k), dtype=torch.float32, device="cuda"),
+           "counts": torch.empty(E, **i32), "offsets": torch.empty(E + 1, **i32),
+           "sorted_assign": torch.empty(T * k, **i32), "pos": torch.empty(T * k, **i32),
+           "block_offsets": torch.empty(E + 1, **i32),
+           "block_map": torch.empty((plan.info.max_blocks, 3), **i32),
+           "num_blocks": torch.empty(4, **i32)}
+    x = moe.bf16_tensor(x_bits, "cuda")
+    wr = torch.from_numpy(np.ascontiguousarray(w_r, np.float32)).cuda()
+    br = None if b_r is None else torch.from_numpy(np.ascontiguousarray(b_r, np.float32)).cuda()
+    plan.route(T, x, wr, br, out, ws)
+    torch.cuda.synchronize()
+    assert plan.read_status(ws) == (0, 0)
+    return out
+
+
+def fast_case(moe, T, d, E, k, seed, kind):
+    inp = mi.make_inputs(mi.Shape(T, d, E, k, 128, 64), seed, weights=False)
+    assert T >= 1024  # the int8 tensor-core router takes batches of 1024 tokens and more
+    w = inp.w_r.copy()
+    b = None
+    if kind == "duplicate_columns":      # experts 2j and 2j+1 tie exactly for every token
+        w[:, 1::2] = w[:, 0::2]
+    elif kind == "one_ulp_apart":        # experts 2j and 2j+1 differ in one entry's last bit
+        w[:, 1::2] = w[:, 0::2]
+        w[5, 1::2] = np.nextafter(w[5, 0::2], np.float32(np.inf))
+    elif kind == "all_tied":             # every logit 0: every expert is a candidate
+        w[:] = 0.0
+    elif kind == "bias_only":            # every token on experts 0..k-1
+        w[:] = 0.0
+        b = -np.arange(E, dtype=np.float32)
+    out = route_only(moe, T, d, E, k, inp.x, w, b)
+    sub = mi.Inputs(inp.shape, seed, inp.x, w, b, None, None, None)
+    check_route(out, oracle_route(sub), T, k)
+    return out
+
+
+@pytest.mark.parametrize("kind", ["duplicate_columns", "one_ulp_apart", "all_tied", "bias_only"])
+def test_fast_router_ties(moe, kind):
+    out = fast_case(moe, 1500, 256, 16, 4, 90, kind)
+    idx = out["topk_idx"].cpu().numpy()
+    if kind in ("all_tied", "bias_only"):
+        assert (idx == np.arange(4)).all()
+
+
+def test_fast_router_near_ties_wide(moe):
+    # the 2048-wide, 128-expert router with pairs of experts one ulp apart
+    fast_case(moe, 1024, 2048, 128, 8, 91, "one_ulp_apart")
