@@ -20,19 +20,22 @@
 //                       butterfly levels and the bias give the logits; top-k,
 //                       weights, counts, offsets, block map and scatter are
 //                       computed in every CTA identically (CTA 0 writes them)
-//   3. experts          the units (gate/up: expert, 128-feature tile, two
-//                       64-wide K chunks; down: expert, 128-output tile, half
-//                       of K) are dealt round robin to the CTAs, gate/up units
-//                       first.  A producer warp streams each unit's packed
-//                       blocks into a shared-memory ring with bulk copies, as
-//                       far ahead as the ring allows, so every SM keeps its
-//                       share of the weights in flight; eight warps multiply
-//                       them on the warp-level tensor-core MMA.  Partial sums
-//                       go to the workspace; the last unit of a tile (an
-//                       atomic count) adds them in a fixed order: SwiGLU into
-//                       h for gate/up, and for down the weighted sum of each
-//                       token's expert outputs in slot order into y
-//   4. exit             the last CTA to leave resets the flags for the next
+//   3. experts          the units (one expert's 64-feature slice: its 64 gate
+//                       and 64 up rows over all of K, then the 64 matching
+//                       columns of W_down for every output tile) are dealt
+//                       round robin to the CTAs.  A producer warp streams
+//                       each unit's weights into a shared-memory ring with
+//                       bulk copies, as far ahead as the ring allows, so every
+//                       SM keeps its share of the weights in flight; eight
+//                       warps multiply them on the warp-level tensor-core MMA.
+//                       SwiGLU of the slice stays in shared memory (no h round
+//                       trip); the slice's down partial sums go to the
+//                       workspace
+//   4. combine          after a grid-wide count of finished CTAs, every CTA
+//                       adds, for its share of the outputs, each expert's
+//                       slice partials in slice order, rounds the expert output
+//                       to bf16 and sums a token's slots in slot order into y;
+//                       the last CTA to leave resets the flags for the next
 //                       call
 //
 // MMA form (m16n8k16, bf16 operands from registers, fp32 accumulators): a
@@ -59,12 +62,16 @@ constexpr int kDecComputeWarps = 8;
 constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;  // + one producer warp
 constexpr int kDecProducerWarp = kDecComputeWarps;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
-constexpr int kDecStages = 16;
-constexpr int kDecStageBytes = packed_block_bytes(2, 32);  // a gate/up block (group 32: largest)
+constexpr int kDecStages = 32;
+// One stage = one 64-wide K chunk of a slice's 64 gate and 64 up rows
+// (nibbles, then scale/bias words), or one down block (128 rows x 64 K):
+// both 4096 + 512 * (64 / group) bytes.
+constexpr int kDecStageBytes = 4096 + 512 * 2;
 constexpr int kDecMaxAssign = 64;                          // T * k the path takes
-constexpr int kDecGuChunks = 2;                            // 64-wide K chunks per gate/up unit
-constexpr int kDecMaxNT = 16;                              // f / 128
+constexpr int kDecSlice = 64;                              // features per unit
+constexpr int kDecMaxSlices = 32;                          // f / 64
 constexpr int kDecMaxNTd = 64;                             // d / 128
+constexpr int kDecHStride = kDecSlice + 32;                // h row stride (elements) in shared memory
 constexpr int kDecWRows = 256;                             // W_r rows per tensor load (box limit)
 constexpr uint32_t kDecMagic0 = 0x4D6F4544u, kDecMagic1 = 0x53796E63u;
 
@@ -73,10 +80,8 @@ constexpr int kSyncMagic = 0;     // two words: the region has been initialised
 constexpr int kSyncRoute = 2;     // routing items published
 constexpr int kSyncExit = 3;      // CTAs that have finished
 constexpr int kSyncAbort = 4;     // a CTA gave up waiting
-constexpr int kSyncHReady = 16;   // [kDecMaxAssign] gate/up tiles done per block
-constexpr int kSyncDn = kSyncHReady + kDecMaxAssign;  // [kDecMaxNTd] down units done per tile
-constexpr int kSyncGu = kSyncDn + kDecMaxNTd;         // [kDecMaxAssign * kDecMaxNT] per (block, tile)
-constexpr int kSyncInts = kSyncGu + kDecMaxAssign * kDecMaxNT;
+constexpr int kSyncUnits = 5;     // CTAs done with their units
+constexpr int kSyncInts = 8;
 static_assert(kSyncInts * 4 <= kDecodeSyncBytes, "decode flags fit their workspace region");
 
 __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
@@ -197,6 +202,31 @@ __device__ __forceinline__ void chunk_mma(float (&acc)[4], const uint8_t* blk, i
         vector_mma(D, wa1, wb1, xb1);
         group_fold(acc, D, lds_u32(blk + nib_bytes + ra * 4), lds_u32(blk + nib_bytes + rb * 4),
                    xs0[0] + xs0[1], xs1[0] + xs1[1]);
+    }
+}
+
+// The same for rows held apart (the gate and the up rows of a slice): na, nb
+// = the two rows' 32 bytes of nibbles, sa, sb = their (scale, bias) words.
+template <int kGpc>
+__device__ __forceinline__ void chunk_mma_rows(float (&acc)[4], const uint8_t* na, const uint8_t* nb,
+                                               const uint8_t* sa, const uint8_t* sb, int c,
+                                               const uint16_t* xrow, const float* xs0, const float* xs1) {
+    const uint32_t wa0 = lds_u32(na + 4 * c);
+    const uint32_t wa1 = lds_u32(na + 16 + 4 * c);
+    const uint32_t wb0 = lds_u32(nb + 4 * c);
+    const uint32_t wb1 = lds_u32(nb + 16 + 4 * c);
+    const uint4 xb0 = *reinterpret_cast<const uint4*>(xrow);
+    const uint4 xb1 = *reinterpret_cast<const uint4*>(xrow + 32);
+    float D[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    vector_mma(D, wa0, wb0, xb0);
+    if constexpr (kGpc == 2) {
+        group_fold(acc, D, lds_u32(sa), lds_u32(sb), xs0[0], xs1[0]);
+        D[0] = D[1] = D[2] = D[3] = 0.0f;
+        vector_mma(D, wa1, wb1, xb1);
+        group_fold(acc, D, lds_u32(sa + 4), lds_u32(sb + 4), xs0[1], xs1[1]);
+    } else {
+        vector_mma(D, wa1, wb1, xb1);
+        group_fold(acc, D, lds_u32(sa), lds_u32(sb), xs0[0] + xs0[1], xs1[0] + xs1[1]);
     }
 }
 
@@ -327,8 +357,8 @@ __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     L.ring = take(kDecStages * kDecStageBytes);
     L.x = take(T * (d + 32) * 2);
     L.xsum = take(T * (d / 32) * 4);
-    L.h = take(kDecodeMaxT * (f + 32) * 2);
-    L.hsum = take(kDecodeMaxT * (f / 32) * 4);
+    L.h = take(kDecodeMaxT * kDecHStride * 2);
+    L.hsum = take(kDecodeMaxT * (kDecSlice / 32) * 4);
     L.lg = take(T * E * 4);
     L.route = take(static_cast<int>(sizeof(DecRoute)));
     L.bars = take((2 * kDecStages + 1) * 8);
@@ -347,9 +377,7 @@ struct DecParams {
         *num_blocks;
     float* topk_w;
     float* U;             // router partials [T][E][8]
-    float* pgu;           // gate/up partial sums [T*k][f/128][KS][256]
-    float* pdn;           // down partial sums [T*k][d/128][DS][128]
-    uint16_t* h;          // [T*k][f]
+    float* pdn;           // down partial sums [T*k][f/64][d]: one per (row, slice)
     uint16_t* y;          // [T][d]
     int32_t* status;
     int32_t* sync;        // the decode flags
@@ -559,45 +587,46 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     }
 
     // ---- phase 3: expert units ------------------------------------------------
-    const int NT = f / 128, KC = d / kKChunk, KS = KC / kDecGuChunks;
-    const int NTd = d / 128, KCd = f / kKChunk;
-    const int DS = (KCd % 4 == 0) ? 2 : 1;  // K halves of a down unit
-    const int dn_chunks = KCd / DS;         // chunks per down unit (even)
-    const int u_gu = nb * NT * KS;
-    const int u_total = u_gu + nb * NTd * DS;
+    // unit u = (block u / S, slice u % S); S = f / 64 slices per expert
+    const int NT = f / 128, KC = d / kKChunk, NTd = d / 128, KCd = f / kKChunk;
+    const int S = f / kDecSlice;
+    const int u_total = nb * S;
+    const int nib_gu = 256 * 32;                 // nibble bytes of a gate/up block
+    const int sc_bytes = kDecSlice * kGpc * 4;   // (scale, bias) words of 64 rows
 
     if (warp == kDecProducerWarp) {
         // the whole warp runs the loop; one elected lane issues the copies
         uint32_t q = 0;
         bool ok = true;
-        for (int i = cta; ok && i < u_total; i += G) {
-            const uint8_t* src;
-            int nst;
-            if (i < u_gu) {
-                const int b = i / (NT * KS);
-                const int j = (i / KS) % NT;
-                const int s = i % KS;
-                src = p.wgu + ((static_cast<size_t>(R.blk_e[b]) * NT + j) * KC + s * kDecGuChunks) * p.bb_gu;
-                nst = kDecGuChunks;
-            } else {
-                const int v = i - u_gu;
-                const int b = v / (NTd * DS);
-                const int jd = (v / DS) % NTd;
-                const int s2 = v % DS;
-                src = p.wdn + ((static_cast<size_t>(R.blk_e[b]) * NTd + jd) * KCd + s2 * dn_chunks) * p.bb_dn;
-                nst = dn_chunks / 2;
-            }
-            // one stage = one gate/up block = two consecutive down blocks (same bytes)
-            for (int st = 0; st < nst; ++st, ++q) {
+        for (int u = cta; ok && u < u_total; u += G) {
+            const int b = u / S;
+            const int fs = u - b * S;
+            const int e = R.blk_e[b];
+            const int j = fs >> 1, hh = fs & 1;  // 128-feature tile, half of it
+            for (int st = 0; st < KC + NTd; ++st, ++q) {
                 const int slot = q % kDecStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(empty(slot), ((q / kDecStages) & 1) ^ 1, &R.abort_local))) {
                     ok = false;
                     break;
                 }
                 if (elect_one()) {
-                    mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(p.bb_gu));
-                    bulk_copy_g2s(smem_u32(ring + slot * kDecStageBytes), src + static_cast<size_t>(st) * p.bb_gu,
-                                  static_cast<uint32_t>(p.bb_gu), full(slot));
+                    const uint32_t dst = smem_u32(ring + slot * kDecStageBytes);
+                    mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(p.bb_dn));
+                    if (st < KC) {
+                        // chunk st of the slice: gate rows 64 hh .., up rows 128 + 64 hh ..
+                        const uint8_t* blk = p.wgu + ((static_cast<size_t>(e) * NT + j) * KC + st) * p.bb_gu;
+                        bulk_copy_g2s(dst, blk + hh * kDecSlice * 32, kDecSlice * 32, full(slot));
+                        bulk_copy_g2s(dst + kDecSlice * 32, blk + (128 + hh * kDecSlice) * 32, kDecSlice * 32,
+                                      full(slot));
+                        bulk_copy_g2s(dst + 2 * kDecSlice * 32, blk + nib_gu + hh * sc_bytes, sc_bytes, full(slot));
+                        bulk_copy_g2s(dst + 2 * kDecSlice * 32 + sc_bytes,
+                                      blk + nib_gu + (128 / kDecSlice + hh) * sc_bytes, sc_bytes, full(slot));
+                    } else {
+                        // down block (expert, output tile st - KC, K chunk fs)
+                        const uint8_t* blk =
+                            p.wdn + ((static_cast<size_t>(e) * NTd + (st - KC)) * KCd + fs) * p.bb_dn;
+                        bulk_copy_g2s(dst, blk, static_cast<uint32_t>(p.bb_dn), full(slot));
+                    }
                 }
                 __syncwarp();
             }
@@ -617,64 +646,25 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
         const int g = lane >> 2;
         const int c = lane & 3;
         uint32_t q = 0;
-        int h_block = -1;  // block whose h rows are staged in hsh
-        const int nvd = d / 32, nvf = f / 32;
-        for (int i = cta; i < u_total; i += G) {
-            const bool gu = i < u_gu;
-            int b, j, s;
-            if (gu) {
-                b = i / (NT * KS);
-                j = (i / KS) % NT;
-                s = i % KS;
-            } else {
-                const int v = i - u_gu;
-                b = v / (NTd * DS);
-                j = (v / DS) % NTd;
-                s = v % DS;
-            }
+        const int nvd = d / 32;
+        for (int u = cta; u < u_total; u += G) {
+            const int b = u / S;
+            const int fs = u - b * S;
             const int row0 = R.blk_row0[b];
             const int n = R.blk_n[b];
-            if (!gu && h_block != b) {
-                // h rows of this block: wait until all its gate/up tiles are in
-                if (tid == 0) {
-                    R.hok = 1;
-                    if (!wait_flag(sync + kSyncHReady + b, NT, abort_g)) {
-                        dec_fail(p, R, 504);
-                        R.hok = 0;
-                    }
-                }
-                compute_sync();  // also: every warp is done with the previous h rows
-                if (!vload(R.hok)) break;
-                stage_rows(hsh, hsum, p.h + static_cast<size_t>(row0) * f, n, f, [](int r) { return r; }, tid,
-                           kDecComputeThreads);
-                compute_sync();
-                h_block = b;
-            }
-            // B columns: column g is row min(g, n-1) of the block; the
-            // accumulator's columns 2c, 2c + 1 need their vector sums
-            const int cg = min(g, n - 1), c0 = min(2 * c, n - 1), c1 = min(2 * c + 1, n - 1);
-            const uint16_t* brow;
-            const float *bs0, *bs1;
-            if (gu) {
-                brow = xsh + (R.sa[row0 + cg] / k) * (d + 32) + 8 * c;
-                bs0 = xsum + (R.sa[row0 + c0] / k) * nvd;
-                bs1 = xsum + (R.sa[row0 + c1] / k) * nvd;
-            } else {
-                brow = hsh + cg * (f + 32) + 8 * c;
-                bs0 = hsum + c0 * nvf;
-                bs1 = hsum + c1 * nvf;
-            }
-            // gate/up: warp w takes rows 32w .. 32w + 31 of the 256-row block
-            // (two 16-row tiles); down: rows 16w .. 16w + 15 of the 128-row tile
-            float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-            const int nst = gu ? kDecGuChunks : dn_chunks / 2;
             if (tid == 0) R.fail = 0;
-            compute_sync();
-            for (int st = 0; st < nst; ++st, ++q) {
+            compute_sync();  // also: every warp is done with the previous unit's h rows
+            // gate/up: warp w takes features 8w .. 8w + 7 of the slice; the MMA
+            // tile's rows g and g + 8 are the gate and the up row of feature 8w + g
+            const int cg = min(g, n - 1), c0 = min(2 * c, n - 1), c1 = min(2 * c + 1, n - 1);
+            const uint16_t* brow = xsh + (R.sa[row0 + cg] / k) * (d + 32) + 8 * c;
+            const float* bs0 = xsum + (R.sa[row0 + c0] / k) * nvd;
+            const float* bs1 = xsum + (R.sa[row0 + c1] / k) * nvd;
+            const int fr = 8 * warp + g;  // row of the slice
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int st = 0; st < KC; ++st, ++q) {
                 const int slot = q % kDecStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
-                    // give up on this unit; the others learn of it at the
-                    // barrier below, so every compute warp leaves together
                     if (lane == 0) {
                         R.fail = 1;
                         if (!vload(R.abort_local)) dec_fail(p, R, 505);
@@ -682,103 +672,117 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     continue;
                 }
                 const uint8_t* stage = ring + slot * kDecStageBytes;
-                if (gu) {
-                    const int kc = s * kDecGuChunks + st;  // K chunk of d
-                    const uint16_t* xr = brow + kKChunk * kc;
-#pragma unroll
-                    for (int tt = 0; tt < 2; ++tt)
-                        chunk_mma<kGpc>(acc[tt], stage, 256 * 32, 32 * warp + 16 * tt + g, c, xr,
-                                        bs0 + 2 * kc, bs1 + 2 * kc);
-                } else {
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int kc = s * dn_chunks + 2 * st + half;  // K chunk of f
-                        chunk_mma<kGpc>(acc[0], stage + half * p.bb_dn, 128 * 32, 16 * warp + g, c,
-                                        brow + kKChunk * kc, bs0 + 2 * kc, bs1 + 2 * kc);
-                    }
-                }
+                chunk_mma_rows<kGpc>(acc, stage + fr * 32, stage + (kDecSlice + fr) * 32,
+                                     stage + 2 * kDecSlice * 32 + fr * kGpc * 4,
+                                     stage + 2 * kDecSlice * 32 + sc_bytes + fr * kGpc * 4, c,
+                                     brow + kKChunk * st, bs0 + 2 * st, bs1 + 2 * st);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(slot));
             }
+            // SwiGLU of the slice, rounded to bf16, into shared memory [token][64]
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int col = 2 * c + e2;
+                if (col < n) {
+                    const float gv = acc[e2];
+                    const float uv = acc[2 + e2];
+                    hsh[col * kDecHStride + fr] = bf16_round_bits(__fdividef(gv * uv, 1.0f + __expf(-gv)));
+                }
+            }
             compute_sync();
             if (vload(R.fail)) break;
-            // partial sums of this unit -> workspace, then count the unit
-            if (gu) {
-#pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    const int ra = 32 * warp + 16 * tt + g;
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const int col = 2 * c + e2;
-                        if (col < n) {
-                            float* dst = p.pgu + ((static_cast<size_t>(row0 + col) * NT + j) * KS + s) * 256;
-                            dst[ra] = acc[tt][e2];
-                            dst[ra + 8] = acc[tt][2 + e2];
-                        }
+            // the 32-wide vector sums of the h rows (K order), for the group folds
+            if (tid < 2 * n) {
+                const int col = tid >> 1, v = tid & 1;
+                float sacc = 0.0f;
+                for (int i = 0; i < 32; ++i) sacc += bf16_bits_to_float(hsh[col * kDecHStride + 32 * v + i]);
+                hsum[col * 2 + v] = sacc;
+            }
+            compute_sync();
+            // down: output tile jd, rows 16w .. 16w + 15 of its 128; K = the slice
+            const uint16_t* hrow = hsh + cg * kDecHStride + 8 * c;
+            const float* hs0 = hsum + c0 * 2;
+            const float* hs1 = hsum + c1 * 2;
+            const int ra = 16 * warp + g;
+            for (int jd = 0; jd < NTd; ++jd, ++q) {
+                const int slot = q % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
+                    if (lane == 0) {
+                        R.fail = 1;
+                        if (!vload(R.abort_local)) dec_fail(p, R, 506);
                     }
+                    continue;
                 }
-            } else {
-                const int ra = 16 * warp + g;
+                const uint8_t* stage = ring + slot * kDecStageBytes;
+                float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                chunk_mma<kGpc>(o, stage, 128 * 32, ra, c, hrow, hs0, hs1);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty(slot));
 #pragma unroll
                 for (int e2 = 0; e2 < 2; ++e2) {
                     const int col = 2 * c + e2;
                     if (col < n) {
-                        float* dst = p.pdn + ((static_cast<size_t>(row0 + col) * NTd + j) * DS + s) * 128;
-                        dst[ra] = acc[0][e2];
-                        dst[ra + 8] = acc[0][2 + e2];
+                        float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128;
+                        dst[ra] = o[e2];
+                        dst[ra + 8] = o[2 + e2];
                     }
                 }
             }
-            __threadfence();
             compute_sync();
-            if (tid == 0) {
-                int* cnt = gu ? sync + kSyncGu + b * NT + j : sync + kSyncDn + j;
-                const int last = gu ? KS - 1 : nb * DS - 1;
-                R.flag = atom_acq_rel_add(cnt, 1) == last;
-            }
-            compute_sync();
-            if (vload(R.flag)) {
-                if (gu) {
-                    // the block's h for this tile: sum the K parts in order,
-                    // SwiGLU, round to bf16
-                    for (int it = tid; it < 128 * n; it += kDecComputeThreads) {
-                        const int r = it & 127;
-                        const int col = it >> 7;
-                        const float* src = p.pgu + (static_cast<size_t>(row0 + col) * NT + j) * KS * 256;
-                        float gs = 0.0f, us = 0.0f;
-                        for (int s2 = 0; s2 < KS; ++s2) {
-                            gs += ld_cg_f32(src + s2 * 256 + r);
-                            us += ld_cg_f32(src + s2 * 256 + 128 + r);
-                        }
-                        p.h[static_cast<size_t>(row0 + col) * f + j * 128 + r] =
-                            bf16_round_bits(__fdividef(gs * us, 1.0f + __expf(-gs)));
-                    }
-                    __threadfence();
-                    compute_sync();
-                    if (tid == 0) red_release_add(sync + kSyncHReady + b, 1);
-                } else {
-                    // output tile j of every token: each expert output is the sum
-                    // of its K halves rounded to bf16; the token's slots are
-                    // summed in slot order
-                    for (int it = tid; it < 128 * T; it += kDecComputeThreads) {
-                        const int m = it & 127;
-                        const int t = it >> 7;
-                        float yv = 0.0f;
-                        for (int jj = 0; jj < k; ++jj) {
-                            const int pr = R.pos[t * k + jj];
-                            const float* src = p.pdn + (static_cast<size_t>(pr) * NTd + j) * DS * 128 + m;
-                            float o = ld_cg_f32(src);
-                            for (int s2 = 1; s2 < DS; ++s2) o += ld_cg_f32(src + s2 * 128);
-                            yv = fmaf(R.w[t * k + jj], bf16_round(o), yv);
-                        }
-                        p.y[static_cast<size_t>(t) * d + j * 128 + m] = bf16_round_bits(yv);
-                    }
-                }
-            }
+            if (vload(R.fail)) break;
         }
     }
 
-    // ---- phase 4: exit; the last CTA resets the flags ----------------------
+    // ---- phase 4: combine, after every CTA is done with its units ----------
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        red_release_add(sync + kSyncUnits, 1);
+        R.hok = routed && !vload(R.abort_local);
+        if (R.hok && !wait_flag(sync + kSyncUnits, G, abort_g)) {
+            dec_fail(p, R, 507);
+            R.hok = 0;
+        }
+    }
+    __syncthreads();
+    if (vload(R.hok)) {
+        // this CTA's outputs: flattened (t, m) in [o0, o1); first each
+        // (output, slot) pair's expert output (the slice partials summed in
+        // slice order, rounded to bf16), then each output's slots in order
+        float* ob = reinterpret_cast<float*>(ring);  // the ring is idle now
+        const int per = (T * d + G - 1) / G;
+        const int o0 = cta * per;
+        const int o1 = min(T * d, o0 + per);
+        const int cnt = max(o1 - o0, 0);
+        for (int it = tid; it < cnt * k; it += kDecThreads) {
+            const int jj = it / cnt;
+            const int li = it - jj * cnt;
+            const int oi = o0 + li;
+            const int t = oi / d;
+            const int m = oi - t * d;
+            const float* src = p.pdn + static_cast<size_t>(R.pos[t * k + jj]) * S * d + m;
+            float v[kDecMaxSlices];
+#pragma unroll
+            for (int sl = 0; sl < kDecMaxSlices; ++sl)
+                if (sl < S) v[sl] = ld_cg_f32(src + static_cast<size_t>(sl) * d);
+            float sum = v[0];
+#pragma unroll
+            for (int sl = 1; sl < kDecMaxSlices; ++sl)
+                if (sl < S) sum += v[sl];
+            ob[jj * cnt + li] = bf16_round(sum);
+        }
+        __syncthreads();
+        for (int li = tid; li < cnt; li += kDecThreads) {
+            const int oi = o0 + li;
+            const int t = oi / d;
+            const int m = oi - t * d;
+            float yv = 0.0f;
+            for (int jj = 0; jj < k; ++jj) yv = fmaf(R.w[t * k + jj], ob[jj * cnt + li], yv);
+            p.y[static_cast<size_t>(t) * d + m] = bf16_round_bits(yv);
+        }
+    }
+
+    // ---- exit: the last CTA resets the flags --------------------------------
     __syncthreads();
     if (tid == 0) {
         __threadfence();
@@ -798,20 +802,15 @@ constexpr int kDecSmemLimit = 227 * 1024;
 bool decode_supported(const moe_shape_t& s, int T) {
     if (T < 1 || T > kDecodeMaxT) return false;
     if (T * s.k > kDecMaxAssign || s.E > kMaxExperts || s.E % 8 != 0) return false;
-    if (s.f / 128 > kDecMaxNT || s.d / 128 > kDecMaxNTd) return false;
+    if (s.f / kDecSlice > kDecMaxSlices || s.d / 128 > kDecMaxNTd) return false;
     return dec_smem_layout(T, s.d, s.E, s.f).total <= kDecSmemLimit;
 }
 
 size_t decode_workspace_bytes(const moe_shape_t& s, int T_max) {
     const size_t T = static_cast<size_t>(std::min(T_max, kDecodeMaxT));
     const size_t Tk = T * s.k;
-    const size_t KS = (s.d / kKChunk) / kDecGuChunks;
-    const size_t DS = ((s.f / kKChunk) % 4 == 0) ? 2 : 1;
-    const size_t u = T * s.E * 8 * 4;
-    const size_t gu = Tk * (s.f / 128) * KS * 256 * 4;
-    const size_t dn = Tk * (s.d / 128) * DS * 128 * 4;
     auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
-    return r256(u) + r256(gu) + r256(dn);
+    return r256(T * s.E * 8 * 4) + r256(Tk * (s.f / kDecSlice) * s.d * 4);
 }
 
 cudaError_t prepare_decode_kernels() {
@@ -850,14 +849,10 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t st) {
     p.num_blocks = a.num_blocks;
     p.topk_w = a.topk_w;
     const size_t T = static_cast<size_t>(a.T);
-    const size_t Tk = T * s.k;
-    const size_t KS = (s.d / kKChunk) / kDecGuChunks;
     auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
     uint8_t* scratch = a.scratch;
     p.U = reinterpret_cast<float*>(scratch);
-    p.pgu = reinterpret_cast<float*>(scratch + r256(T * s.E * 8 * 4));
-    p.pdn = reinterpret_cast<float*>(scratch + r256(T * s.E * 8 * 4) + r256(Tk * (s.f / 128) * KS * 256 * 4));
-    p.h = a.h;
+    p.pdn = reinterpret_cast<float*>(scratch + r256(T * s.E * 8 * 4));
     p.y = a.y;
     p.status = a.status;
     p.sync = a.sync;
