@@ -297,6 +297,11 @@ def run_ours(args, name):
 
     shape, seed, zipf = mi.WORKLOADS[name]
     inp = mi.workload(name)
+    if args.tokens:
+        # the first `tokens` tokens of the workload (a smaller case of the same layer)
+        n = min(args.tokens, inp.shape.T)
+        inp = mi.Inputs(mi.Shape(n, *[getattr(inp.shape, f) for f in ("d", "E", "k", "f", "group")]),
+                        inp.seed, inp.x[:n], inp.w_r, inp.b_r, inp.gate, inp.up, inp.down)
     s = inp.shape
     layer = MoeLayer.from_inputs(inp)
     x = bf16_tensor(inp.x, "cuda")
@@ -413,9 +418,9 @@ def run_ours(args, name):
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum (bytes) of one gate/up GEMM
-# launch, from the ncu capture summarised in profiles/kernels_prefill_t8192.md;
-# workloads without a capture of the current kernel report None.
-TRAFFIC_GATEUP: dict = {"prefill_t8192": 583670528}
+# launch from an ncu capture of the current kernel build (profiles/); workloads
+# without such a capture report None.
+TRAFFIC_GATEUP: dict = {}
 
 
 def main():
@@ -430,6 +435,8 @@ def main():
                     help="repeats of the timed loop of K steps; the median is reported")
     ap.add_argument("--no-configs", action="store_true",
                     help="time only the main workload (not the other layer configurations)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="use only the first TOKENS tokens of the workload (smaller cases for profilers)")
     ap.add_argument("--profile", type=int, default=0,
                     help="run this many extra layer calls after set-up and exit (for ncu)")
     args = ap.parse_args()

@@ -61,18 +61,23 @@ struct ApproxArgs {
 };
 
 // ---------------------------------------------------------------------------
-// Prep.  Blocks [0, nxb): eight tokens each (warp per token).  Blocks
-// [nxb, nxb + E/8): eight experts each (thread (g, el): rows i = g, g + 32, ...
-// of expert 8o + el).
+// Prep.  Blocks [0, nxb): eight tokens each (warp per token; the row stays in
+// registers, 16-byte vectors v = lane, lane + 32, ...).  Blocks [nxb, nxb + E):
+// one expert each (thread t holds rows t, t + 256, ... of the column).
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 256;
+constexpr int kPrepMaxVec = 16;   // 16-byte vectors of a token row per lane: d <= 4096
+constexpr int kPrepMaxRows = 16;  // W_r rows per thread of an expert block: d <= 4096
 
-// smallest power of two p with m < 128 p (m > 0); exact
+// power of two p with m < 2^span_log2 * p (m > 0); exact
 __device__ __forceinline__ float pow2_scale(float m, int span_log2) {
     int ex;
     frexpf(m, &ex);  // m = f 2^ex, f in [0.5, 1): m < 2^ex
     return ldexpf(1.0f, ex - span_log2);
 }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __global__ void __launch_bounds__(kPrepThreads)
 router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, int T, int d, int E,
@@ -91,16 +96,19 @@ router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, 
         const int t = blockIdx.x * 8 + warp;
         if (t >= T) return;
         const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
-        const int nv = d >> 3;  // 16-byte vectors, <= 8 per lane for d <= 2048... general loop
+        const int nv = d >> 3;
+        uint4 q[kPrepMaxVec];
         float m = 0.0f;
-        for (int v = lane; v < nv; v += 32) {
-            const uint4 q = __ldg(row + v);
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                m = fmaxf(m, fabsf(__uint_as_float(w[i] << 16)));
-                m = fmaxf(m, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
-            }
+        for (int j = 0; j < kPrepMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            q[j] = v < nv ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < kPrepMaxVec; ++j) {
+            const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -112,24 +120,28 @@ router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, 
         float emax = 0.0f;
         int8_t* pa = ws.xa + static_cast<size_t>(t) * d;
         int8_t* pb = ws.xb + static_cast<size_t>(t) * d;
-        for (int v = lane; v < nv; v += 32) {
-            const uint4 q = __ldg(row + v);
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < kPrepMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            if (v >= nv) continue;
+            const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
             uint32_t oa[2] = {0u, 0u}, ob[2] = {0u, 0u};
+            float fs = 0.0f, fq = 0.0f;  // exact: eight bf16 values
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float xv = __uint_as_float(i & 1 ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16));
+                const float xv = i & 1 ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
                 const float z = xv * inv;                     // exact
                 const float a = fminf(fmaxf(rintf(z), -127.0f), 127.0f);
                 const float r = z - a;                        // exact, |r| <= 0.5
                 const float b = rintf(r * 128.0f);            // |b| <= 64
-                const float e = fabsf(s * (r - b * 0.0078125f));  // exact: the remainder of x
-                emax = fmaxf(emax, e);
-                sabs += fabs(static_cast<double>(xv));
-                ssq += static_cast<double>(xv) * xv;
+                emax = fmaxf(emax, fabsf(s * (r - b * 0.0078125f)));  // exact: the remainder of x
+                fs += fabsf(xv);
+                fq = fmaf(xv, xv, fq);
                 oa[i >> 2] |= (static_cast<uint32_t>(static_cast<int>(a)) & 0xFFu) << (8 * (i & 3));
                 ob[i >> 2] |= (static_cast<uint32_t>(static_cast<int>(b)) & 0xFFu) << (8 * (i & 3));
             }
+            sabs += static_cast<double>(fs);
+            ssq += static_cast<double>(fq);
             *reinterpret_cast<uint2*>(pa + 8 * v) = make_uint2(oa[0], oa[1]);
             *reinterpret_cast<uint2*>(pb + 8 * v) = make_uint2(ob[0], ob[1]);
         }
@@ -142,58 +154,69 @@ router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, 
         if (lane == 0) {
             ws.s_t[t] = s;
             ws.E_t[t] = emax;
-            // sum |x'| <= sum |x| + d max|x - x'|; the double sums are exact to
-            // far below the 1e-9 margin
-            ws.A_t[t] = __double2float_ru((sabs + static_cast<double>(d) * emax) * (1.0 + 1e-9));
-            ws.N_t[t] = __double2float_ru(sqrt(ssq) * (1.0 + 1e-9));
+            // sum |x'| <= sum |x| + d max|x - x'|; eight-term fp32 partial sums
+            // and the double sums are off by far less than the 1e-6 margin
+            ws.A_t[t] = __double2float_ru((sabs + static_cast<double>(d) * emax) * (1.0 + 1e-6));
+            ws.N_t[t] = __double2float_ru(sqrt(ssq) * (1.0 + 1e-6));
         }
         return;
     }
-    // experts 8o .. 8o + 7: thread (g, el), g = threadIdx.x >> 3 (0..31),
-    // el = threadIdx.x & 7, rows i = g + 32 j
-    __shared__ float sm_max[32][8];
-    __shared__ double sm_abs[32][8], sm_sq[32][8];
-    __shared__ float sm_u[8];
-    __shared__ float sm_f[32][8];
-    const int o = blockIdx.x - nxb;
-    const int g = threadIdx.x >> 3;
-    const int el = threadIdx.x & 7;
-    const int e = 8 * o + el;
+    // expert e: thread t holds rows i = t + 256 j
+    __shared__ float sm_max[kPrepThreads / 32], sm_f[kPrepThreads / 32];
+    __shared__ double sm_abs[kPrepThreads / 32], sm_sq[kPrepThreads / 32];
+    __shared__ float sm_u;
+    const int e = blockIdx.x - nxb;
+    float w[kPrepMaxRows];
     float m = 0.0f;
     double sabs = 0.0, ssq = 0.0;
-    for (int i = g; i < d; i += 32) {
-        const float w = __ldg(W + static_cast<size_t>(i) * E + e);
-        m = fmaxf(m, fabsf(w));
-        sabs += fabs(static_cast<double>(w));
-        ssq += static_cast<double>(w) * w;
+#pragma unroll
+    for (int j = 0; j < kPrepMaxRows; ++j) {
+        const int i = threadIdx.x + kPrepThreads * j;
+        w[j] = i < d ? __ldg(W + static_cast<size_t>(i) * E + e) : 0.0f;
     }
-    sm_max[g][el] = m;
-    sm_abs[g][el] = sabs;
-    sm_sq[g][el] = ssq;
+#pragma unroll
+    for (int j = 0; j < kPrepMaxRows; ++j) {
+        m = fmaxf(m, fabsf(w[j]));
+        sabs += fabs(static_cast<double>(w[j]));
+        ssq += static_cast<double>(w[j]) * w[j];
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        sabs += __shfl_xor_sync(0xffffffffu, sabs, o);
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    }
+    if (lane == 0) {
+        sm_max[warp] = m;
+        sm_abs[warp] = sabs;
+        sm_sq[warp] = ssq;
+    }
     __syncthreads();
-    if (threadIdx.x < 8) {
+    if (threadIdx.x == 0) {
         float mm = 0.0f;
         double a = 0.0, q = 0.0;
-        for (int i = 0; i < 32; ++i) {
-            mm = fmaxf(mm, sm_max[i][threadIdx.x]);
-            a += sm_abs[i][threadIdx.x];
-            q += sm_sq[i][threadIdx.x];
+        for (int i = 0; i < kPrepThreads / 32; ++i) {
+            mm = fmaxf(mm, sm_max[i]);
+            a += sm_abs[i];
+            q += sm_sq[i];
         }
         // |w / u| < 64: c = round(w / u), remainder r with |r| <= 0.5,
         // d = round(128 r), |d| <= 64, no clamping
         const float u = mm > 0.0f ? pow2_scale(mm, 6) : 1.0f;
-        sm_u[threadIdx.x] = u;
-        ws.u_e[8 * o + threadIdx.x] = u;
-        ws.B_e[8 * o + threadIdx.x] = __double2float_ru(a * (1.0 + 1e-9));
-        ws.Wn_e[8 * o + threadIdx.x] = __double2float_ru(sqrt(q) * (1.0 + 1e-9));
+        sm_u = u;
+        ws.u_e[e] = u;
+        ws.B_e[e] = __double2float_ru(a * (1.0 + 1e-9));
+        ws.Wn_e[e] = __double2float_ru(sqrt(q) * (1.0 + 1e-9));
     }
     __syncthreads();
-    const float u = sm_u[el];
+    const float u = sm_u;
     const float inv = 1.0f / u;
     float fmax_ = 0.0f;
-    for (int i = g; i < d; i += 32) {
-        const float w = __ldg(W + static_cast<size_t>(i) * E + e);
-        const float z = w * inv;               // exact
+#pragma unroll
+    for (int j = 0; j < kPrepMaxRows; ++j) {
+        const int i = threadIdx.x + kPrepThreads * j;
+        if (i >= d) continue;
+        const float z = w[j] * inv;            // exact
         const float c = rintf(z);
         const float r = z - c;                 // exact
         const float dd = rintf(r * 128.0f);
@@ -201,15 +224,16 @@ router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, 
         ws.wc[static_cast<size_t>(e) * d + i] = static_cast<int8_t>(static_cast<int>(c));
         ws.wd[static_cast<size_t>(e) * d + i] = static_cast<int8_t>(static_cast<int>(dd));
     }
-    sm_f[g][el] = fmax_;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) fmax_ = fmaxf(fmax_, __shfl_xor_sync(0xffffffffu, fmax_, o));
+    if (lane == 0) sm_f[warp] = fmax_;
     __syncthreads();
-    if (threadIdx.x < 8) {
+    if (threadIdx.x == 0) {
         float f = 0.0f;
-        for (int i = 0; i < 32; ++i) f = fmaxf(f, sm_f[i][threadIdx.x]);
-        ws.F_e[8 * o + threadIdx.x] = f;
+        for (int i = 0; i < kPrepThreads / 32; ++i) f = fmaxf(f, sm_f[i]);
+        ws.F_e[e] = f;
     }
 }
-
 
 // ---------------------------------------------------------------------------
 // Approximate logits on the tensor cores.  One CTA per 64 tokens x 128
@@ -494,15 +518,16 @@ router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, i
 // in the router's fixed order: lane p runs chain p with fused multiply-add,
 // then the xor butterfly, then the bias.  One CTA per slice of 16 experts
 // (W_r slice in shared memory, rows padded to 20 floats) sweeps 64-token
-// tiles; a tile's pairs are listed in shared memory and done 64 at a time
-// (eight per warp) while the tile's x rows stream through a double-buffered
-// ring of 128-wide K chunks.
+// tiles; a tile's pairs are listed in shared memory and done up to 128 at a
+// time (16 per warp) while the tile's x rows stream through a ring of six
+// 64-wide K chunks (five in flight).
 // ---------------------------------------------------------------------------
-constexpr int kExES = 16, kExWS = 20, kExTile = 64, kExKc = 128, kExWarps = 8;
-constexpr int kExPairsPerWarp = 8;
+constexpr int kExES = 16, kExWS = 20, kExTile = 64, kExKc = 64, kExStages = 6, kExWarps = 8;
+constexpr int kExPairsPerWarp = 16;
 constexpr int kExPass = kExWarps * kExPairsPerWarp;
+constexpr int kExChunkBytes = kExTile * kExKc * 2;
 __host__ __device__ constexpr int ex_smem_bytes(int d) {
-    return d * kExWS * 4 + 2 * kExTile * kExKc * 2 + kExTile * kExES * 4 + 64;
+    return d * kExWS * 4 + kExStages * kExChunkBytes + kExTile * kExES * 4 + 64;
 }
 
 __global__ void __launch_bounds__(kExWarps * 32, 1)
@@ -511,7 +536,7 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     extern __shared__ __align__(16) uint8_t ex_raw[];
     float* Ws = reinterpret_cast<float*>(ex_raw);
     uint16_t* xs = reinterpret_cast<uint16_t*>(ex_raw + static_cast<size_t>(d) * kExWS * 4);
-    int* pairs = reinterpret_cast<int*>(ex_raw + static_cast<size_t>(d) * kExWS * 4 + 2 * kExTile * kExKc * 2);
+    int* pairs = reinterpret_cast<int*>(ex_raw + static_cast<size_t>(d) * kExWS * 4 + kExStages * kExChunkBytes);
     int* npairs = pairs + kExTile * kExES;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -531,16 +556,21 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     const uint32_t xs_base = smem_u32(xs);
     const int ntiles = (T + kExTile - 1) / kExTile;
     const int nkc = d / kExKc;
-    auto load_chunk = [&](int t0, int kc, int buf) {
-        // 64 rows x 256 bytes = 1024 pieces of 16 bytes, 4 per thread
+    // one K chunk of the tile (64 rows x 128 bytes = 512 pieces of 16 bytes,
+    // two per thread) into ring stage kc % kExStages; every call commits one
+    // group (empty past the last chunk), so wait_group counts stay uniform
+    auto load_chunk = [&](int t0, int kc) {
+        if (kc < nkc) {
 #pragma unroll
-        for (int j = 0; j < (kExTile * kExKc * 2 / 16) / (kExWarps * 32); ++j) {
-            const int piece = threadIdx.x + j * kExWarps * 32;
-            const int row = piece / (kExKc * 2 / 16);
-            const int col = piece % (kExKc * 2 / 16);
-            const int t = t0 + row;
-            const uint16_t* src = x + static_cast<size_t>(t < T ? t : 0) * d + kc * kExKc + col * 8;
-            cp_async_16(xs_base + ((buf * kExTile + row) * kExKc + col * 8) * 2, src, t < T ? 16u : 0u);
+            for (int j = 0; j < (kExChunkBytes / 16) / (kExWarps * 32); ++j) {
+                const int piece = threadIdx.x + j * kExWarps * 32;
+                const int row = piece / (kExKc * 2 / 16);
+                const int col = piece % (kExKc * 2 / 16);
+                const int t = t0 + row;
+                const uint16_t* src = x + static_cast<size_t>(t < T ? t : 0) * d + kc * kExKc + col * 8;
+                cp_async_16(xs_base + (kc % kExStages) * kExChunkBytes + (row * kExKc + col * 8) * 2, src,
+                            t < T ? 16u : 0u);
+            }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -573,26 +603,24 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
                 el[j] = code % kExES;
                 acc[j] = 0.0f;
             }
-            load_chunk(t0, 0, 0);
+            __syncthreads();  // every thread has read the ring's previous contents
+#pragma unroll
+            for (int kc = 0; kc < kExStages - 1; ++kc) load_chunk(t0, kc);
             for (int kc = 0; kc < nkc; ++kc) {
-                if (kc + 1 < nkc) {
-                    load_chunk(t0, kc + 1, (kc + 1) & 1);
-                    asm volatile("cp.async.wait_group 1;" ::: "memory");
-                } else {
-                    asm volatile("cp.async.wait_group 0;" ::: "memory");
-                }
+                load_chunk(t0, kc + kExStages - 1);
+                asm volatile("cp.async.wait_group %0;" ::"n"(kExStages - 1) : "memory");
                 __syncthreads();
-                const uint16_t* xb = xs + (kc & 1) * kExTile * kExKc;
+                const uint16_t* xb = xs + (kc % kExStages) * (kExTile * kExKc);
 #pragma unroll
                 for (int s = 0; s < kExKc / 32; ++s) {
-                    const int il = 32 * s + lane;             // chain lane: i = kc*128 + il
+                    const int il = 32 * s + lane;             // chain lane: i = kc*64 + il
                     const float* wrow = Ws + (kc * kExKc + il) * kExWS;
 #pragma unroll
                     for (int j = 0; j < kExPairsPerWarp; ++j)
                         if (on[j])
                             acc[j] = __fmaf_rn(bf16_bits_to_float(xb[tl[j] * kExKc + il]), wrow[el[j]], acc[j]);
                 }
-                __syncthreads();  // the buffer is refilled by the next chunk's copies
+                __syncthreads();  // the stage is refilled by a later chunk's copies
             }
 #pragma unroll
             for (int j = 0; j < kExPairsPerWarp; ++j) {
@@ -607,6 +635,7 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
             }
         }
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -645,7 +674,7 @@ router_select_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, int 
 
 bool router_fast_supported(int T, int d, int E) {
     return T >= kFastRouterMinT && E % kExES == 0 && E <= kMaxExperts && d % 128 == 0 &&
-           ex_smem_bytes(d) <= 227 * 1024;
+           d <= kPrepThreads * kPrepMaxRows && d <= 8 * 32 * kPrepMaxVec && ex_smem_bytes(d) <= 227 * 1024;
 }
 
 size_t router_fast_ws_bytes(int T, int d, int E) {
@@ -716,7 +745,7 @@ cudaError_t launch_router_fast(const uint16_t* x, const float* W, const float* b
     cudaError_t e = router_fast_setup(&num_sms);
     if (e != cudaSuccess) return e;
     const int nxb = (T + 7) / 8;
-    e = launch_pdl(router_prep_kernel, dim3(nxb + E / 8), dim3(kPrepThreads), 0, st, x, W, T, d, E, nxb, ws,
+    e = launch_pdl(router_prep_kernel, dim3(nxb + E), dim3(kPrepThreads), 0, st, x, W, T, d, E, nxb, ws,
                    hist, hist_n, status);
     if (e != cudaSuccess) return e;
     ApproxArgs a{};
