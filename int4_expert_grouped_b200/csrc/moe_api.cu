@@ -359,11 +359,8 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.out_ld = s.f;
     g.group = s.group;
     g.block_bytes = plan->group_bytes;
-    // pairs of CTAs share each MMA (M = 256) when the tiles pair up
-    g.pair = g.NT % 2 == 0;
-    g.max_units = mb * (g.pair ? g.NT / 2 : g.NT);
-    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, xs, static_cast<uint64_t>(Tk), s.d,
-                                       g.pair ? moe::kBlockT / 2 : moe::kBlockT));
+    g.max_units = mb * g.NT;
+    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
     if (ev && !mark(ev->gate_up)) return MOE_ERR_CUDA;
 
@@ -374,10 +371,8 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.NT = s.d / (128 * moe::kDownTiles);
     g.out_ld = s.d;
     g.block_bytes = plan->down_block_bytes;
-    g.pair = g.NT % 2 == 0;
-    g.max_units = mb * (g.pair ? g.NT / 2 : g.NT);
-    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(Tk), s.f,
-                                       g.pair ? moe::kBlockT / 2 : moe::kBlockT));
+    g.max_units = mb * g.NT;
+    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;
     MOE_CUDA(moe::launch_combine(xs, r.pos, r.w, T, s.k, s.d, y, status, num_sms, st));

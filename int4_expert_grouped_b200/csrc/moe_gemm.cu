@@ -42,8 +42,6 @@
 // MMA but exposes the epilogue).
 #include <cudaTypedefs.h>
 
-#include <algorithm>
-
 #include "moe_internal.h"
 
 namespace moe {
@@ -60,23 +58,18 @@ constexpr int kNumEpiWarps = 4;
 constexpr int kGemmThreads = 16 * 32;
 constexpr int kTransformThreads = kNumTransformWarps * 32;
 constexpr int kATileBytes = 128 * 128;     // 128 rows x 64 bf16 (128B swizzle)
+constexpr int kBStageBytes = kBlockT * 128;  // up to 256 token rows x 64 bf16
 constexpr int kEpiRowBytes = 80;    // staging row: 32 bf16 + 16 bytes of padding
 constexpr uint32_t kTmemCols = 512;
 
-// Per-projection configuration.  kPair: a pair of CTAs (a cluster of two)
-// shares each MMA (cta_group::2, M = 256): every CTA expands its own 128-row
-// weight tiles and holds half of the token tile, so each SM's shared memory
-// serves half the token operand per flop; the first CTA of the pair issues
-// the MMAs for both.
-template <bool kDown, bool kPair>
+// Per-projection configuration.
+template <bool kDown>
 struct Cfg {
     static constexpr int kTiles = kDown ? kDownTiles : 2;     // A tiles (of 128 rows) per unit
     static constexpr bool kOneTile = kTiles == 1;
-    static constexpr int kBRows = kPair ? kBlockT / 2 : kBlockT;  // token rows per CTA and stage
-    static constexpr int kBStageBytes = kBRows * 128;
     static constexpr int kNW = kOneTile ? 4 : 2;              // packed weight ring
-    static constexpr int kNA = kOneTile ? 4 : (kPair ? 4 : 3);  // expanded bf16 A ring
-    static constexpr int kNB = kPair ? (kOneTile ? 6 : 4) : 3;  // token B ring
+    static constexpr int kNA = kOneTile ? 4 : 3;              // expanded bf16 A ring
+    static constexpr int kNB = 3;                             // token B ring
     static constexpr int kAccBufs = kOneTile ? 2 : 1;         // TMEM accumulator buffers
     static constexpr int kAccCols = kTiles * kBlockT;         // columns per buffer
     static constexpr int kAStageBytes = kTiles * kATileBytes;
@@ -87,7 +80,6 @@ struct Cfg {
     static constexpr int kGroups = kOneTile ? 2 : 1;
     static constexpr int kGroupThreads = kTransformThreads / kGroups;
     static constexpr int kTasks = kTiles * 256 / kGroupThreads;  // (row, half) tasks per thread
-    static constexpr int kCtas = kPair ? 2 : 1;               // CTAs whose arrivals a phase counts
 
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + kNA * kAStageBytes;
@@ -98,8 +90,7 @@ struct Cfg {
     static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base
 
-    static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0 && kAStageBytes % 1024 == 0 &&
-                      kBStageBytes % 1024 == 0,
+    static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0 && kAStageBytes % 1024 == 0,
                   "UMMA tiles need 1024-byte alignment");
     static_assert(kOffW % 16 == 0 && kWStageBytes % 16 == 0, "bulk copies need 16-byte alignment");
     static_assert(kOffBar % 8 == 0, "mbarriers are 8-byte aligned");
@@ -132,34 +123,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
-// The same for a barrier that the other CTA of the pair also arrives on:
-// acquire at cluster scope.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    bool ok = mbar_try_wait_cluster(bar, parity);
-    if (!ok) {
-        const uint64_t t0 = globaltimer();
-        for (uint32_t n = 1;; ++n) {
-            if (mbar_try_wait_cluster(bar, parity)) {
-                ok = true;
-                break;
-            }
-            if ((n & 63u) == 0 && (*abort_flag || globaltimer() - t0 > kWaitTimeoutNs)) break;
-        }
-    }
-    return __all_sync(0xffffffffu, ok);
-}
-
 // Wait used only while shutting down after an abort: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = globaltimer();
@@ -169,74 +132,9 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
     return true;
 }
 
-// Address of the same shared-memory word in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Arrive on an mbarrier given by its shared::cluster address (release at
-// cluster scope: this thread's earlier writes are visible to the waiter).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// ---- tcgen05 forms for a pair of CTAs ----
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                              uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// Arrive once on the mbarrier at `bar` in both CTAs of the pair when every
-// tcgen05 operation this thread issued so far has completed.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-        ::"r"(bar), "h"(static_cast<uint16_t>(3))
-        : "memory");
-}
-// The same, arriving only on this CTA's barrier.
-__device__ __forceinline__ void mma_commit_pair_local(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-// 2-D TMA tile into this CTA's shared memory whose completion is counted on
-// the barrier at `cluster_bar` (the first CTA of the pair's).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int c0, int c1,
-                                                 uint32_t cluster_bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(cluster_bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-template <bool kDown, bool kPair>
+template <bool kDown>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
-    using C = Cfg<kDown, kPair>;
+    using C = Cfg<kDown>;
     extern __shared__ uint8_t smem_raw[];
     pdl_launch_dependents();
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -244,9 +142,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint32_t rank = kPair ? cluster_rank() : 0;   // 0: issues the pair's MMAs
-    const int cta_id = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-    const int n_ctas = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     // barrier addresses
     const uint32_t bar0 = sbase + C::kOffBar;
@@ -270,7 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             mbar_init(wempty(s), kNumTransformWarps / C::kGroups);
         }
         for (int s = 0; s < C::kNA; ++s) {
-            mbar_init(afull(s), C::kCtas * kNumTransformWarps / C::kGroups);
+            mbar_init(afull(s), kNumTransformWarps / C::kGroups);
             mbar_init(aempty(s), 1);
         }
         for (int s = 0; s < C::kNB; ++s) {
@@ -279,53 +174,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         }
         for (int s = 0; s < C::kAccBufs; ++s) {
             mbar_init(accfull(s), 1);
-            mbar_init(accempty(s), C::kCtas * kNumEpiWarps);
+            mbar_init(accempty(s), kNumEpiWarps);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
     if (warp == kWarpMma) {
-        if constexpr (kPair) {
-            tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-            tmem_relinquish();
-        }
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
     }
     tc_fence_before();
-    if constexpr (kPair)
-        cluster_sync_all();  // both CTAs' barriers exist before either arrives on the other's
-    else
-        __syncthreads();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     pdl_wait();  // the block map, the token rows and (down) h come from earlier kernels
 
-    // with a pair, the barriers that count both CTAs' work live in the first CTA
-    auto lead = [&](uint32_t bar) { return kPair ? cluster_addr(bar, 0) : bar; };
-
-    const int NT = a.NT;          // 128-row output tiles per expert
-    const int NU = kPair ? NT / 2 : NT;  // output tiles per unit row: 256 rows for a pair
+    const int NT = a.NT;
     const int KC = a.K / kKChunk;
-    const int num_units = min(*a.num_blocks * NU, a.max_units);
+    const int num_units = min(*a.num_blocks * NT, a.max_units);
 
     auto fail = [&](int where) {
         *abort_flag = 1;
         report_error(a.status, MOE_ERR_DEVICE_TIMEOUT, (kDown ? 200 : 100) + where);
     };
-    // rows of the unit's token tile the MMA reads (a multiple of 32 for a
-    // pair, so each CTA holds a multiple of 16)
-    auto mma_n = [&](int rows) { return kPair ? (rows + 31) & ~31 : (rows + 15) & ~15; };
 
     if (warp == kWarpWProducer) {
         // the whole warp runs the loop; one elected lane issues the copies
         uint32_t it = 0;
         bool ok = true;
-        for (int u = cta_id; ok && u < num_units; u += n_ctas) {
-            const int b = u / NU;
-            const int j = (u - b * NU) * C::kCtas + static_cast<int>(rank);  // this CTA's tile
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            const int b = u / NT;
+            const int j = u - b * NT;
             const int e = a.block_map[3 * b];
             const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
             for (int c = 0; c < KC; ++c, ++it) {
@@ -352,22 +232,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     } else if (warp == kWarpMma) {
         // The whole warp runs the issue loop so descriptors and ring indices
         // stay warp-uniform; one elected lane issues each MMA and commit.
-        // With a pair only the first CTA issues (M = 256: its tiles and the
-        // other CTA's, at the same shared-memory offsets).
         uint32_t it = 0, ucount = 0;
         bool ok = true;
         bool ready = false;  // the current stage was already seen full
-        bool issued = false;
-        for (int u = cta_id; ok && rank == 0 && u < num_units; u += n_ctas, ++ucount) {
-            const int b = u / NU;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x, ++ucount) {
+            const int b = u / NT;
             const int rows = a.block_map[3 * b + 2];
-            const int N = mma_n(rows);
-            const uint32_t idesc = make_idesc_bf16(128 * C::kCtas, N);
+            const int N = (rows + 15) & ~15;
+            const uint32_t idesc = make_idesc_bf16(128, N);
             const int buf = ucount % C::kAccBufs;
             const uint32_t use = ucount / C::kAccBufs;
-            const bool acc_ok = kPair ? warp_wait_cluster(accempty(buf), (use & 1) ^ 1, abort_flag)
-                                      : warp_wait(accempty(buf), (use & 1) ^ 1, abort_flag);
-            if (!acc_ok) {
+            if (!warp_wait(accempty(buf), (use & 1) ^ 1, abort_flag)) {
                 fail(2);
                 ok = false;
                 break;
@@ -377,14 +252,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             for (int c = 0; c < KC; ++c, ++it) {
                 const int sa = it % C::kNA;
                 const int sb = it % C::kNB;
-                if (!ready) {
-                    const bool aok = kPair ? warp_wait_cluster(afull(sa), (it / C::kNA) & 1, abort_flag)
-                                           : warp_wait(afull(sa), (it / C::kNA) & 1, abort_flag);
-                    if (!aok || !warp_wait(bfull(sb), (it / C::kNB) & 1, abort_flag)) {
-                        fail(3);
-                        ok = false;
-                        break;
-                    }
+                if (!ready && (!warp_wait(afull(sa), (it / C::kNA) & 1, abort_flag) ||
+                               !warp_wait(bfull(sb), (it / C::kNB) & 1, abort_flag))) {
+                    fail(3);
+                    ok = false;
+                    break;
                 }
                 // order the asynchronous MMAs after the waits (the transform
                 // warps fence their generic-proxy stores to A before arriving;
@@ -398,7 +270,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 const uint32_t ra = mbar_test(afull(nx % C::kNA), (nx / C::kNA) & 1);
                 const uint32_t rb = mbar_test(bfull(nx % C::kNB), (nx / C::kNB) & 1);
                 const uint32_t abase = sbase + C::kOffA + sa * C::kAStageBytes;
-                const uint64_t db = make_sw128_desc(sbase + C::kOffB + sb * C::kBStageBytes);
+                const uint64_t db = make_sw128_desc(sbase + C::kOffB + sb * kBStageBytes);
                 uint64_t da[C::kTiles];
 #pragma unroll
                 for (int t = 0; t < C::kTiles; ++t) da[t] = make_sw128_desc(abase + t * kATileBytes);
@@ -407,56 +279,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     for (int kk = 0; kk < kKChunk / 16; ++kk) {
                         const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
-                        for (int t = 0; t < C::kTiles; ++t) {
-                            if constexpr (kPair)
-                                mma_bf16_pair(dacc + t * kBlockT, da[t] + 2 * kk, db + 2 * kk, idesc, acc);
-                            else
-                                mma_bf16(dacc + t * kBlockT, da[t] + 2 * kk, db + 2 * kk, idesc, acc);
-                        }
+                        for (int t = 0; t < C::kTiles; ++t)
+                            mma_bf16(dacc + t * kBlockT, da[t] + 2 * kk, db + 2 * kk, idesc, acc);
                     }
-                    if constexpr (kPair) {
-                        mma_commit_pair(aempty(sa));
-                        mma_commit_pair(bempty(sb));
-                    } else {
-                        mma_commit(aempty(sa));
-                        mma_commit(bempty(sb));
-                    }
+                    mma_commit(aempty(sa));
+                    mma_commit(bempty(sb));
                 }
-                issued = true;
-                // with a pair a barrier test sees only this CTA's arrivals:
-                // wait on the cluster scope every stage
-                ready = !kPair && __all_sync(0xffffffffu, (ra & rb) != 0);
+                ready = __all_sync(0xffffffffu, (ra & rb) != 0);
             }
-            if (ok && elect_one()) {
-                if constexpr (kPair)
-                    mma_commit_pair(accfull(buf));
-                else
-                    mma_commit(accfull(buf));
-            }
+            if (ok && elect_one()) mma_commit(accfull(buf));
             __syncwarp();
         }
-        if (!ok && issued) {
-            if (elect_one()) {
-                if constexpr (kPair)
-                    mma_commit_pair_local(drain_bar);
-                else
-                    mma_commit(drain_bar);
-            }
+        if (!ok) {
+            if (elect_one()) mma_commit(drain_bar);
             __syncwarp();
             mbar_wait_drain(drain_bar, 0);
         }
     } else if (warp == kWarpLoader) {
-        // one 2-D TMA tile of token rows per stage (rows past the block belong
-        // to the next expert or lie past the end and are zero-filled; the MMA
-        // ignores columns >= N and the epilogue columns >= rows).  With a pair
-        // each CTA loads its half of the N columns: the first CTA rows
-        // row0 .. row0 + N/2 - 1, the second from row0 + N/2; both tiles count
-        // on the first CTA's barrier, whose expected bytes that CTA sets.
+        // one 2-D TMA tile of kBlockT token rows per stage (rows past the block
+        // belong to the next expert or lie past the end and are zero-filled;
+        // the MMA ignores columns >= N and the epilogue columns >= rows)
         uint32_t it = 0;
         bool ok = true;
-        for (int u = cta_id; ok && u < num_units; u += n_ctas) {
-            const int b = u / NU;
-            const int row0 = a.block_map[3 * b + 1] + static_cast<int>(rank) * (mma_n(a.block_map[3 * b + 2]) / 2);
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            const int row0 = a.block_map[3 * (u / NT) + 1];
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNB;
                 if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
@@ -465,20 +311,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     break;
                 }
                 if (elect_one()) {
-                    if constexpr (kPair) {
-                        if (rank == 0) mbar_arrive_expect_tx(bfull(s), 2 * C::kBStageBytes);
-                        tma_load_2d_pair(sbase + C::kOffB + s * C::kBStageBytes, &a.bmap, c * kKChunk, row0,
-                                         lead(bfull(s)));
-                    } else {
-                        mbar_arrive_expect_tx(bfull(s), C::kBStageBytes);
-                        tma_load_2d(sbase + C::kOffB + s * C::kBStageBytes, &a.bmap, c * kKChunk, row0,
-                                    bfull(s));
-                    }
+                    mbar_arrive_expect_tx(bfull(s), kBStageBytes);
+                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
                 }
                 __syncwarp();
             }
         }
-        if (!ok && lane == 0 && (!kPair || rank == 0)) {
+        if (!ok && lane == 0) {
             const uint32_t first = it > C::kNB ? it - C::kNB : 0;
             for (uint32_t i = first; i < it; ++i)
                 mbar_wait_drain(bfull(i % C::kNB), (i / C::kNB) & 1);
@@ -492,7 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         const int gpc = kKChunk / a.group;
         uint32_t it = 0;
         bool ok = true;
-        for (int u = cta_id; ok && u < num_units; u += n_ctas) {
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
             for (int c = 0; c < KC; ++c, ++it) {
                 if (static_cast<int>(it % C::kGroups) != grp) continue;
                 const int sw = it % C::kNW;
@@ -536,10 +375,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    if constexpr (kPair)
-                        mbar_arrive_cluster(lead(afull(sa)));
-                    else
-                        mbar_arrive(afull(sa));
+                    mbar_arrive(afull(sa));
                     mbar_arrive(wempty(sw));
                 }
             }
@@ -558,9 +394,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         // feature octet (16 bytes), row c = lane % 8 the token within a group of 8
         const uint32_t st_addr = stg + (lane & 7) * kEpiRowBytes + (lane >> 3) * 16;
         uint32_t ucount = 0;
-        for (int u = cta_id; u < num_units; u += n_ctas, ++ucount) {
-            const int b = u / NU;
-            const int j = (u - b * NU) * C::kCtas + static_cast<int>(rank);
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++ucount) {
+            const int b = u / NT;
+            const int j = u - b * NT;
             const int row0 = a.block_map[3 * b + 1];
             const int rows = a.block_map[3 * b + 2];
             const int ncb = (rows + 31) >> 5;
@@ -574,16 +410,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             // gate/up: one output tile (gate at column 0, up at kBlockT); down:
             // kTiles output tiles of 128 features at columns t * kBlockT
             constexpr int kOutTiles = kDown ? C::kTiles : 1;
-            auto hand_back = [&]() {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if constexpr (kPair)
-                        mbar_arrive_cluster(lead(accempty(buf)));
-                    else
-                        mbar_arrive(accempty(buf));
-                }
-            };
 #pragma unroll 1
             for (int it = 0; it < kOutTiles * ncb; ++it) {
                 const int t = it / ncb;
@@ -634,9 +460,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                             p[h][i] = o.u;
                         }
                 }
-                // every TMEM read of this unit has completed: hand the
-                // accumulator back to the MMA warp before the last stores
-                if (it == kOutTiles * ncb - 1) hand_back();
+                if (it == kOutTiles * ncb - 1) {
+                    // every TMEM read of this unit has completed: hand the
+                    // accumulator back to the MMA warp before the last stores
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(accempty(buf));
+                }
                 // token group g (8 tokens): matrices (h, octet) = registers
                 // p[h][2g] (features 16h + 0..7) and p[h][2g+1] (16h + 8..15)
 #pragma unroll
@@ -657,21 +487,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 }
                 __syncwarp();
             }
-            if (ncb == 0) hand_back();  // a block always has rows; keep the hand-back unconditional
+            if (ncb == 0) {  // a block always has rows; keep the hand-back unconditional
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accempty(buf));
+            }
         }
     }
 
-    tc_fence_before();
-    if constexpr (kPair)
-        cluster_sync_all();  // both CTAs are done with the pair's TMEM and barriers
-    else
-        __syncthreads();
+    __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
-        if constexpr (kPair)
-            tmem_dealloc_pair(tmem, kTmemCols);
-        else
-            tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -728,17 +555,12 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
-    cudaError_t e;
-#define MOE_SET_SMEM(D, P)                                                                     \
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             Cfg<D, P>::kSmemBytes);                                           \
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<false>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    MOE_SET_SMEM(false, false)
-    MOE_SET_SMEM(true, false)
-    MOE_SET_SMEM(false, true)
-    MOE_SET_SMEM(true, true)
-#undef MOE_SET_SMEM
-    return cudaSuccess;
+    return cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<true>::kSmemBytes);
 }
 
 static cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
@@ -828,39 +650,16 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
     return cudaGetLastError();
 }
 
-template <bool kDown, bool kPair>
-static cudaError_t launch_gemm_t(const GemmArgs& a, int num_sms, cudaStream_t st) {
-    // Plain launches: letting the next kernel's CTAs be scheduled early measured
-    // slower around the GEMMs (their pdl_wait then returns at once).
-    if constexpr (kPair) {
-        const int pairs = std::min(a.max_units, num_sms / 2);
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * pairs);
-        cfg.blockDim = dim3(kGemmThreads);
-        cfg.dynamicSmemBytes = Cfg<kDown, kPair>::kSmemBytes;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kDown, kPair>, a);
-    } else {
-        const int grid = a.max_units < num_sms ? a.max_units : num_sms;
-        grouped_gemm_kernel<kDown, kPair><<<grid, kGemmThreads, Cfg<kDown, kPair>::kSmemBytes, st>>>(a);
-        return cudaGetLastError();
-    }
-}
-
 static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaStream_t st) {
     if (a.max_units <= 0) return cudaSuccess;
-    // a pair of CTAs shares each MMA when the projection has an even number of
-    // 128-row output tiles (max_units then counts pair units)
-    const bool pair = a.pair;
-    if (down) return pair ? launch_gemm_t<true, true>(a, num_sms, st) : launch_gemm_t<true, false>(a, num_sms, st);
-    return pair ? launch_gemm_t<false, true>(a, num_sms, st) : launch_gemm_t<false, false>(a, num_sms, st);
+    const int grid = a.max_units < num_sms ? a.max_units : num_sms;
+    // Plain launches: letting the next kernel's CTAs be scheduled early measured
+    // slower around the GEMMs (their pdl_wait then returns at once).
+    if (down)
+        grouped_gemm_kernel<true><<<grid, kGemmThreads, Cfg<true>::kSmemBytes, st>>>(a);
+    else
+        grouped_gemm_kernel<false><<<grid, kGemmThreads, Cfg<false>::kSmemBytes, st>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st) {

@@ -121,7 +121,7 @@ struct GemmArgs {
     // B operand (token rows in expert order) for 2-D TMA tiles of 64 columns x
     // kBlockT rows with the 128-byte swizzle, the K-major layout the MMA
     // reads: gate/up reads xs [T*k, d], down reads h [T*k, f].
-    CUtensorMap bmap;              // box rows: kBlockT, or kBlockT / 2 with a pair of CTAs
+    CUtensorMap bmap;
     const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
     const int32_t* block_map;      // [num_blocks, 3]
     const int32_t* num_blocks;     // [1], device
@@ -132,8 +132,7 @@ struct GemmArgs {
     int out_ld;                    // f (gate/up) or d (down)
     int group;
     int block_bytes;
-    int max_units;                 // upper bound of num_blocks * NT (pair: num_blocks * NT / 2)
-    int pair;                      // a pair of CTAs shares each MMA (NT even)
+    int max_units;                 // upper bound of num_blocks * NT
 };
 // Encode the tensor map of a row-major fp32 matrix [rows, cols] read in boxes
 // of box_cols columns x box_rows rows, unswizzled.

@@ -1,5 +1,4 @@
-"""Host-side model of the grouped GEMM's mbarrier protocol (one CTA, or a
-pair of CTAs sharing each MMA).
+"""Host-side model of the grouped GEMM's mbarrier protocol (one CTA).
 
 The persistent GEMM kernel runs five roles that hand ring stages to each other
 through mbarriers: the packed-weight producer (W ring), the token-tile loader
@@ -13,12 +12,6 @@ count and accumulator buffers read from the kernel source, and checks that
   - every stage read sees the iteration its consumer expects (no role is
     released by a parity wait one phase too early: mbarrier parity waits only
     tell a phase from the one before it).
-
-With a pair of CTAs (cta_group::2) each CTA runs its own weight producer,
-token loader, transform and epilogue warps; the first CTA's MMA warp waits on
-its A barrier for both CTAs' transform warps, on its B barrier for both CTAs'
-token tiles and on its accumulator barrier for both CTAs' epilogue warps, and
-its commits arrive on the A, B and accumulator barriers of both CTAs.
 
 A configuration that breaks the kernel's static_assert (ring sizes that are
 not multiples of the transform group count) is shown to fail the model.
@@ -39,8 +32,7 @@ EPILOGUE_WARPS = 4
 
 
 def kernel_configs():
-    """(name, NW, NA, NB, G, acc_bufs, ctas) of the two projections, one CTA
-    and a pair of CTAs, from the source."""
+    """(name, NW, NA, NB, G, acc_bufs) of the two projections, from the source."""
     src = open(GEMM_SRC).read()
     down_tiles = int(re.search(r"constexpr int kDownTiles = (\d+);", open(INTERNAL_H).read()).group(1))
 
@@ -49,22 +41,14 @@ def kernel_configs():
         assert m, name
         return int(m.group(1)), int(m.group(2))
 
-    nw, acc, g = pick("kNW"), pick("kAccBufs"), pick("kGroups")
-    m = re.search(r"static constexpr int kNA = kOneTile \? (\d+) : \(kPair \? (\d+) : (\d+)\);", src)
-    assert m, "kNA"
-    na_one, na_two_pair, na_two = (int(v) for v in m.groups())
-    m = re.search(r"static constexpr int kNB = kPair \? \(kOneTile \? (\d+) : (\d+)\) : (\d+);", src)
-    assert m, "kNB"
-    nb_pair_one, nb_pair_two, nb_single = (int(v) for v in m.groups())
-    # gate/up always has two weight tiles per unit, down has kDownTiles
+    nw, na, acc, g = pick("kNW"), pick("kNA"), pick("kAccBufs"), pick("kGroups")
+    nb = int(re.search(r"static constexpr int kNB = (\d+);", src).group(1))
+    # each pair is (value with one weight tile per unit, value with two);
+    # gate/up always has two tiles, down has kDownTiles
+    gu = ("gate/up", nw[1], na[1], nb, g[1], acc[1])
     i = 0 if down_tiles == 1 else 1
-    na = (na_one, na_two)
-    na_pair = (na_one, na_two_pair)
-    nb_pair = (nb_pair_one, nb_pair_two)
-    return [("gate/up", nw[1], na[1], nb_single, g[1], acc[1], 1),
-            ("down", nw[i], na[i], nb_single, g[i], acc[i], 1),
-            ("gate/up, pair", nw[1], na_pair[1], nb_pair[1], g[1], acc[1], 2),
-            ("down, pair", nw[i], na_pair[i], nb_pair[i], g[i], acc[i], 2)]
+    dn = ("down", nw[i], na[i], nb, g[i], acc[i])
+    return [gu, dn]
 
 
 class Barrier:
@@ -83,23 +67,19 @@ class Barrier:
         return (self.phase & 1) != parity
 
 
-def simulate(NW, NA, NB, G, acc_bufs, units=5, KC=7, seed=0, ctas=1):
+def simulate(NW, NA, NB, G, acc_bufs, units=5, KC=7, seed=0):
     """Returns (finished, races): finished is False on a deadlock."""
     rng = random.Random(seed)
-    C = range(ctas)
-    wfull = [[Barrier(1) for _ in range(NW)] for _ in C]
-    wempty = [[Barrier(TRANSFORM_WARPS // G) for _ in range(NW)] for _ in C]
-    aempty = [[Barrier(1) for _ in range(NA)] for _ in C]
-    bempty = [[Barrier(1) for _ in range(NB)] for _ in C]
-    accfull = [[Barrier(1) for _ in range(acc_bufs)] for _ in C]
-    # the MMA issuer's barriers count both CTAs' arrivals
-    afull = [Barrier(ctas * TRANSFORM_WARPS // G) for _ in range(NA)]
-    bfull = [Barrier(ctas) for _ in range(NB)]
-    accempty = [Barrier(ctas * EPILOGUE_WARPS) for _ in range(acc_bufs)]
-    # iteration held by each stage of each CTA (what a reader must find there)
-    w_slot = [[None] * NW for _ in C]
-    a_slot = [[None] * NA for _ in C]
-    b_slot = [[None] * NB for _ in C]
+    wfull = [Barrier(1) for _ in range(NW)]
+    wempty = [Barrier(TRANSFORM_WARPS // G) for _ in range(NW)]
+    afull = [Barrier(TRANSFORM_WARPS // G) for _ in range(NA)]
+    aempty = [Barrier(1) for _ in range(NA)]
+    bfull = [Barrier(1) for _ in range(NB)]
+    bempty = [Barrier(1) for _ in range(NB)]
+    accfull = [Barrier(1) for _ in range(acc_bufs)]
+    accempty = [Barrier(EPILOGUE_WARPS) for _ in range(acc_bufs)]
+    # iteration held by each stage (what a reader must find there)
+    w_slot, a_slot, b_slot = [None] * NW, [None] * NA, [None] * NB
     races = []
     clock = [0.0]
     queue, seq = [], [0]
@@ -109,40 +89,40 @@ def simulate(NW, NA, NB, G, acc_bufs, units=5, KC=7, seed=0, ctas=1):
         seq[0] += 1
         heapq.heappush(queue, (clock[0] + delay, seq[0], fn))
 
-    def w_producer(c):
+    def w_producer():
         for it in range(total):
             s = it % NW
-            yield wempty[c][s], ((it // NW) & 1) ^ 1
+            yield wempty[s], ((it // NW) & 1) ^ 1
 
             def land(s=s, it=it):
-                w_slot[c][s] = it
-                wfull[c][s].arrive()
+                w_slot[s] = it
+                wfull[s].arrive()
             later(rng.uniform(1, 30), land)
 
-    def b_loader(c):
+    def b_loader():
         for it in range(total):
             s = it % NB
-            yield bempty[c][s], ((it // NB) & 1) ^ 1
+            yield bempty[s], ((it // NB) & 1) ^ 1
 
             def land(s=s, it=it):
-                b_slot[c][s] = it
+                b_slot[s] = it
                 bfull[s].arrive()
             later(rng.uniform(1, 30), land)
 
-    def transform_warp(c, group, member):
+    def transform_warp(group, member):
         for it in range(total):
             if it % G != group:
                 continue
             sw, sa = it % NW, it % NA
-            yield wfull[c][sw], (it // NW) & 1
-            yield aempty[c][sa], ((it // NA) & 1) ^ 1
-            if w_slot[c][sw] != it:
-                races.append(("transform reads W", c, it, w_slot[c][sw]))
+            yield wfull[sw], (it // NW) & 1
+            yield aempty[sa], ((it // NA) & 1) ^ 1
+            if w_slot[sw] != it:
+                races.append(("transform reads W", it, w_slot[sw]))
             yield None, rng.uniform(1, 10)  # expanding
             if member == 0:
-                a_slot[c][sa] = it
+                a_slot[sa] = it
             afull[sa].arrive()
-            wempty[c][sw].arrive()
+            wempty[sw].arrive()
 
     def mma():
         it = 0
@@ -153,32 +133,26 @@ def simulate(NW, NA, NB, G, acc_bufs, units=5, KC=7, seed=0, ctas=1):
                 sa, sb = it % NA, it % NB
                 yield afull[sa], (it // NA) & 1
                 yield bfull[sb], (it // NB) & 1
-                for c in C:
-                    if a_slot[c][sa] != it:
-                        races.append(("MMA reads A", c, it, a_slot[c][sa]))
-                    if b_slot[c][sb] != it:
-                        races.append(("MMA reads B", c, it, b_slot[c][sb]))
+                if a_slot[sa] != it:
+                    races.append(("MMA reads A", it, a_slot[sa]))
+                if b_slot[sb] != it:
+                    races.append(("MMA reads B", it, b_slot[sb]))
                 done = rng.uniform(1, 8)  # the commits fire when the MMAs complete
-                for c in C:
-                    later(done, lambda c=c, sa=sa: aempty[c][sa].arrive())
-                    later(done, lambda c=c, sb=sb: bempty[c][sb].arrive())
+                later(done, lambda sa=sa: aempty[sa].arrive())
+                later(done, lambda sb=sb: bempty[sb].arrive())
                 it += 1
-            fin = rng.uniform(1, 8)
-            for c in C:
-                later(fin, lambda c=c, buf=buf: accfull[c][buf].arrive())
+            later(rng.uniform(1, 8), lambda buf=buf: accfull[buf].arrive())
 
-    def epilogue_warp(c):
+    def epilogue_warp():
         for u in range(units):
             buf, use = u % acc_bufs, u // acc_bufs
-            yield accfull[c][buf], use & 1
+            yield accfull[buf], use & 1
             yield None, rng.uniform(1, 40)
             accempty[buf].arrive()
 
-    roles = [mma()]
-    for c in C:
-        roles += [w_producer(c), b_loader(c)]
-        roles += [transform_warp(c, g, m) for g in range(G) for m in range(TRANSFORM_WARPS // G)]
-        roles += [epilogue_warp(c) for _ in range(EPILOGUE_WARPS)]
+    roles = [w_producer(), b_loader(), mma()]
+    roles += [transform_warp(g, m) for g in range(G) for m in range(TRANSFORM_WARPS // G)]
+    roles += [epilogue_warp() for _ in range(EPILOGUE_WARPS)]
     blocked = {}
     finished = [0]
 
@@ -217,10 +191,10 @@ def simulate(NW, NA, NB, G, acc_bufs, units=5, KC=7, seed=0, ctas=1):
 
 @pytest.mark.parametrize("cfg", kernel_configs(), ids=lambda c: c[0])
 def test_kernel_ring_configuration_is_sound(cfg):
-    name, NW, NA, NB, G, acc, ctas = cfg
+    name, NW, NA, NB, G, acc = cfg
     assert NW % G == 0 and NA % G == 0, "the kernel's static_assert"
     for seed in range(150):
-        finished, races = simulate(NW, NA, NB, G, acc, seed=seed, ctas=ctas)
+        finished, races = simulate(NW, NA, NB, G, acc, seed=seed)
         assert finished, (name, "deadlock", seed)
         assert not races, (name, races[:3], seed)
 
