@@ -72,8 +72,19 @@ typedef struct moe_shape {
     int32_t k;     /* experts per token                                    */
     int32_t f;     /* expert intermediate size                             */
     int32_t group; /* int4 group size along the reduction dimension        */
-    uint32_t flags;/* must be 0                                            */
+    uint32_t flags;/* 0, or MOE_SHAPE_TEST_TIMEOUT                         */
 } moe_shape_t;
+
+/*
+ * Test hook, not for production plans: in moe_forward's batched path the
+ * gate/up grouped GEMM's weight producer withholds its first copy and every
+ * wait of that kernel gives up after 5 ms, so the call records
+ * MOE_ERR_DEVICE_TIMEOUT (detail 101..106: the role that gave up) in the
+ * workspace status word instead of a result.  It exercises the bounded-wait
+ * and abort path without faulting or hanging the GPU; the workspace stays
+ * usable for the next call.
+ */
+#define MOE_SHAPE_TEST_TIMEOUT 1u
 
 typedef struct moe_plan moe_plan_t;
 

@@ -29,6 +29,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 MOE_OK = 0
+SHAPE_TEST_TIMEOUT = 1  # MOE_SHAPE_TEST_TIMEOUT: test hook of the bounded-wait path
 STATUS_NAMES = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
     3: "MOE_ERR_ALIGNMENT", 4: "MOE_ERR_WORKSPACE_TOO_SMALL", 5: "MOE_ERR_CUDA",
@@ -144,8 +145,8 @@ def _check(code: int, where: str):
 class Plan:
     """moe_plan_create for one layer shape (host only, touches no GPU)."""
 
-    def __init__(self, T_max: int, d: int, E: int, k: int, f: int, group: int):
-        self.shape = Shape(T_max, d, E, k, f, group, 0)
+    def __init__(self, T_max: int, d: int, E: int, k: int, f: int, group: int, flags: int = 0):
+        self.shape = Shape(T_max, d, E, k, f, group, flags)
         self._h = _P()
         self.info = PlanInfo()
         _check(_lib.moe_plan_create(ctypes.byref(self.shape), ctypes.byref(self._h),

@@ -22,7 +22,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status_t check_shape(const moe_shape_t& s) {
-    if (s.flags != 0) return MOE_ERR_INVALID_ARG;
+    if ((s.flags & ~static_cast<uint32_t>(MOE_SHAPE_TEST_TIMEOUT)) != 0) return MOE_ERR_INVALID_ARG;
     if (s.T_max <= 0 || s.d <= 0 || s.E <= 0 || s.k <= 0 || s.f <= 0) return MOE_ERR_INVALID_ARG;
     if (s.k > s.E) return MOE_ERR_INVALID_ARG;
     if (s.group != 32 && s.group != 64) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -360,6 +360,11 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.group = s.group;
     g.block_bytes = plan->group_bytes;
     g.max_units = mb * g.NT;
+    // test hook (MOE_SHAPE_TEST_TIMEOUT): the gate/up GEMM withholds a stage and
+    // its waits give up after 5 ms
+    const bool test_timeout = (s.flags & MOE_SHAPE_TEST_TIMEOUT) != 0;
+    g.withhold_first = test_timeout ? 1 : 0;
+    g.wait_ns = test_timeout ? 5000000ull : moe::kWaitTimeoutNs;
     MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
     if (ev && !mark(ev->gate_up)) return MOE_ERR_CUDA;
@@ -372,6 +377,8 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.out_ld = s.d;
     g.block_bytes = plan->down_block_bytes;
     g.max_units = mb * g.NT;
+    g.withhold_first = 0;
+    g.wait_ns = moe::kWaitTimeoutNs;
     MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT));
     MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;

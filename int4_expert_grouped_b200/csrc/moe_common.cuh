@@ -82,17 +82,18 @@ __device__ __forceinline__ uint32_t mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase of `parity` has completed.  Returns false if the
-// CTA's abort flag is raised or the wait exceeds kWaitTimeoutNs; the caller
-// then stops its role.  `abort_flag` lives in shared memory.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort_flag) {
+// CTA's abort flag is raised or the wait exceeds `limit_ns` (kWaitTimeoutNs
+// unless a test shortens it); the caller then stops its role.  `abort_flag`
+// lives in shared memory.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((n & 63u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+            if (globaltimer() - t0 > limit_ns) return false;
         }
     }
 }

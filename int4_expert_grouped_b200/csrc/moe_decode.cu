@@ -27,7 +27,10 @@
 //                       each unit's weights into a shared-memory ring with
 //                       bulk copies, as far ahead as the ring allows, so every
 //                       SM keeps its share of the weights in flight; eight
-//                       warps multiply them on the warp-level tensor-core MMA.
+//                       warps multiply them on the warp-level tensor-core MMA,
+//                       each warp a share of the K chunks (gate/up) or of the
+//                       output tiles (down) with all of the slice's rows, so
+//                       its eight row tiles are independent chains.
 //                       SwiGLU of the slice stays in shared memory (no h round
 //                       trip); the slice's down partial sums go to the
 //                       workspace
@@ -62,7 +65,7 @@ constexpr int kDecComputeWarps = 8;
 constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;  // + one producer warp
 constexpr int kDecProducerWarp = kDecComputeWarps;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
-constexpr int kDecStages = 32;
+constexpr int kDecStages = 24;
 // One stage = one 64-wide K chunk of a slice's 64 gate and 64 up rows
 // (nibbles, then scale/bias words), or one down block (128 rows x 64 K):
 // both 4096 + 512 * (64 / group) bytes.
@@ -72,6 +75,8 @@ constexpr int kDecSlice = 64;                              // features per unit
 constexpr int kDecMaxSlices = 32;                          // f / 64
 constexpr int kDecMaxNTd = 64;                             // d / 128
 constexpr int kDecHStride = kDecSlice + 32;                // h row stride (elements) in shared memory
+constexpr int kDecRowTiles = kDecSlice / 8;                // 16-row MMA tiles of a slice: 8 gate + 8 up rows each
+static_assert(kDecStages % kDecComputeWarps == 0, "a ring slot is always used by the same compute warp");
 constexpr int kDecWRows = 256;                             // W_r rows per tensor load (box limit)
 constexpr uint32_t kDecMagic0 = 0x4D6F4544u, kDecMagic1 = 0x53796E63u;
 
@@ -263,7 +268,6 @@ __device__ __forceinline__ void stage_rows(uint16_t* dst, float* sums, const uin
 
 // Routing of the few tokens, in shared memory (identical in every CTA).
 struct DecRoute {
-    float sel[kDecMaxAssign];  // logit of each selected slot
     int idx[kDecMaxAssign];
     float w[kDecMaxAssign];
     int sa[kDecMaxAssign];
@@ -282,31 +286,27 @@ struct DecRoute {
     int abort_local;           // this CTA gave up
 };
 
-// top-k (each (token, expert) pair finds its slot; ties go to the lower id),
-// the softmax weights over the k slots, counts (integer atomics), offsets
-// (exclusive scan), one block per expert with rows (ascending expert), and
-// the stable scatter (rank of assignment a = number of earlier assignments
-// to its expert).  All kDecThreads threads.
+// top-k per token by one warp (ties go to the lower id) with the softmax
+// weights over the k slots, counts (integer atomics), offsets (exclusive
+// scan), one block per expert with rows (ascending expert), and the stable
+// scatter (rank of assignment a = number of earlier assignments to its
+// expert).  All kDecThreads threads.
 __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int Tk = T * k;
     if (tid < E) R.cnt[tid] = 0;
-    for (int it = tid; it < T * E; it += kDecThreads) {
-        const int t = it / E;
-        const int e = it - t * E;
-        const int slot = expert_slot(lg + t * E, E, e);
-        if (slot < k) {
-            R.idx[t * k + slot] = e;
-            R.sel[t * k + slot] = lg[it];
+    for (int t = warp; t < T; t += kDecThreads / 32) {
+        int id;
+        float wt;
+        warp_topk(lg + t * E, E, k, lane, id, wt);
+        if (lane < k) {
+            R.idx[t * k + lane] = id;
+            R.w[t * k + lane] = wt;
         }
     }
     __syncthreads();
-    for (int t = warp; t < T; t += kDecThreads / 32) {
-        const float wt = warp_slot_weights(lane < k ? R.sel[t * k + lane] : 0.0f, k, lane);
-        if (lane < k) R.w[t * k + lane] = wt;
-    }
     for (int a = tid; a < Tk; a += kDecThreads) atomicAdd(&R.cnt[R.idx[a]], 1);
     __syncthreads();
     const int c = tid < E ? R.cnt[tid] : 0;
@@ -344,7 +344,7 @@ __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
 
 // Layout of the dynamic shared memory (byte offsets; the base is 1024-aligned).
 struct DecSmem {
-    int ring, x, xsum, h, hsum, lg, route, bars, total;
+    int ring, x, xsum, h, hsum, lg, red, route, bars, total;
 };
 __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     DecSmem L;
@@ -360,6 +360,7 @@ __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     L.h = take(kDecodeMaxT * kDecHStride * 2);
     L.hsum = take(kDecodeMaxT * (kDecSlice / 32) * 4);
     L.lg = take(T * E * 4);
+    L.red = take(kDecComputeWarps * kDecRowTiles * 4 * 32 * 4);  // per-warp gate/up partial sums
     L.route = take(static_cast<int>(sizeof(DecRoute)));
     L.bars = take((2 * kDecStages + 1) * 8);
     L.total = o + 1024;  // + slack to align the base
@@ -457,7 +458,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     if (tid == 0) {
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(empty(s), kDecComputeWarps);
+            mbar_init(empty(s), 1);  // one compute warp uses each stage
         }
         mbar_init(wbar, 1);
         R.abort_local = 0;
@@ -645,6 +646,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
         // compute warps: MMA fragment coordinates
         const int g = lane >> 2;
         const int c = lane & 3;
+        float* red = reinterpret_cast<float*>(smem + L.red);
         uint32_t q = 0;
         const int nvd = d / 32;
         for (int u = cta; u < u_total; u += G) {
@@ -654,43 +656,71 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int n = R.blk_n[b];
             if (tid == 0) R.fail = 0;
             compute_sync();  // also: every warp is done with the previous unit's h rows
-            // gate/up: warp w takes features 8w .. 8w + 7 of the slice; the MMA
-            // tile's rows g and g + 8 are the gate and the up row of feature 8w + g
+            // Stage q of the call is used by compute warp q % 8, so the warp that
+            // waits on a ring slot's phase has itself used the slot's previous
+            // phase (a parity wait only tells a phase from the one before it).
+            // gate/up: warp w takes the K chunks whose stage is w mod 8; MMA tile
+            // r has the gate rows of features 8r .. 8r + 7 as rows g and the up
+            // rows as g + 8
             const int cg = min(g, n - 1), c0 = min(2 * c, n - 1), c1 = min(2 * c + 1, n - 1);
             const uint16_t* brow = xsh + (R.sa[row0 + cg] / k) * (d + 32) + 8 * c;
             const float* bs0 = xsum + (R.sa[row0 + c0] / k) * nvd;
             const float* bs1 = xsum + (R.sa[row0 + c1] / k) * nvd;
-            const int fr = 8 * warp + g;  // row of the slice
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            for (int st = 0; st < KC; ++st, ++q) {
-                const int slot = q % kDecStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
+            float acc[kDecRowTiles][4];
+#pragma unroll
+            for (int r = 0; r < kDecRowTiles; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
+            for (int st = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
+                 st < KC; st += kDecComputeWarps) {
+                const uint32_t qs = q + st;
+                const int slot = qs % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (qs / kDecStages) & 1, &R.abort_local))) {
                     if (lane == 0) {
                         R.fail = 1;
                         if (!vload(R.abort_local)) dec_fail(p, R, 505);
                     }
-                    continue;
+                    break;
                 }
                 const uint8_t* stage = ring + slot * kDecStageBytes;
-                chunk_mma_rows<kGpc>(acc, stage + fr * 32, stage + (kDecSlice + fr) * 32,
-                                     stage + 2 * kDecSlice * 32 + fr * kGpc * 4,
-                                     stage + 2 * kDecSlice * 32 + sc_bytes + fr * kGpc * 4, c,
-                                     brow + kKChunk * st, bs0 + 2 * st, bs1 + 2 * st);
+#pragma unroll
+                for (int r = 0; r < kDecRowTiles; ++r) {
+                    const int fr = 8 * r + g;
+                    chunk_mma_rows<kGpc>(acc[r], stage + fr * 32, stage + (kDecSlice + fr) * 32,
+                                         stage + 2 * kDecSlice * 32 + fr * kGpc * 4,
+                                         stage + 2 * kDecSlice * 32 + sc_bytes + fr * kGpc * 4, c,
+                                         brow + kKChunk * st, bs0 + 2 * st, bs1 + 2 * st);
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(slot));
             }
-            // SwiGLU of the slice, rounded to bf16, into shared memory [token][64]
+            q += KC;
+            // partial sums of every warp -> shared memory, added in warp order
 #pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-                const int col = 2 * c + e2;
-                if (col < n) {
-                    const float gv = acc[e2];
-                    const float uv = acc[2 + e2];
-                    hsh[col * kDecHStride + fr] = bf16_round_bits(__fdividef(gv * uv, 1.0f + __expf(-gv)));
+            for (int r = 0; r < kDecRowTiles; ++r)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) red[((warp * kDecRowTiles + r) * 4 + i) * 32 + lane] = acc[r][i];
+            compute_sync();
+            if (vload(R.fail)) break;
+            // SwiGLU of the slice, rounded to bf16, into shared memory [token][64]:
+            // thread (r, lane) of warp r finishes MMA tile r
+            {
+                const int r = warp;
+                float sum[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float v = red[((0 * kDecRowTiles + r) * 4 + i) * 32 + lane];
+                    for (int w = 1; w < kDecComputeWarps; ++w) v += red[((w * kDecRowTiles + r) * 4 + i) * 32 + lane];
+                    sum[i] = v;
+                }
+                const int fr = 8 * r + g;
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int col = 2 * c + e2;
+                    if (col < n)
+                        hsh[col * kDecHStride + fr] =
+                            bf16_round_bits(__fdividef(sum[e2] * sum[2 + e2], 1.0f + __expf(-sum[e2])));
                 }
             }
             compute_sync();
-            if (vload(R.fail)) break;
             // the 32-wide vector sums of the h rows (K order), for the group folds
             if (tid < 2 * n) {
                 const int col = tid >> 1, v = tid & 1;
@@ -699,23 +729,29 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 hsum[col * 2 + v] = sacc;
             }
             compute_sync();
-            // down: output tile jd, rows 16w .. 16w + 15 of its 128; K = the slice
+            // down: warp w takes the output tiles whose stage is w mod 8, all 128
+            // rows of each (eight MMA tiles); K = the slice
             const uint16_t* hrow = hsh + cg * kDecHStride + 8 * c;
             const float* hs0 = hsum + c0 * 2;
             const float* hs1 = hsum + c1 * 2;
-            const int ra = 16 * warp + g;
-            for (int jd = 0; jd < NTd; ++jd, ++q) {
-                const int slot = q % kDecStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
+            for (int jd = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
+                 jd < NTd; jd += kDecComputeWarps) {
+                const uint32_t qs = q + jd;
+                const int slot = qs % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (qs / kDecStages) & 1, &R.abort_local))) {
                     if (lane == 0) {
                         R.fail = 1;
                         if (!vload(R.abort_local)) dec_fail(p, R, 506);
                     }
-                    continue;
+                    break;
                 }
                 const uint8_t* stage = ring + slot * kDecStageBytes;
-                float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                chunk_mma<kGpc>(o, stage, 128 * 32, ra, c, hrow, hs0, hs1);
+                float o[kDecRowTiles][4];
+#pragma unroll
+                for (int r = 0; r < kDecRowTiles; ++r) {
+                    o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.0f;
+                    chunk_mma<kGpc>(o[r], stage, 128 * 32, 16 * r + g, c, hrow, hs0, hs1);
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(slot));
 #pragma unroll
@@ -723,11 +759,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     const int col = 2 * c + e2;
                     if (col < n) {
                         float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128;
-                        dst[ra] = o[e2];
-                        dst[ra + 8] = o[2 + e2];
+#pragma unroll
+                        for (int r = 0; r < kDecRowTiles; ++r) {
+                            dst[16 * r + g] = o[r][e2];
+                            dst[16 * r + g + 8] = o[r][2 + e2];
+                        }
                     }
                 }
             }
+            q += NTd;
             compute_sync();
             if (vload(R.fail)) break;
         }

@@ -119,8 +119,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 
 // mbar_wait for a whole converged warp: every lane waits and the outcome is
 // voted, so the warp takes the same branch whatever happens at a timeout.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, limit_ns));
 }
 
 // Wait used only while shutting down after an abort: ignores the abort flag.
@@ -210,11 +211,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNW;
-                if (!warp_wait(wempty(s), ((it / C::kNW) & 1) ^ 1, abort_flag)) {
+                if (!warp_wait(wempty(s), ((it / C::kNW) & 1) ^ 1, abort_flag, a.wait_ns)) {
                     fail(1);
                     ok = false;
                     break;
                 }
+                // test hook: withhold the first stage, so its consumers' waits run out
+                if (a.withhold_first && it == 0) continue;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(wfull(s), a.block_bytes);
                     bulk_copy_g2s(sbase + C::kOffW + s * C::kWStageBytes, src + c * a.block_bytes,
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             // let the copies already issued land before the CTA exits
             const uint32_t first = it > C::kNW ? it - C::kNW : 0;
             for (uint32_t i = first; i < it; ++i)
-                mbar_wait_drain(wfull(i % C::kNW), (i / C::kNW) & 1);
+                if (!(a.withhold_first && i == 0)) mbar_wait_drain(wfull(i % C::kNW), (i / C::kNW) & 1);
         }
     } else if (warp == kWarpMma) {
         // The whole warp runs the issue loop so descriptors and ring indices
@@ -242,7 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const uint32_t idesc = make_idesc_bf16(128, N);
             const int buf = ucount % C::kAccBufs;
             const uint32_t use = ucount / C::kAccBufs;
-            if (!warp_wait(accempty(buf), (use & 1) ^ 1, abort_flag)) {
+            if (!warp_wait(accempty(buf), (use & 1) ^ 1, abort_flag, a.wait_ns)) {
                 fail(2);
                 ok = false;
                 break;
@@ -252,8 +255,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             for (int c = 0; c < KC; ++c, ++it) {
                 const int sa = it % C::kNA;
                 const int sb = it % C::kNB;
-                if (!ready && (!warp_wait(afull(sa), (it / C::kNA) & 1, abort_flag) ||
-                               !warp_wait(bfull(sb), (it / C::kNB) & 1, abort_flag))) {
+                if (!ready && (!warp_wait(afull(sa), (it / C::kNA) & 1, abort_flag, a.wait_ns) ||
+                               !warp_wait(bfull(sb), (it / C::kNB) & 1, abort_flag, a.wait_ns))) {
                     fail(3);
                     ok = false;
                     break;
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int row0 = a.block_map[3 * (u / NT) + 1];
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNB;
-                if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag)) {
+                if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag, a.wait_ns)) {
                     fail(4);
                     ok = false;
                     break;
@@ -336,8 +339,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 if (static_cast<int>(it % C::kGroups) != grp) continue;
                 const int sw = it % C::kNW;
                 const int sa = it % C::kNA;
-                if (!warp_wait(wfull(sw), (it / C::kNW) & 1, abort_flag) ||
-                    !warp_wait(aempty(sa), ((it / C::kNA) & 1) ^ 1, abort_flag)) {
+                if (!warp_wait(wfull(sw), (it / C::kNW) & 1, abort_flag, a.wait_ns) ||
+                    !warp_wait(aempty(sa), ((it / C::kNA) & 1) ^ 1, abort_flag, a.wait_ns)) {
                     fail(5);
                     ok = false;
                     break;
@@ -402,7 +405,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int ncb = (rows + 31) >> 5;
             const int buf = ucount % C::kAccBufs;
             const uint32_t use = ucount / C::kAccBufs;
-            if (!warp_wait(accfull(buf), use & 1, abort_flag)) {
+            if (!warp_wait(accfull(buf), use & 1, abort_flag, a.wait_ns)) {
                 fail(6);
                 break;
             }

@@ -133,6 +133,8 @@ struct GemmArgs {
     int group;
     int block_bytes;
     int max_units;                 // upper bound of num_blocks * NT
+    int withhold_first;            // test hook: the weight producer skips its first copy
+    uint64_t wait_ns;              // limit of every device-side wait
 };
 // Encode the tensor map of a row-major fp32 matrix [rows, cols] read in boxes
 // of box_cols columns x box_rows rows, unswizzled.

@@ -66,8 +66,8 @@ struct ApproxArgs {
 // one expert each (thread t holds rows t, t + 256, ... of the column).
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 256;
-constexpr int kPrepMaxVec = 16;   // 16-byte vectors of a token row per lane: d <= 4096
-constexpr int kPrepMaxRows = 16;  // W_r rows per thread of an expert block: d <= 4096
+constexpr int kPrepMaxVec = 8;    // 16-byte vectors of a token row per lane: d <= 2048
+constexpr int kPrepMaxRows = 8;   // W_r rows per thread of an expert block: d <= 2048
 
 // power of two p with m < 2^span_log2 * p (m > 0); exact
 __device__ __forceinline__ float pow2_scale(float m, int span_log2) {
@@ -79,7 +79,7 @@ __device__ __forceinline__ float pow2_scale(float m, int span_log2) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__global__ void __launch_bounds__(kPrepThreads)
+__global__ void __launch_bounds__(kPrepThreads, 2)
 router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, int T, int d, int E,
                    int nxb, RouterFastWs ws, int32_t* __restrict__ hist, int hist_n,
                    int32_t* __restrict__ status) {
@@ -517,12 +517,13 @@ router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, i
 // Exact logits of the candidate pairs (upper bound >= the token's threshold),
 // in the router's fixed order: lane p runs chain p with fused multiply-add,
 // then the xor butterfly, then the bias.  One CTA per slice of 16 experts
-// (W_r slice in shared memory, rows padded to 20 floats) sweeps 64-token
+// (W_r slice in shared memory, rows padded to 17 floats so the 32 lanes'
+// single-float reads of 32 consecutive rows fall in distinct banks) sweeps 64-token
 // tiles; a tile's pairs are listed in shared memory and done up to 128 at a
 // time (16 per warp) while the tile's x rows stream through a ring of six
 // 64-wide K chunks (five in flight).
 // ---------------------------------------------------------------------------
-constexpr int kExES = 16, kExWS = 20, kExTile = 64, kExKc = 64, kExStages = 6, kExWarps = 8;
+constexpr int kExES = 16, kExWS = 17, kExTile = 64, kExKc = 64, kExStages = 6, kExWarps = 8;
 constexpr int kExPairsPerWarp = 16;
 constexpr int kExPass = kExWarps * kExPairsPerWarp;
 constexpr int kExChunkBytes = kExTile * kExKc * 2;
@@ -550,7 +551,11 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
         const int i = idx / (kExES / 4);
         const int q = idx % (kExES / 4);
         const float4 v = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) + q);
-        *reinterpret_cast<float4*>(Ws + i * kExWS + 4 * q) = v;
+        float* dst = Ws + i * kExWS + 4 * q;
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
     }
     pdl_wait();
     const uint32_t xs_base = smem_u32(xs);

@@ -28,12 +28,12 @@ def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
 
 class MoeLayer:
     def __init__(self, T_max, d, E, k, f, group, gate, up, down, w_r, b_r=None,
-                 device="cuda", keep_logical=False):
+                 device="cuda", keep_logical=False, flags=0):
         """gate/up/down: objects with .q (uint8 [E,N,K/2]), .scale, .bias
         (uint16 bf16 bits [E,N,K/group]); w_r float32 [d,E]; b_r float32 [E]."""
         self.device = torch.device(device)
         self.T_max, self.d, self.E, self.k, self.f, self.group = T_max, d, E, k, f, group
-        self.plan = Plan(T_max, d, E, k, f, group)
+        self.plan = Plan(T_max, d, E, k, f, group, flags)
         info = self.plan.info
         logical = [tuple(_dev(getattr(p, n), self.device) for n in ("q", "scale", "bias"))
                    for p in (gate, up, down)]
@@ -47,10 +47,10 @@ class MoeLayer:
         torch.cuda.synchronize(self.device)
 
     @classmethod
-    def from_inputs(cls, inp, T_max=None, device="cuda", keep_logical=False):
+    def from_inputs(cls, inp, T_max=None, device="cuda", keep_logical=False, flags=0):
         s = inp.shape
         return cls(T_max or s.T, s.d, s.E, s.k, s.f, s.group, inp.gate, inp.up, inp.down,
-                   inp.w_r, inp.b_r, device=device, keep_logical=keep_logical)
+                   inp.w_r, inp.b_r, device=device, keep_logical=keep_logical, flags=flags)
 
     def route_buffers(self, T):
         dev, k, E = self.device, self.k, self.E

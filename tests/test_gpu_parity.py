@@ -401,3 +401,28 @@ def test_fast_router_ties(moe, kind):
 def test_fast_router_near_ties_wide(moe):
     # the 2048-wide, 128-expert router with pairs of experts one ulp apart
     fast_case(moe, 1024, 2048, 128, 8, 91, "one_ulp_apart")
+
+
+def test_device_timeout_is_reported_and_workspace_recovers(moe):
+    # The test hook withholds one weight stage of the gate/up GEMM and cuts its
+    # wait limit to 5 ms: the consumers' bounded waits run out, the kernel
+    # records MOE_ERR_DEVICE_TIMEOUT with the role that gave up, drains its
+    # copies, frees its TMEM and returns.  A normal call on the same workspace
+    # afterwards is correct.
+    inp = workload("tiny")
+    s = inp.shape
+    bad = moe.MoeLayer.from_inputs(inp, flags=moe.SHAPE_TEST_TIMEOUT)
+    assert bad.plan.forward_path(s.T) == 0
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bad.forward(x)
+    torch.cuda.synchronize()
+    code, detail = bad.read_status()
+    assert code == 6, (code, detail)            # MOE_ERR_DEVICE_TIMEOUT
+    assert 101 <= detail <= 106, detail         # a gate/up GEMM role
+    good = moe.MoeLayer.from_inputs(inp)
+    good.ws = bad.ws                            # same shape: same workspace layout
+    y = good.forward(x)
+    torch.cuda.synchronize()
+    assert good.read_status() == (0, 0)
+    check_y(y[:s.T], oracle.forward(inp)["y"], "after a timeout")
+
