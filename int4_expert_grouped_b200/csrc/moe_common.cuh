@@ -128,6 +128,11 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
                  : "memory");
 }
 
+// 4-byte copy global -> shared (cp.async, completion by cp.async.wait_group).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
 // Order this thread's generic-proxy view of shared memory before its later
 // async-proxy operations (tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -268,6 +268,7 @@ __device__ __forceinline__ void stage_rows(uint16_t* dst, float* sums, const uin
 
 // Routing of the few tokens, in shared memory (identical in every CTA).
 struct DecRoute {
+    float sel[kDecMaxAssign];  // logit of each selected slot
     int idx[kDecMaxAssign];
     float w[kDecMaxAssign];
     int sa[kDecMaxAssign];
@@ -286,25 +287,31 @@ struct DecRoute {
     int abort_local;           // this CTA gave up
 };
 
-// top-k per token by one warp (ties go to the lower id) with the softmax
-// weights over the k slots, counts (integer atomics), offsets (exclusive
-// scan), one block per expert with rows (ascending expert), and the stable
-// scatter (rank of assignment a = number of earlier assignments to its
-// expert).  All kDecThreads threads.
+// top-k (each (token, expert) pair finds its slot by counting the experts
+// ahead of it; ties go to the lower id; measured faster here than a warp
+// top-k per token), the softmax weights over the k slots, counts (integer
+// atomics), offsets (exclusive scan), one block per expert with rows
+// (ascending expert), and the stable scatter (rank of assignment a = number
+// of earlier assignments to its expert).  All kDecThreads threads.
 __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int Tk = T * k;
     if (tid < E) R.cnt[tid] = 0;
-    for (int t = warp; t < T; t += kDecThreads / 32) {
-        int id;
-        float wt;
-        warp_topk(lg + t * E, E, k, lane, id, wt);
-        if (lane < k) {
-            R.idx[t * k + lane] = id;
-            R.w[t * k + lane] = wt;
+    for (int it = tid; it < T * E; it += kDecThreads) {
+        const int t = it / E;
+        const int e = it - t * E;
+        const int slot = expert_slot(lg + t * E, E, e);
+        if (slot < k) {
+            R.idx[t * k + slot] = e;
+            R.sel[t * k + slot] = lg[it];
         }
+    }
+    __syncthreads();
+    for (int t = warp; t < T; t += kDecThreads / 32) {
+        const float wt = warp_slot_weights(lane < k ? R.sel[t * k + lane] : 0.0f, k, lane);
+        if (lane < k) R.w[t * k + lane] = wt;
     }
     __syncthreads();
     for (int a = tid; a < Tk; a += kDecThreads) atomicAdd(&R.cnt[R.idx[a]], 1);

@@ -62,14 +62,18 @@ constexpr int kBStageBytes = kBlockT * 128;  // up to 256 token rows x 64 bf16
 constexpr int kEpiRowBytes = 80;    // staging row: 32 bf16 + 16 bytes of padding
 constexpr uint32_t kTmemCols = 512;
 
-// Per-projection configuration.
-template <bool kDown>
+// Per-projection configuration.  kStream: the ring sizes for blocks of few
+// rows (a batch of at most 64 rows per expert on average), where the kernel
+// is bound by reading the packed weights from HBM: a deep packed-weight ring
+// keeps more of them in flight per SM, at the cost of expanded-A and token
+// stages that such blocks do not need.
+template <bool kDown, bool kStream>
 struct Cfg {
     static constexpr int kTiles = kDown ? kDownTiles : 2;     // A tiles (of 128 rows) per unit
     static constexpr bool kOneTile = kTiles == 1;
-    static constexpr int kNW = kOneTile ? 4 : 2;              // packed weight ring
-    static constexpr int kNA = kOneTile ? 4 : 3;              // expanded bf16 A ring
-    static constexpr int kNB = 3;                             // token B ring
+    static constexpr int kNW = kStream ? (kOneTile ? 20 : 8) : (kOneTile ? 4 : 2);  // packed weight ring
+    static constexpr int kNA = kStream ? 2 : (kOneTile ? 4 : 3);  // expanded bf16 A ring
+    static constexpr int kNB = kStream ? 2 : 3;                   // token B ring
     static constexpr int kAccBufs = kOneTile ? 2 : 1;         // TMEM accumulator buffers
     static constexpr int kAccCols = kTiles * kBlockT;         // columns per buffer
     static constexpr int kAStageBytes = kTiles * kATileBytes;
@@ -133,9 +137,9 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
     return true;
 }
 
-template <bool kDown>
+template <bool kDown, bool kStream>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
-    using C = Cfg<kDown>;
+    using C = Cfg<kDown, kStream>;
     extern __shared__ uint8_t smem_raw[];
     pdl_launch_dependents();
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -558,12 +562,17 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<false>::kSmemBytes);
+    cudaError_t e;
+#define MOE_SET_SMEM(D, S)                                                                     \
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<D, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             Cfg<D, S>::kSmemBytes);                                           \
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg<true>::kSmemBytes);
+    MOE_SET_SMEM(false, false)
+    MOE_SET_SMEM(true, false)
+    MOE_SET_SMEM(false, true)
+    MOE_SET_SMEM(true, true)
+#undef MOE_SET_SMEM
+    return cudaSuccess;
 }
 
 static cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
@@ -653,16 +662,20 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
     return cudaGetLastError();
 }
 
-static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaStream_t st) {
-    if (a.max_units <= 0) return cudaSuccess;
+template <bool kDown, bool kStream>
+static cudaError_t launch_gemm_t(const GemmArgs& a, int num_sms, cudaStream_t st) {
     const int grid = a.max_units < num_sms ? a.max_units : num_sms;
     // Plain launches: letting the next kernel's CTAs be scheduled early measured
     // slower around the GEMMs (their pdl_wait then returns at once).
-    if (down)
-        grouped_gemm_kernel<true><<<grid, kGemmThreads, Cfg<true>::kSmemBytes, st>>>(a);
-    else
-        grouped_gemm_kernel<false><<<grid, kGemmThreads, Cfg<false>::kSmemBytes, st>>>(a);
+    grouped_gemm_kernel<kDown, kStream><<<grid, kGemmThreads, Cfg<kDown, kStream>::kSmemBytes, st>>>(a);
     return cudaGetLastError();
+}
+
+static cudaError_t launch_gemm(const GemmArgs& a, int num_sms, bool down, cudaStream_t st) {
+    if (a.max_units <= 0) return cudaSuccess;
+    if (down)
+        return a.stream ? launch_gemm_t<true, true>(a, num_sms, st) : launch_gemm_t<true, false>(a, num_sms, st);
+    return a.stream ? launch_gemm_t<false, true>(a, num_sms, st) : launch_gemm_t<false, false>(a, num_sms, st);
 }
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, int num_sms, cudaStream_t st) {

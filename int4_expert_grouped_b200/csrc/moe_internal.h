@@ -82,7 +82,8 @@ constexpr int kFastRouterMinT = 1024;  // smallest batch the int8 tensor-core ro
 struct RouterFastWs {
     int8_t *xa, *xb;            // token digits [T][d]
     int8_t *wc, *wd;            // expert digits [E][d]
-    float *s_t, *E_t, *A_t, *N_t, *theta;  // per token: scale, remainder max, sum |x'|, ||x||, threshold
+    float *s_t, *E_t, *A_t, *N_t;  // per token: scale, remainder max, sum |x'|, ||x||
+    uint32_t* cmask;            // [T][E/32] candidate experts of each token (bit e % 32 of word e / 32)
     float *u_e, *F_e, *B_e, *Wn_e;         // per expert: scale, remainder max, sum |w|, ||w||
     float* L;                   // [T][E] approximate logits with the bias
     float* exact;               // [T][E] fixed-order logits of the candidate pairs
@@ -133,6 +134,7 @@ struct GemmArgs {
     int group;
     int block_bytes;
     int max_units;                 // upper bound of num_blocks * NT
+    int stream;                    // ring sizes for blocks of few rows (weight streaming)
     int withhold_first;            // test hook: the weight producer skips its first copy
     uint64_t wait_ns;              // limit of every device-side wait
 };

@@ -182,12 +182,16 @@ router_logits_smem_kernel(const uint16_t* __restrict__ x, const float* __restric
 
     pdl_launch_dependents();
     // the W_r slice, row i -> Ws[i * WS .. + ES) (an input: loaded while the
-    // previous kernel in the stream finishes)
-    for (int idx = threadIdx.x; idx < d * (ES / 4); idx += blockDim.x) {
-        const int i = idx / (ES / 4);
-        const int q = idx % (ES / 4);
-        const float4 v = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) + q);
-        *reinterpret_cast<float4*>(Ws + i * WS + 4 * q) = v;
+    // previous kernel in the stream finishes), as asynchronous 16-byte copies
+    // that are all in flight at once
+    {
+        const uint32_t ws_base = smem_u32(Ws);
+        for (int idx = threadIdx.x; idx < d * (ES / 4); idx += blockDim.x) {
+            const int i = idx / (ES / 4);
+            const int q = idx % (ES / 4);
+            cp_async_16(ws_base + (i * WS + 4 * q) * 4, W + static_cast<size_t>(i) * E + e0 + 4 * q, 16u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
     pdl_wait();
     if (blockIdx.x == 0) {

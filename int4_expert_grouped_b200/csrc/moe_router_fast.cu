@@ -20,6 +20,8 @@
 //                           so the only error against the exact dot product
 //                           is the digits' remainder, which is bounded
 //   router_threshold_kernel per token the k-th largest lower bound l' - delta
+//                           and the mask of candidates: the experts whose
+//                           upper bound l' + delta reaches it
 //   router_exact_kernel     the fixed-order fp32 logit of every pair whose
 //                           upper bound l' + delta reaches the token's
 //                           threshold (a few per token), with W_r slices in
@@ -446,17 +448,6 @@ __device__ __forceinline__ float route_delta(float L, float A_t, float E_t, floa
     return __fadd_ru(__fadd_ru(d1, d2), __fadd_ru(d3, __fadd_ru(d4, 1e-30f)));
 }
 
-struct TokenBound {
-    float A, E, N, theta;
-};
-
-__device__ __forceinline__ float pair_upper(const RouterFastWs& ws, const float* b_r, int E, int t,
-                                            int e, const TokenBound& tb) {
-    const float L = ws.L[static_cast<size_t>(t) * E + e];
-    const float babs = b_r != nullptr ? fabsf(__ldg(b_r + e)) : 0.0f;
-    return __fadd_ru(L, route_delta(L, tb.A, tb.E, tb.N, ws.F_e[e], ws.B_e[e], ws.Wn_e[e], babs));
-}
-
 // ---------------------------------------------------------------------------
 // Threshold: per token (one warp), the k-th largest lower bound L - delta.
 // ---------------------------------------------------------------------------
@@ -471,28 +462,34 @@ router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, i
     if (t >= T) return;
     const float A = ws.A_t[t], Et = ws.E_t[t], N = ws.N_t[t];
     constexpr int kPer = kMaxExperts / 32;
-    float lo[kPer];
+    float lo[kPer], up[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
+        lo[i] = -INFINITY;
+        up[i] = -INFINITY;
         if (e < E) {
             const float L = ws.L[static_cast<size_t>(t) * E + e];
             const float babs = b_r != nullptr ? fabsf(__ldg(b_r + e)) : 0.0f;
-            lo[i] = __fsub_rd(L, route_delta(L, A, Et, N, ws.F_e[e], ws.B_e[e], ws.Wn_e[e], babs));
-        } else {
-            lo[i] = -INFINITY;
+            const float dl = route_delta(L, A, Et, N, ws.F_e[e], ws.B_e[e], ws.Wn_e[e], babs);
+            lo[i] = __fsub_rd(L, dl);
+            up[i] = __fadd_ru(L, dl);
         }
     }
-    // k rounds of a warp arg-max (value desc, slot asc); the k-th value taken
+    // theta: the k-th largest lower bound (k rounds of a warp arg-max, value
+    // desc, expert asc; the taken entry is removed)
     float theta = -INFINITY;
+    float lw[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) lw[i] = lo[i];
     for (int j = 0; j < k; ++j) {
         float bv = -INFINITY;
         int bi = 1 << 30;
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
             const int id = lane + 32 * i;
-            if (id < E && (lo[i] > bv || (lo[i] == bv && id < bi))) {
-                bv = lo[i];
+            if (id < E && (lw[i] > bv || (lw[i] == bv && id < bi))) {
+                bv = lw[i];
                 bi = id;
             }
         }
@@ -507,10 +504,16 @@ router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, i
         }
 #pragma unroll
         for (int i = 0; i < kPer; ++i)
-            if (lane + 32 * i == bi) lo[i] = -INFINITY, bi = -1;  // taken (bi < 0 only in its lane)
+            if (lane + 32 * i == bi) lw[i] = -INFINITY;
         theta = bv;
     }
-    if (lane == 0) ws.theta[t] = theta;
+    // candidates: upper bound >= theta
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        if (32 * i >= E) break;
+        const unsigned m = __ballot_sync(0xffffffffu, lane + 32 * i < E && up[i] >= theta);
+        if (lane == 0) ws.cmask[static_cast<size_t>(t) * ((E + 31) / 32) + i] = m;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -531,6 +534,9 @@ __host__ __device__ constexpr int ex_smem_bytes(int d) {
     return d * kExWS * 4 + kExStages * kExChunkBytes + kExTile * kExES * 4 + 64;
 }
 
+// barrier of the first two warps (the pair-list builders)
+__device__ __forceinline__ void named_sync_64() { asm volatile("bar.sync 2, 64;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kExWarps * 32, 1)
 router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
                     const float* __restrict__ b_r, RouterFastWs ws, int T, int d, int E) {
@@ -538,7 +544,7 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     float* Ws = reinterpret_cast<float*>(ex_raw);
     uint16_t* xs = reinterpret_cast<uint16_t*>(ex_raw + static_cast<size_t>(d) * kExWS * 4);
     int* pairs = reinterpret_cast<int*>(ex_raw + static_cast<size_t>(d) * kExWS * 4 + kExStages * kExChunkBytes);
-    int* npairs = pairs + kExTile * kExES;
+    int* npairs = pairs + kExTile * kExES;  // [0]: pairs of the tile; [1], [2]: per-warp counts
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int nslices = E / kExES;
@@ -547,15 +553,17 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     const int ctas = gridDim.x / nslices;
     const int e0 = slice * kExES;
     pdl_launch_dependents();
-    for (int idx = threadIdx.x; idx < d * (kExES / 4); idx += blockDim.x) {
-        const int i = idx / (kExES / 4);
-        const int q = idx % (kExES / 4);
-        const float4 v = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(i) * E + e0) + q);
-        float* dst = Ws + i * kExWS + 4 * q;
-        dst[0] = v.x;
-        dst[1] = v.y;
-        dst[2] = v.z;
-        dst[3] = v.w;
+    // the W_r slice (model weights, never written by this library: loaded
+    // before waiting for the previous kernel), one asynchronous 4-byte copy
+    // per element so all of them are in flight at once
+    {
+        const uint32_t ws_base = smem_u32(Ws);
+        for (int idx = threadIdx.x; idx < d * kExES; idx += blockDim.x) {
+            const int i = idx / kExES;
+            const int el = idx % kExES;
+            cp_async_4(ws_base + (i * kExWS + el) * 4, W + static_cast<size_t>(i) * E + e0 + el);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
     pdl_wait();
     const uint32_t xs_base = smem_u32(xs);
@@ -581,20 +589,40 @@ router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
     };
     for (int tile = cta; tile < ntiles; tile += ctas) {
         const int t0 = tile * kExTile;
-        __syncthreads();  // the previous tile's pair list and x buffers are no longer read
-        if (threadIdx.x == 0) *npairs = 0;
+        // (first tile: the W_r slice has landed) the previous tile's pair list
+        // and x buffers are no longer read
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
-        for (int it = threadIdx.x; it < kExTile * kExES; it += blockDim.x) {
-            const int tl = it / kExES;
-            const int el = it % kExES;
+        // the tile's candidate pairs in this slice, in (token, expert) order:
+        // thread tl < 64 takes token t0 + tl's 16 mask bits; the first two warps
+        // scan the counts
+        if (threadIdx.x < kExTile) {
+            const int tl = threadIdx.x;
             const int t = t0 + tl;
-            if (t < T) {
-                const TokenBound tb{ws.A_t[t], ws.E_t[t], ws.N_t[t], ws.theta[t]};
-                if (pair_upper(ws, b_r, E, t, e0 + el, tb) >= tb.theta) pairs[atomicAdd(npairs, 1)] = it;
+            uint32_t bits = 0;
+            if (t < T)
+                bits = (ws.cmask[static_cast<size_t>(t) * ((E + 31) / 32) + (e0 >> 5)] >> (e0 & 31)) &
+                       ((1u << kExES) - 1u);
+            const int cnt = __popc(bits);
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, inc, o);
+                if ((tl & 31) >= o) inc += nb;
             }
+            if ((tl & 31) == 31) npairs[1 + (tl >> 5)] = inc;  // per-warp totals
+            __syncwarp();
+            named_sync_64();
+            int base = inc - cnt + (tl >= 32 ? npairs[1] : 0);
+            while (bits) {
+                const int el = __ffs(bits) - 1;
+                bits &= bits - 1;
+                pairs[base++] = tl * kExES + el;
+            }
+            if (tl == kExTile - 1) npairs[0] = base;
         }
         __syncthreads();
-        const int np = *npairs;
+        const int np = npairs[0];
         for (int base = 0; base < np; base += kExPass) {
             int tl[kExPairsPerWarp], el[kExPairsPerWarp];
             bool on[kExPairsPerWarp];
@@ -659,11 +687,10 @@ router_select_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, int 
     pdl_wait();
     const int t = blockIdx.x * kSelWarps + warp;
     if (t >= T) return;
-    const TokenBound tb{ws.A_t[t], ws.E_t[t], ws.N_t[t], ws.theta[t]};
-    for (int e = lane; e < E; e += 32)
-        rows[warp][e] = pair_upper(ws, b_r, E, t, e, tb) >= tb.theta
-                            ? ws.exact[static_cast<size_t>(t) * E + e]
-                            : -INFINITY;
+    for (int e = lane; e < E; e += 32) {
+        const uint32_t m = ws.cmask[static_cast<size_t>(t) * ((E + 31) / 32) + (e >> 5)];
+        rows[warp][e] = (m >> (e & 31)) & 1u ? ws.exact[static_cast<size_t>(t) * E + e] : -INFINITY;
+    }
     __syncwarp();
     int my_id;
     float my_w;
@@ -685,7 +712,8 @@ bool router_fast_supported(int T, int d, int E) {
 size_t router_fast_ws_bytes(int T, int d, int E) {
     auto r = [](size_t v) { return (v + 255) / 256 * 256; };
     const size_t t = static_cast<size_t>(T), dd = static_cast<size_t>(d), e = static_cast<size_t>(E);
-    return 2 * r(t * dd) + 2 * r(e * dd) + 5 * r(t * 4) + 4 * r(e * 4) + r(t * e * 4);
+    return 2 * r(t * dd) + 2 * r(e * dd) + 4 * r(t * 4) + r(t * ((e + 31) / 32) * 4) + 4 * r(e * 4) +
+           r(t * e * 4);
 }
 
 RouterFastWs router_fast_ws(uint8_t* base, float* L, int T, int d, int E) {
@@ -706,7 +734,7 @@ RouterFastWs router_fast_ws(uint8_t* base, float* L, int T, int d, int E) {
     w.E_t = reinterpret_cast<float*>(take(t * 4));
     w.A_t = reinterpret_cast<float*>(take(t * 4));
     w.N_t = reinterpret_cast<float*>(take(t * 4));
-    w.theta = reinterpret_cast<float*>(take(t * 4));
+    w.cmask = reinterpret_cast<uint32_t*>(take(t * ((e + 31) / 32) * 4));
     w.u_e = reinterpret_cast<float*>(take(e * 4));
     w.F_e = reinterpret_cast<float*>(take(e * 4));
     w.B_e = reinterpret_cast<float*>(take(e * 4));

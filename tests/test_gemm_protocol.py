@@ -32,7 +32,8 @@ EPILOGUE_WARPS = 4
 
 
 def kernel_configs():
-    """(name, NW, NA, NB, G, acc_bufs) of the two projections, from the source."""
+    """(name, NW, NA, NB, G, acc_bufs) of the two projections in both ring
+    variants (large blocks; weight streaming for small blocks), from the source."""
     src = open(GEMM_SRC).read()
     down_tiles = int(re.search(r"constexpr int kDownTiles = (\d+);", open(INTERNAL_H).read()).group(1))
 
@@ -41,14 +42,24 @@ def kernel_configs():
         assert m, name
         return int(m.group(1)), int(m.group(2))
 
-    nw, na, acc, g = pick("kNW"), pick("kNA"), pick("kAccBufs"), pick("kGroups")
-    nb = int(re.search(r"static constexpr int kNB = (\d+);", src).group(1))
+    acc, g = pick("kAccBufs"), pick("kGroups")
+    m = re.search(r"static constexpr int kNW = kStream \? \(kOneTile \? (\d+) : (\d+)\) : "
+                  r"\(kOneTile \? (\d+) : (\d+)\);", src)
+    assert m, "kNW"
+    nw_s, nw = (int(m.group(1)), int(m.group(2))), (int(m.group(3)), int(m.group(4)))
+    m = re.search(r"static constexpr int kNA = kStream \? (\d+) : \(kOneTile \? (\d+) : (\d+)\);", src)
+    assert m, "kNA"
+    na_s, na = (int(m.group(1)),) * 2, (int(m.group(2)), int(m.group(3)))
+    m = re.search(r"static constexpr int kNB = kStream \? (\d+) : (\d+);", src)
+    assert m, "kNB"
+    nb_s, nb = int(m.group(1)), int(m.group(2))
     # each pair is (value with one weight tile per unit, value with two);
     # gate/up always has two tiles, down has kDownTiles
-    gu = ("gate/up", nw[1], na[1], nb, g[1], acc[1])
     i = 0 if down_tiles == 1 else 1
-    dn = ("down", nw[i], na[i], nb, g[i], acc[i])
-    return [gu, dn]
+    return [("gate/up", nw[1], na[1], nb, g[1], acc[1]),
+            ("down", nw[i], na[i], nb, g[i], acc[i]),
+            ("gate/up, streaming", nw_s[1], na_s[1], nb_s, g[1], acc[1]),
+            ("down, streaming", nw_s[i], na_s[i], nb_s, g[i], acc[i])]
 
 
 class Barrier:
