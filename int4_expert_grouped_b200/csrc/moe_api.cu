@@ -368,7 +368,8 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     const bool test_timeout = (s.flags & MOE_SHAPE_TEST_TIMEOUT) != 0;
     g.withhold_first = test_timeout ? 1 : 0;
     g.wait_ns = test_timeout ? 5000000ull : moe::kWaitTimeoutNs;
-    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT));
+    for (int i = 0; i < moe::kBoxSizes; ++i)
+        MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap[i], xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT >> i));
     MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
     if (ev && !mark(ev->gate_up)) return MOE_ERR_CUDA;
 
@@ -382,7 +383,8 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.max_units = mb * g.NT;
     g.withhold_first = 0;
     g.wait_ns = moe::kWaitTimeoutNs;
-    MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap, h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT));
+    for (int i = 0; i < moe::kBoxSizes; ++i)
+        MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap[i], h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT >> i));
     MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;
     MOE_CUDA(moe::launch_combine(xs, r.pos, r.w, T, s.k, s.d, y, status, num_sms, st));

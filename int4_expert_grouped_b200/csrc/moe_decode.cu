@@ -65,11 +65,11 @@ constexpr int kDecComputeWarps = 8;
 constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;  // + one producer warp
 constexpr int kDecProducerWarp = kDecComputeWarps;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
-constexpr int kDecStages = 24;
-// One stage = one 64-wide K chunk of a slice's 64 gate and 64 up rows
-// (nibbles, then scale/bias words), or one down block (128 rows x 64 K):
-// both 4096 + 512 * (64 / group) bytes.
-constexpr int kDecStageBytes = 4096 + 512 * 2;
+constexpr int kDecStages = 16;
+// One stage = two 64-wide K chunks of a slice's 64 gate and 64 up rows (two
+// consecutive half-blocks, one bulk copy), or two down blocks (128 rows x
+// 64 K each): 2 * half_block_bytes(group) bytes.
+constexpr int kDecStageBytes = 2 * half_block_bytes(32);
 constexpr int kDecMaxAssign = 64;                          // T * k the path takes
 constexpr int kDecSlice = 64;                              // features per unit
 constexpr int kDecMaxSlices = 32;                          // f / 64
@@ -367,7 +367,7 @@ __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     L.h = take(kDecodeMaxT * kDecHStride * 2);
     L.hsum = take(kDecodeMaxT * (kDecSlice / 32) * 4);
     L.lg = take(T * E * 4);
-    L.red = take(kDecComputeWarps * kDecRowTiles * 4 * 32 * 4);  // per-warp gate/up partial sums
+    L.red = take(kDecComputeWarps / 2 * kDecRowTiles * 4 * 32 * 4);  // gate/up partial sums, half the warps
     L.route = take(static_cast<int>(sizeof(DecRoute)));
     L.bars = take((2 * kDecStages + 1) * 8);
     L.total = o + 1024;  // + slack to align the base
@@ -599,8 +599,6 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     const int NT = f / 128, KC = d / kKChunk, NTd = d / 128, KCd = f / kKChunk;
     const int S = f / kDecSlice;
     const int u_total = nb * S;
-    const int nib_gu = 256 * 32;                 // nibble bytes of a gate/up block
-    const int sc_bytes = kDecSlice * kGpc * 4;   // (scale, bias) words of 64 rows
 
     if (warp == kDecProducerWarp) {
         // the whole warp runs the loop; one elected lane issues the copies
@@ -611,7 +609,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int fs = u - b * S;
             const int e = R.blk_e[b];
             const int j = fs >> 1, hh = fs & 1;  // 128-feature tile, half of it
-            for (int st = 0; st < KC + NTd; ++st, ++q) {
+            const uint8_t* gsrc = p.wgu + ((static_cast<size_t>(e) * NT + j) * 2 + hh) * KC * p.bb_dn;
+            for (int st = 0; st < KC / 2 + NTd / 2; ++st, ++q) {
                 const int slot = q % kDecStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(empty(slot), ((q / kDecStages) & 1) ^ 1, &R.abort_local))) {
                     ok = false;
@@ -619,21 +618,19 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 }
                 if (elect_one()) {
                     const uint32_t dst = smem_u32(ring + slot * kDecStageBytes);
-                    mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(p.bb_dn));
-                    if (st < KC) {
-                        // chunk st of the slice: gate rows 64 hh .., up rows 128 + 64 hh ..
-                        const uint8_t* blk = p.wgu + ((static_cast<size_t>(e) * NT + j) * KC + st) * p.bb_gu;
-                        bulk_copy_g2s(dst, blk + hh * kDecSlice * 32, kDecSlice * 32, full(slot));
-                        bulk_copy_g2s(dst + kDecSlice * 32, blk + (128 + hh * kDecSlice) * 32, kDecSlice * 32,
-                                      full(slot));
-                        bulk_copy_g2s(dst + 2 * kDecSlice * 32, blk + nib_gu + hh * sc_bytes, sc_bytes, full(slot));
-                        bulk_copy_g2s(dst + 2 * kDecSlice * 32 + sc_bytes,
-                                      blk + nib_gu + (128 / kDecSlice + hh) * sc_bytes, sc_bytes, full(slot));
+                    mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(2 * p.bb_dn));
+                    if (st < KC / 2) {
+                        // K chunks 2 st, 2 st + 1 of the slice: consecutive half-blocks
+                        bulk_copy_g2s(dst, gsrc + static_cast<size_t>(2 * st) * p.bb_dn,
+                                      static_cast<uint32_t>(2 * p.bb_dn), full(slot));
                     } else {
-                        // down block (expert, output tile st - KC, K chunk fs)
-                        const uint8_t* blk =
-                            p.wdn + ((static_cast<size_t>(e) * NTd + (st - KC)) * KCd + fs) * p.bb_dn;
-                        bulk_copy_g2s(dst, blk, static_cast<uint32_t>(p.bb_dn), full(slot));
+                        // down blocks (expert, output tiles jd, jd + 1, K chunk fs)
+                        const int jd = 2 * (st - KC / 2);
+                        for (int h = 0; h < 2; ++h) {
+                            const uint8_t* blk =
+                                p.wdn + ((static_cast<size_t>(e) * NTd + jd + h) * KCd + fs) * p.bb_dn;
+                            bulk_copy_g2s(dst + h * p.bb_dn, blk, static_cast<uint32_t>(p.bb_dn), full(slot));
+                        }
                     }
                 }
                 __syncwarp();
@@ -677,7 +674,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
 #pragma unroll
             for (int r = 0; r < kDecRowTiles; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
             for (int st = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
-                 st < KC; st += kDecComputeWarps) {
+                 st < KC / 2; st += kDecComputeWarps) {
                 const uint32_t qs = q + st;
                 const int slot = qs % kDecStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (qs / kDecStages) & 1, &R.abort_local))) {
@@ -687,44 +684,54 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     }
                     break;
                 }
-                const uint8_t* stage = ring + slot * kDecStageBytes;
 #pragma unroll
-                for (int r = 0; r < kDecRowTiles; ++r) {
-                    const int fr = 8 * r + g;
-                    chunk_mma_rows<kGpc>(acc[r], stage + fr * 32, stage + (kDecSlice + fr) * 32,
-                                         stage + 2 * kDecSlice * 32 + fr * kGpc * 4,
-                                         stage + 2 * kDecSlice * 32 + sc_bytes + fr * kGpc * 4, c,
-                                         brow + kKChunk * st, bs0 + 2 * st, bs1 + 2 * st);
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint8_t* hb = ring + slot * kDecStageBytes + cc * p.bb_dn;  // half-block of chunk kc
+                    const int kc = 2 * st + cc;
+#pragma unroll
+                    for (int r = 0; r < kDecRowTiles; ++r) {
+                        const int fr = 8 * r + g;
+                        chunk_mma_rows<kGpc>(acc[r], hb + gu_nib_offset(0, fr), hb + gu_nib_offset(1, fr),
+                                             hb + gu_word_offset(0, fr, 0, kGpc), hb + gu_word_offset(1, fr, 0, kGpc),
+                                             c, brow + kKChunk * kc, bs0 + 2 * kc, bs1 + 2 * kc);
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(slot));
             }
-            q += KC;
-            // partial sums of every warp -> shared memory, added in warp order
-#pragma unroll
-            for (int r = 0; r < kDecRowTiles; ++r)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) red[((warp * kDecRowTiles + r) * 4 + i) * 32 + lane] = acc[r][i];
+            q += KC / 2;
+            // the warps' partial sums added in a fixed tree: ((w0 + w4) + (w2 + w6))
+            // + ((w1 + w5) + (w3 + w7)), through half-size shared memory
             compute_sync();
             if (vload(R.fail)) break;
-            // SwiGLU of the slice, rounded to bf16, into shared memory [token][64]:
-            // thread (r, lane) of warp r finishes MMA tile r
-            {
-                const int r = warp;
-                float sum[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float v = red[((0 * kDecRowTiles + r) * 4 + i) * 32 + lane];
-                    for (int w = 1; w < kDecComputeWarps; ++w) v += red[((w * kDecRowTiles + r) * 4 + i) * 32 + lane];
-                    sum[i] = v;
-                }
-                const int fr = 8 * r + g;
+            for (int half = kDecComputeWarps / 2; half >= 1; half >>= 1) {
+                if (warp >= half && warp < 2 * half)
 #pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    const int col = 2 * c + e2;
-                    if (col < n)
-                        hsh[col * kDecHStride + fr] =
-                            bf16_round_bits(__fdividef(sum[e2] * sum[2 + e2], 1.0f + __expf(-sum[e2])));
+                    for (int r = 0; r < kDecRowTiles; ++r)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) red[(((warp - half) * kDecRowTiles + r) * 4 + i) * 32 + lane] = acc[r][i];
+                compute_sync();
+                if (warp < half)
+#pragma unroll
+                    for (int r = 0; r < kDecRowTiles; ++r)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[r][i] += red[((warp * kDecRowTiles + r) * 4 + i) * 32 + lane];
+                compute_sync();
+            }
+            // SwiGLU of the slice (warp 0 holds the sums), rounded to bf16, into
+            // shared memory [token][64]
+            if (warp == 0) {
+#pragma unroll
+                for (int r = 0; r < kDecRowTiles; ++r) {
+                    const int fr = 8 * r + g;
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int col = 2 * c + e2;
+                        if (col < n)
+                            hsh[col * kDecHStride + fr] =
+                                bf16_round_bits(__fdividef(acc[r][e2] * acc[r][2 + e2], 1.0f + __expf(-acc[r][e2])));
+                    }
                 }
             }
             compute_sync();
@@ -741,9 +748,9 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const uint16_t* hrow = hsh + cg * kDecHStride + 8 * c;
             const float* hs0 = hsum + c0 * 2;
             const float* hs1 = hsum + c1 * 2;
-            for (int jd = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
-                 jd < NTd; jd += kDecComputeWarps) {
-                const uint32_t qs = q + jd;
+            for (int sd = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
+                 sd < NTd / 2; sd += kDecComputeWarps) {
+                const uint32_t qs = q + sd;
                 const int slot = qs % kDecStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (qs / kDecStages) & 1, &R.abort_local))) {
                     if (lane == 0) {
@@ -752,29 +759,32 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     }
                     break;
                 }
-                const uint8_t* stage = ring + slot * kDecStageBytes;
-                float o[kDecRowTiles][4];
+                for (int h = 0; h < 2; ++h) {
+                    const int jd = 2 * sd + h;
+                    const uint8_t* stage = ring + slot * kDecStageBytes + h * p.bb_dn;
+                    float o[kDecRowTiles][4];
 #pragma unroll
-                for (int r = 0; r < kDecRowTiles; ++r) {
-                    o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.0f;
-                    chunk_mma<kGpc>(o[r], stage, 128 * 32, 16 * r + g, c, hrow, hs0, hs1);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty(slot));
+                    for (int r = 0; r < kDecRowTiles; ++r) {
+                        o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.0f;
+                        chunk_mma<kGpc>(o[r], stage, 128 * 32, 16 * r + g, c, hrow, hs0, hs1);
+                    }
 #pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    const int col = 2 * c + e2;
-                    if (col < n) {
-                        float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128;
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int col = 2 * c + e2;
+                        if (col < n) {
+                            float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128;
 #pragma unroll
-                        for (int r = 0; r < kDecRowTiles; ++r) {
-                            dst[16 * r + g] = o[r][e2];
-                            dst[16 * r + g + 8] = o[r][2 + e2];
+                            for (int r = 0; r < kDecRowTiles; ++r) {
+                                dst[16 * r + g] = o[r][e2];
+                                dst[16 * r + g + 8] = o[r][2 + e2];
+                            }
                         }
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty(slot));
             }
-            q += NTd;
+            q += NTd / 2;
             compute_sync();
             if (vload(R.fail)) break;
         }

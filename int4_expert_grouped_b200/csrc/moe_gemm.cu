@@ -212,7 +212,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int b = u / NT;
             const int j = u - b * NT;
             const int e = a.block_map[3 * b];
+            // down: blocks (e, j, c) in a row; gate/up: half-blocks (e, j, 0, c) and (e, j, 1, c)
             const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
+            const size_t half_stride = static_cast<size_t>(KC) * (a.block_bytes / 2);
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNW;
                 if (!warp_wait(wempty(s), ((it / C::kNW) & 1) ^ 1, abort_flag, a.wait_ns)) {
@@ -224,8 +226,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 if (a.withhold_first && it == 0) continue;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(wfull(s), a.block_bytes);
-                    bulk_copy_g2s(sbase + C::kOffW + s * C::kWStageBytes, src + c * a.block_bytes,
-                                  a.block_bytes, wfull(s));
+                    const uint32_t dst = sbase + C::kOffW + s * C::kWStageBytes;
+                    if constexpr (kDown) {
+                        bulk_copy_g2s(dst, src + c * a.block_bytes, a.block_bytes, wfull(s));
+                    } else {
+                        const uint32_t hb = a.block_bytes / 2;
+                        bulk_copy_g2s(dst, src + c * hb, hb, wfull(s));
+                        bulk_copy_g2s(dst + hb, src + half_stride + c * hb, hb, wfull(s));
+                    }
                 }
                 __syncwarp();
             }
@@ -303,13 +311,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             mbar_wait_drain(drain_bar, 0);
         }
     } else if (warp == kWarpLoader) {
-        // one 2-D TMA tile of kBlockT token rows per stage (rows past the block
+        // one 2-D TMA tile of token rows per stage, 256, 128, 64 or 32 rows: the
+        // smallest that covers the N rows the MMA reads (rows past the block
         // belong to the next expert or lie past the end and are zero-filled;
         // the MMA ignores columns >= N and the epilogue columns >= rows)
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
             const int row0 = a.block_map[3 * (u / NT) + 1];
+            // the smallest box (256 >> bi rows) that covers the N rows the MMA reads
+            const int N = (a.block_map[3 * (u / NT) + 2] + 15) & ~15;
+            int bi = 0;
+            while (bi + 1 < kBoxSizes && (kBlockT >> (bi + 1)) >= N) ++bi;
+            const uint32_t box_bytes = static_cast<uint32_t>(kBlockT >> bi) * (kKChunk * 2);
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNB;
                 if (!warp_wait(bempty(s), ((it / C::kNB) & 1) ^ 1, abort_flag, a.wait_ns)) {
@@ -318,8 +332,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     break;
                 }
                 if (elect_one()) {
-                    mbar_arrive_expect_tx(bfull(s), kBStageBytes);
-                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap, c * kKChunk, row0, bfull(s));
+                    mbar_arrive_expect_tx(bfull(s), box_bytes);
+                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap[bi], c * kKChunk, row0, bfull(s));
                 }
                 __syncwarp();
             }
@@ -357,14 +371,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 // latencies overlap.
                 const int half = gtid & 1;       // K 0..31 or 32..63 of the chunk
                 const int g = half * (gpc - 1);  // group 64: 0; group 32: half
+                const int hbytes = a.block_bytes / 2;  // gate/up half-block
                 uint4 pk[C::kTasks];
                 uint32_t sb[C::kTasks];
 #pragma unroll
                 for (int rep = 0; rep < C::kTasks; ++rep) {
                     const int row = (gtid + C::kGroupThreads * rep) >> 1;
-                    pk[rep] = *reinterpret_cast<const uint4*>(wst + row * 32 + half * 16);
-                    sb[rep] = *reinterpret_cast<const uint32_t*>(wst + C::kNibbleBytes +
-                                                                 (row * gpc + g) * 4);
+                    int nib_off, w_off;
+                    if constexpr (kDown) {
+                        nib_off = row * 32;
+                        w_off = C::kNibbleBytes + (row * gpc + g) * 4;
+                    } else {  // row: tile row >> 7, feature row & 127 in half-block (row & 127) >> 6
+                        const int hoff = ((row & 127) >> 6) * hbytes;
+                        nib_off = hoff + gu_nib_offset(row >> 7, row & 63);
+                        w_off = hoff + gu_word_offset(row >> 7, row & 63, g, gpc);
+                    }
+                    pk[rep] = *reinterpret_cast<const uint4*>(wst + nib_off + half * 16);
+                    sb[rep] = *reinterpret_cast<const uint32_t*>(wst + w_off);
                 }
 #pragma unroll
                 for (int rep = 0; rep < C::kTasks; ++rep) {
@@ -534,7 +557,13 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
         const uint16_t* bsrc = second ? s.b1 : s.b0;
         const size_t row = static_cast<size_t>(e) * s.N + n;
         const uint8_t* qrow = qsrc + row * (s.K / 2) + c * 32;
-        uint8_t* dst = out + ((static_cast<size_t>(e) * s.NT + j) * KC + c) * bb;
+        // down: block (e, j, c); gate/up: half-block (e, j, half, c) (see packed_block_bytes)
+        const int f = rr & 127;
+        const int hb = half_block_bytes(group);
+        uint8_t* dst = s.tiles == 1
+                           ? out + ((static_cast<size_t>(e) * s.NT + j) * KC + c) * bb
+                           : out + (((static_cast<size_t>(e) * s.NT + j) * 2 + (f >> 6)) * KC + c) * hb;
+        const int nib_off = s.tiles == 1 ? rr * 32 : gu_nib_offset(second ? 1 : 0, f & 63);
         uint32_t words[8];
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
@@ -547,14 +576,16 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
             }
             words[w] = word;
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + rr * 32);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + nib_off);
         d4[0] = make_uint4(words[0], words[1], words[2], words[3]);
         d4[1] = make_uint4(words[4], words[5], words[6], words[7]);
         const size_t grow = row * (s.K / group) + static_cast<size_t>(c) * gpc;
         for (int g = 0; g < gpc; ++g) {
             const uint32_t sv = ssrc[grow + g];
             const uint32_t bv = bsrc[grow + g];
-            *reinterpret_cast<uint32_t*>(dst + nibble_bytes + (rr * gpc + g) * 4) = sv | (bv << 16);
+            const int w_off = s.tiles == 1 ? nibble_bytes + (rr * gpc + g) * 4
+                                           : gu_word_offset(second ? 1 : 0, f & 63, g, gpc);
+            *reinterpret_cast<uint32_t*>(dst + w_off) = sv | (bv << 16);
         }
     }
 }

@@ -53,14 +53,26 @@ constexpr int kBlockT = 256;      // block map tile height = largest MMA N
 constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
 constexpr int kDecodeMaxT = 8;    // largest batch the small-batch (decode) path takes
 constexpr int kDownTiles = 1;     // 128-row down-projection tiles per packed block and GEMM unit
+constexpr int kBoxSizes = 4;      // token-tile boxes of 256, 128, 64 and 32 rows
 constexpr int kDecodeSyncBytes = 8192;  // flags of the small-batch kernel (workspace bytes 256 ..)
 
 // Packed weight block: `tiles` 128-row A tiles of one 64-wide K chunk
-// (gate/up: the gate rows, then the up rows of 128 features; down: 128 rows):
-// 128*tiles rows x 32 bytes of nibbles, then per row and group one
-// (scale, bias) bf16 pair.
+// (gate/up: the gate and the up rows of 128 features; down: 128 rows).
+// A down block is 128 rows x 32 bytes of nibbles, then per row and group one
+// (scale, bias) bf16 pair.  A gate/up block is two half-blocks of the same
+// form, one per 64 features: [64 gate rows][64 up rows] of nibbles, then the
+// gate rows' and the up rows' words; each half-block is stored with the same
+// half of the expert's other K chunks (layout [E][f/128][2][d/64][half-block]),
+// so the 64-feature slice of an expert is contiguous over K.
 __host__ __device__ constexpr int packed_block_bytes(int tiles, int group) {
     return 128 * tiles * 32 + 128 * tiles * (kKChunk / group) * 4;
+}
+__host__ __device__ constexpr int half_block_bytes(int group) { return packed_block_bytes(1, group); }
+// Byte offsets, inside a gate/up half-block, of the nibbles of row fl (< 64)
+// of tile t (0 gate, 1 up) and of its word for group g of the chunk.
+__host__ __device__ inline int gu_nib_offset(int t, int fl) { return t * 64 * 32 + fl * 32; }
+__host__ __device__ inline int gu_word_offset(int t, int fl, int g, int gpc) {
+    return 128 * 32 + (t * 64 + fl) * gpc * 4 + g * 4;
 }
 
 // ---- routing (moe_route.cu) ----
@@ -119,10 +131,11 @@ cudaError_t launch_prepack(const PrepackSource& src, int E, int group, uint8_t* 
                            cudaStream_t st);
 
 struct GemmArgs {
-    // B operand (token rows in expert order) for 2-D TMA tiles of 64 columns x
-    // kBlockT rows with the 128-byte swizzle, the K-major layout the MMA
-    // reads: gate/up reads xs [T*k, d], down reads h [T*k, f].
-    CUtensorMap bmap;
+    // B operand (token rows in expert order) for 2-D TMA tiles of 64 columns
+    // with the 128-byte swizzle, the K-major layout the MMA reads: gate/up
+    // reads xs [T*k, d], down reads h [T*k, f].  bmap[i] has boxes of
+    // kBlockT >> i rows; a unit loads the smallest box that covers its rows.
+    CUtensorMap bmap[kBoxSizes];
     const uint8_t* wpack;          // packed blocks [E][NT][K/64][block_bytes]
     const int32_t* block_map;      // [num_blocks, 3]
     const int32_t* num_blocks;     // [1], device
