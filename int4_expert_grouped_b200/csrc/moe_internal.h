@@ -95,10 +95,9 @@ struct RouterFastWs {
     int8_t *xa, *xb;            // token digits [T][d]
     int8_t *wc, *wd;            // expert digits [E][d]
     float *s_t, *E_t, *A_t, *N_t;  // per token: scale, remainder max, sum |x'|, ||x||
-    uint32_t* cmask;            // [T][E/32] candidate experts of each token (bit e % 32 of word e / 32)
     float *u_e, *F_e, *B_e, *Wn_e;         // per expert: scale, remainder max, sum |w|, ||w||
     float* L;                   // [T][E] approximate logits with the bias
-    float* exact;               // [T][E] fixed-order logits of the candidate pairs
+    float* wt;                  // [E][d] W_r transposed (fp32, exact copy)
 };
 bool router_fast_supported(int T, int d, int E);
 size_t router_fast_ws_bytes(int T, int d, int E);

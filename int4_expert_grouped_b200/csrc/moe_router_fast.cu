@@ -19,15 +19,14 @@
 //                           (a c, a d, b c, b d) accumulate in int32 in TMEM,
 //                           so the only error against the exact dot product
 //                           is the digits' remainder, which is bounded
-//   router_threshold_kernel per token the k-th largest lower bound l' - delta
-//                           and the mask of candidates: the experts whose
-//                           upper bound l' + delta reaches it
-//   router_exact_kernel     the fixed-order fp32 logit of every pair whose
-//                           upper bound l' + delta reaches the token's
-//                           threshold (a few per token), with W_r slices in
-//                           shared memory
-//   router_select_kernel    top-k among those pairs by (logit desc, id asc),
-//                           softmax weights, per-group histograms
+//   router_select_kernel    one warp per token: the bounds delta, the k-th
+//                           largest lower bound l' - delta (theta), the
+//                           candidates (upper bound l' + delta >= theta, a
+//                           few per token), their fixed-order fp32 logits
+//                           (lane p runs chain p over the transposed W_r
+//                           column, then the butterfly and the bias), top-k
+//                           among them by (logit desc, id asc), the softmax
+//                           weights and the per-group histograms
 //
 // Why the selection is exact: with delta_te >= |l_te - l'_te| for every pair,
 // at least k experts have l >= theta_t (the k-th largest lower bound), so
@@ -163,7 +162,8 @@ router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, 
         }
         return;
     }
-    // expert e: thread t holds rows i = t + 256 j
+    // expert e: thread t holds rows i = t + 256 j (also written out as row e
+    // of the transposed W_r, read by the selection kernel's exact logits)
     __shared__ float sm_max[kPrepThreads / 32], sm_f[kPrepThreads / 32];
     __shared__ double sm_abs[kPrepThreads / 32], sm_sq[kPrepThreads / 32];
     __shared__ float sm_u;
@@ -178,6 +178,8 @@ router_prep_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, 
     }
 #pragma unroll
     for (int j = 0; j < kPrepMaxRows; ++j) {
+        const int i = threadIdx.x + kPrepThreads * j;
+        if (i < d) ws.wt[static_cast<size_t>(e) * d + i] = w[j];
         m = fmaxf(m, fabsf(w[j]));
         sabs += fabs(static_cast<double>(w[j]));
         ssq += static_cast<double>(w[j]) * w[j];
@@ -449,25 +451,36 @@ __device__ __forceinline__ float route_delta(float L, float A_t, float E_t, floa
 }
 
 // ---------------------------------------------------------------------------
-// Threshold: per token (one warp), the k-th largest lower bound L - delta.
+// Selection, one warp per token.
 // ---------------------------------------------------------------------------
 constexpr int kSelWarps = 8;
+constexpr int kSelPer = kMaxExperts / 32;   // experts per lane
+constexpr int kSelXPer = 64;                // x values per lane: d <= 2048
 
 __global__ void __launch_bounds__(kSelWarps * 32)
-router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, int E, int k) {
+router_select_kernel(const uint16_t* __restrict__ x, RouterFastWs ws, const float* __restrict__ b_r, int T,
+                     int d, int E, int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                     int32_t* __restrict__ hist) {
+    __shared__ float rows[kSelWarps][kMaxExperts];
     const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     pdl_launch_dependents();
     pdl_wait();
-    const int t = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
+    const int t = blockIdx.x * kSelWarps + warp;
     if (t >= T) return;
-    const float A = ws.A_t[t], Et = ws.E_t[t], N = ws.N_t[t];
-    constexpr int kPer = kMaxExperts / 32;
-    float lo[kPer], up[kPer];
+    // the token's x: lane p holds elements p, p + 32, ... (chain p)
+    const int steps = d >> 5;
+    float xv[kSelXPer];
+    const uint16_t* xr = x + static_cast<size_t>(t) * d + lane;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
+    for (int m = 0; m < kSelXPer; ++m) xv[m] = m < steps ? bf16_bits_to_float(__ldg(xr + 32 * m)) : 0.0f;
+    // bounds: lower / upper of every expert
+    const float A = ws.A_t[t], Et = ws.E_t[t], N = ws.N_t[t];
+    float lo[kSelPer], up[kSelPer], lw[kSelPer];
+#pragma unroll
+    for (int i = 0; i < kSelPer; ++i) {
         const int e = lane + 32 * i;
-        lo[i] = -INFINITY;
-        up[i] = -INFINITY;
+        lo[i] = up[i] = -INFINITY;
         if (e < E) {
             const float L = ws.L[static_cast<size_t>(t) * E + e];
             const float babs = b_r != nullptr ? fabsf(__ldg(b_r + e)) : 0.0f;
@@ -475,18 +488,15 @@ router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, i
             lo[i] = __fsub_rd(L, dl);
             up[i] = __fadd_ru(L, dl);
         }
+        lw[i] = lo[i];
     }
-    // theta: the k-th largest lower bound (k rounds of a warp arg-max, value
-    // desc, expert asc; the taken entry is removed)
+    // theta: the k-th largest lower bound (k rounds of a warp arg-max)
     float theta = -INFINITY;
-    float lw[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) lw[i] = lo[i];
     for (int j = 0; j < k; ++j) {
         float bv = -INFINITY;
         int bi = 1 << 30;
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
+        for (int i = 0; i < kSelPer; ++i) {
             const int id = lane + 32 * i;
             if (id < E && (lw[i] > bv || (lw[i] == bv && id < bi))) {
                 bv = lw[i];
@@ -503,193 +513,28 @@ router_threshold_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, i
             }
         }
 #pragma unroll
-        for (int i = 0; i < kPer; ++i)
+        for (int i = 0; i < kSelPer; ++i)
             if (lane + 32 * i == bi) lw[i] = -INFINITY;
         theta = bv;
     }
-    // candidates: upper bound >= theta
+    // the candidates' fixed-order logits; the other experts read as -inf
+    for (int e = lane; e < E; e += 32) rows[warp][e] = -INFINITY;
+    __syncwarp();
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        if (32 * i >= E) break;
-        const unsigned m = __ballot_sync(0xffffffffu, lane + 32 * i < E && up[i] >= theta);
-        if (lane == 0) ws.cmask[static_cast<size_t>(t) * ((E + 31) / 32) + i] = m;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Exact logits of the candidate pairs (upper bound >= the token's threshold),
-// in the router's fixed order: lane p runs chain p with fused multiply-add,
-// then the xor butterfly, then the bias.  One CTA per slice of 16 experts
-// (W_r slice in shared memory, rows padded to 17 floats so the 32 lanes'
-// single-float reads of 32 consecutive rows fall in distinct banks) sweeps 64-token
-// tiles; a tile's pairs are listed in shared memory and done up to 128 at a
-// time (16 per warp) while the tile's x rows stream through a ring of six
-// 64-wide K chunks (five in flight).
-// ---------------------------------------------------------------------------
-constexpr int kExES = 16, kExWS = 17, kExTile = 64, kExKc = 64, kExStages = 6, kExWarps = 8;
-constexpr int kExPairsPerWarp = 16;
-constexpr int kExPass = kExWarps * kExPairsPerWarp;
-constexpr int kExChunkBytes = kExTile * kExKc * 2;
-__host__ __device__ constexpr int ex_smem_bytes(int d) {
-    return d * kExWS * 4 + kExStages * kExChunkBytes + kExTile * kExES * 4 + 64;
-}
-
-// barrier of the first two warps (the pair-list builders)
-__device__ __forceinline__ void named_sync_64() { asm volatile("bar.sync 2, 64;" ::: "memory"); }
-
-__global__ void __launch_bounds__(kExWarps * 32, 1)
-router_exact_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
-                    const float* __restrict__ b_r, RouterFastWs ws, int T, int d, int E) {
-    extern __shared__ __align__(16) uint8_t ex_raw[];
-    float* Ws = reinterpret_cast<float*>(ex_raw);
-    uint16_t* xs = reinterpret_cast<uint16_t*>(ex_raw + static_cast<size_t>(d) * kExWS * 4);
-    int* pairs = reinterpret_cast<int*>(ex_raw + static_cast<size_t>(d) * kExWS * 4 + kExStages * kExChunkBytes);
-    int* npairs = pairs + kExTile * kExES;  // [0]: pairs of the tile; [1], [2]: per-warp counts
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int nslices = E / kExES;
-    const int slice = blockIdx.x % nslices;
-    const int cta = blockIdx.x / nslices;
-    const int ctas = gridDim.x / nslices;
-    const int e0 = slice * kExES;
-    pdl_launch_dependents();
-    // the W_r slice (model weights, never written by this library: loaded
-    // before waiting for the previous kernel), one asynchronous 4-byte copy
-    // per element so all of them are in flight at once
-    {
-        const uint32_t ws_base = smem_u32(Ws);
-        for (int idx = threadIdx.x; idx < d * kExES; idx += blockDim.x) {
-            const int i = idx / kExES;
-            const int el = idx % kExES;
-            cp_async_4(ws_base + (i * kExWS + el) * 4, W + static_cast<size_t>(i) * E + e0 + el);
+    for (int i = 0; i < kSelPer; ++i) {
+        unsigned cand = __ballot_sync(0xffffffffu, lane + 32 * i < E && up[i] >= theta);
+        while (cand) {
+            const int e = 32 * i + __ffs(cand) - 1;
+            cand &= cand - 1;
+            const float* wc = ws.wt + static_cast<size_t>(e) * d + lane;
+            float acc = 0.0f;
+#pragma unroll
+            for (int m = 0; m < kSelXPer; ++m)
+                if (m < steps) acc = __fmaf_rn(xv[m], __ldg(wc + 32 * m), acc);
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, m));
+            if (lane == 0) rows[warp][e] = b_r != nullptr ? __fadd_rn(acc, __ldg(b_r + e)) : acc;
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    }
-    pdl_wait();
-    const uint32_t xs_base = smem_u32(xs);
-    const int ntiles = (T + kExTile - 1) / kExTile;
-    const int nkc = d / kExKc;
-    // one K chunk of the tile (64 rows x 128 bytes = 512 pieces of 16 bytes,
-    // two per thread) into ring stage kc % kExStages; every call commits one
-    // group (empty past the last chunk), so wait_group counts stay uniform
-    auto load_chunk = [&](int t0, int kc) {
-        if (kc < nkc) {
-#pragma unroll
-            for (int j = 0; j < (kExChunkBytes / 16) / (kExWarps * 32); ++j) {
-                const int piece = threadIdx.x + j * kExWarps * 32;
-                const int row = piece / (kExKc * 2 / 16);
-                const int col = piece % (kExKc * 2 / 16);
-                const int t = t0 + row;
-                const uint16_t* src = x + static_cast<size_t>(t < T ? t : 0) * d + kc * kExKc + col * 8;
-                cp_async_16(xs_base + (kc % kExStages) * kExChunkBytes + (row * kExKc + col * 8) * 2, src,
-                            t < T ? 16u : 0u);
-            }
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    for (int tile = cta; tile < ntiles; tile += ctas) {
-        const int t0 = tile * kExTile;
-        // (first tile: the W_r slice has landed) the previous tile's pair list
-        // and x buffers are no longer read
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();
-        // the tile's candidate pairs in this slice, in (token, expert) order:
-        // thread tl < 64 takes token t0 + tl's 16 mask bits; the first two warps
-        // scan the counts
-        if (threadIdx.x < kExTile) {
-            const int tl = threadIdx.x;
-            const int t = t0 + tl;
-            uint32_t bits = 0;
-            if (t < T)
-                bits = (ws.cmask[static_cast<size_t>(t) * ((E + 31) / 32) + (e0 >> 5)] >> (e0 & 31)) &
-                       ((1u << kExES) - 1u);
-            const int cnt = __popc(bits);
-            int inc = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int nb = __shfl_up_sync(0xffffffffu, inc, o);
-                if ((tl & 31) >= o) inc += nb;
-            }
-            if ((tl & 31) == 31) npairs[1 + (tl >> 5)] = inc;  // per-warp totals
-            __syncwarp();
-            named_sync_64();
-            int base = inc - cnt + (tl >= 32 ? npairs[1] : 0);
-            while (bits) {
-                const int el = __ffs(bits) - 1;
-                bits &= bits - 1;
-                pairs[base++] = tl * kExES + el;
-            }
-            if (tl == kExTile - 1) npairs[0] = base;
-        }
-        __syncthreads();
-        const int np = npairs[0];
-        for (int base = 0; base < np; base += kExPass) {
-            int tl[kExPairsPerWarp], el[kExPairsPerWarp];
-            bool on[kExPairsPerWarp];
-            float acc[kExPairsPerWarp];
-#pragma unroll
-            for (int j = 0; j < kExPairsPerWarp; ++j) {
-                const int pi = base + warp * kExPairsPerWarp + j;
-                on[j] = pi < np;
-                const int code = on[j] ? pairs[pi] : 0;
-                tl[j] = code / kExES;
-                el[j] = code % kExES;
-                acc[j] = 0.0f;
-            }
-            __syncthreads();  // every thread has read the ring's previous contents
-#pragma unroll
-            for (int kc = 0; kc < kExStages - 1; ++kc) load_chunk(t0, kc);
-            for (int kc = 0; kc < nkc; ++kc) {
-                load_chunk(t0, kc + kExStages - 1);
-                asm volatile("cp.async.wait_group %0;" ::"n"(kExStages - 1) : "memory");
-                __syncthreads();
-                const uint16_t* xb = xs + (kc % kExStages) * (kExTile * kExKc);
-#pragma unroll
-                for (int s = 0; s < kExKc / 32; ++s) {
-                    const int il = 32 * s + lane;             // chain lane: i = kc*64 + il
-                    const float* wrow = Ws + (kc * kExKc + il) * kExWS;
-#pragma unroll
-                    for (int j = 0; j < kExPairsPerWarp; ++j)
-                        if (on[j])
-                            acc[j] = __fmaf_rn(bf16_bits_to_float(xb[tl[j] * kExKc + il]), wrow[el[j]], acc[j]);
-                }
-                __syncthreads();  // the stage is refilled by a later chunk's copies
-            }
-#pragma unroll
-            for (int j = 0; j < kExPairsPerWarp; ++j) {
-                float v = acc[j];
-#pragma unroll
-                for (int m = 16; m >= 1; m >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, m));
-                if (on[j] && lane == 0) {
-                    const int e = e0 + el[j];
-                    const float l = b_r != nullptr ? __fadd_rn(v, __ldg(b_r + e)) : v;
-                    ws.exact[static_cast<size_t>(t0 + tl[j]) * E + e] = l;
-                }
-            }
-        }
-    }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-
-// ---------------------------------------------------------------------------
-// Selection: per token (one warp) the candidates' exact logits (others -inf)
-// go through the same warp top-k as the dense router: top-k by (logit desc,
-// id asc), softmax over the k, per-group histogram.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kSelWarps * 32)
-router_select_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, int E, int k,
-                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                     int32_t* __restrict__ hist) {
-    __shared__ float rows[kSelWarps][kMaxExperts];
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    pdl_launch_dependents();
-    pdl_wait();
-    const int t = blockIdx.x * kSelWarps + warp;
-    if (t >= T) return;
-    for (int e = lane; e < E; e += 32) {
-        const uint32_t m = ws.cmask[static_cast<size_t>(t) * ((E + 31) / 32) + (e >> 5)];
-        rows[warp][e] = (m >> (e & 31)) & 1u ? ws.exact[static_cast<size_t>(t) * E + e] : -INFINITY;
     }
     __syncwarp();
     int my_id;
@@ -705,15 +550,14 @@ router_select_kernel(RouterFastWs ws, const float* __restrict__ b_r, int T, int 
 }  // namespace
 
 bool router_fast_supported(int T, int d, int E) {
-    return T >= kFastRouterMinT && E % kExES == 0 && E <= kMaxExperts && d % 128 == 0 &&
-           d <= kPrepThreads * kPrepMaxRows && d <= 8 * 32 * kPrepMaxVec && ex_smem_bytes(d) <= 227 * 1024;
+    return T >= kFastRouterMinT && E % 8 == 0 && E <= kMaxExperts && d % 128 == 0 &&
+           d <= kPrepThreads * kPrepMaxRows && d <= 8 * 32 * kPrepMaxVec && d <= 32 * kSelXPer;
 }
 
 size_t router_fast_ws_bytes(int T, int d, int E) {
     auto r = [](size_t v) { return (v + 255) / 256 * 256; };
     const size_t t = static_cast<size_t>(T), dd = static_cast<size_t>(d), e = static_cast<size_t>(E);
-    return 2 * r(t * dd) + 2 * r(e * dd) + 4 * r(t * 4) + r(t * ((e + 31) / 32) * 4) + 4 * r(e * 4) +
-           r(t * e * 4);
+    return 2 * r(t * dd) + 2 * r(e * dd) + 4 * r(t * 4) + 4 * r(e * 4) + r(e * dd * 4);
 }
 
 RouterFastWs router_fast_ws(uint8_t* base, float* L, int T, int d, int E) {
@@ -734,12 +578,11 @@ RouterFastWs router_fast_ws(uint8_t* base, float* L, int T, int d, int E) {
     w.E_t = reinterpret_cast<float*>(take(t * 4));
     w.A_t = reinterpret_cast<float*>(take(t * 4));
     w.N_t = reinterpret_cast<float*>(take(t * 4));
-    w.cmask = reinterpret_cast<uint32_t*>(take(t * ((e + 31) / 32) * 4));
     w.u_e = reinterpret_cast<float*>(take(e * 4));
     w.F_e = reinterpret_cast<float*>(take(e * 4));
     w.B_e = reinterpret_cast<float*>(take(e * 4));
     w.Wn_e = reinterpret_cast<float*>(take(e * 4));
-    w.exact = reinterpret_cast<float*>(take(t * e * 4));
+    w.wt = reinterpret_cast<float*>(take(e * dd * 4));
     w.L = L;
     return w;
 }
@@ -753,8 +596,6 @@ static cudaError_t router_fast_setup(int* num_sms) {
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (ready[dev].load(std::memory_order_acquire) == 0) {
         e = cudaFuncSetAttribute(router_approx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kApSmem);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(router_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         int n = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -798,16 +639,7 @@ cudaError_t launch_router_fast(const uint16_t* x, const float* W, const float* b
                    kApSmem, st, a);
     if (e != cudaSuccess) return e;
     const int sel_grid = (T + kSelWarps - 1) / kSelWarps;
-    e = launch_pdl(router_threshold_kernel, dim3(sel_grid), dim3(kSelWarps * 32), 0, st, ws, b, T, E, k);
-    if (e != cudaSuccess) return e;
-    const int nslices = E / kExES;
-    const int ntiles = (T + kExTile - 1) / kExTile;
-    int per_slice = std::max(1, num_sms / nslices);
-    per_slice = std::min(per_slice, ntiles);
-    e = launch_pdl(router_exact_kernel, dim3(nslices * per_slice), dim3(kExWarps * 32), ex_smem_bytes(d), st,
-                   x, W, b, ws, T, d, E);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(router_select_kernel, dim3(sel_grid), dim3(kSelWarps * 32), 0, st, ws, b, T, E, k,
+    return launch_pdl(router_select_kernel, dim3(sel_grid), dim3(kSelWarps * 32), 0, st, x, ws, b, T, d, E, k,
                       topk_idx, topk_w, hist);
 }
 
