@@ -39,6 +39,17 @@ KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, do
 KERNELS_PER_STEP_DECODE = 1  # one persistent kernel (batches of at most 8 tokens)
 
 
+def build_library():
+    """Compile libmoe_b200.so when its sources are newer (build.py by path:
+    the package refuses to import until the library exists)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "moe_libbuild", os.path.join(ROOT, "int4_expert_grouped_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -291,8 +302,7 @@ def run_ours(args, name):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    from int4_expert_grouped_b200 import build
-    build.build()
+    build_library()
     from int4_expert_grouped_b200.layer import MoeLayer, bf16_tensor
 
     shape, seed, zipf = mi.WORKLOADS[name]

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "libmoe_b200.so is not built; run `python -m int4_expert_grouped_b200.build` "
+        "libmoe_b200.so is not built; run `python int4_expert_grouped_b200/build.py` "
         "(needs nvcc with sm_100a support)")
 
 _lib = ctypes.CDLL(LIB_PATH)

@@ -456,24 +456,28 @@ __device__ __forceinline__ float route_delta(float L, float A_t, float E_t, floa
 constexpr int kSelWarps = 8;
 constexpr int kSelPer = kMaxExperts / 32;   // experts per lane
 constexpr int kSelXPer = 64;                // x values per lane: d <= 2048
+constexpr int kSelChunk = 16;               // column loads in flight per candidate
 
 __global__ void __launch_bounds__(kSelWarps * 32)
 router_select_kernel(const uint16_t* __restrict__ x, RouterFastWs ws, const float* __restrict__ b_r, int T,
                      int d, int E, int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                      int32_t* __restrict__ hist) {
     __shared__ float rows[kSelWarps][kMaxExperts];
+    __shared__ __align__(16) uint16_t xsm[kSelWarps][32 * kSelXPer];
+    __shared__ int clist[kSelWarps][kMaxExperts];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     pdl_launch_dependents();
     pdl_wait();
     const int t = blockIdx.x * kSelWarps + warp;
     if (t >= T) return;
-    // the token's x: lane p holds elements p, p + 32, ... (chain p)
+    // the token's x row into shared memory (16-byte pieces)
     const int steps = d >> 5;
-    float xv[kSelXPer];
-    const uint16_t* xr = x + static_cast<size_t>(t) * d + lane;
-#pragma unroll
-    for (int m = 0; m < kSelXPer; ++m) xv[m] = m < steps ? bf16_bits_to_float(__ldg(xr + 32 * m)) : 0.0f;
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+        uint4* dst = reinterpret_cast<uint4*>(xsm[warp]);
+        for (int v = lane; v < d / 8; v += 32) dst[v] = __ldg(src + v);
+    }
     // bounds: lower / upper of every expert
     const float A = ws.A_t[t], Et = ws.E_t[t], N = ws.N_t[t];
     float lo[kSelPer], up[kSelPer], lw[kSelPer];
@@ -519,21 +523,55 @@ router_select_kernel(const uint16_t* __restrict__ x, RouterFastWs ws, const floa
     }
     // the candidates' fixed-order logits; the other experts read as -inf
     for (int e = lane; e < E; e += 32) rows[warp][e] = -INFINITY;
-    __syncwarp();
+    // candidate list (ascending id) in this warp's shared list
+    int nc = 0;
 #pragma unroll
     for (int i = 0; i < kSelPer; ++i) {
-        unsigned cand = __ballot_sync(0xffffffffu, lane + 32 * i < E && up[i] >= theta);
-        while (cand) {
-            const int e = 32 * i + __ffs(cand) - 1;
-            cand &= cand - 1;
-            const float* wc = ws.wt + static_cast<size_t>(e) * d + lane;
-            float acc = 0.0f;
+        const unsigned cand = __ballot_sync(0xffffffffu, lane + 32 * i < E && up[i] >= theta);
+        if ((cand >> lane) & 1u) clist[warp][nc + __popc(cand & ((1u << lane) - 1u))] = 32 * i + lane;
+        nc += __popc(cand);
+    }
+    __syncwarp();  // the x row and the list are in shared memory
+    // two candidates at a time; lane p runs chain p = fma(x[p + 32 m],
+    // W_r[p + 32 m][e], chain p) in ascending m for each, with the column's
+    // loads issued sixteen at a time ahead of their multiply-adds
+    const uint16_t* xw = xsm[warp] + lane;
+    for (int c0 = 0; c0 < nc; c0 += 2) {
+        const int e0 = clist[warp][c0];
+        const int e1 = c0 + 1 < nc ? clist[warp][c0 + 1] : e0;
+        const float* w0 = ws.wt + static_cast<size_t>(e0) * d + lane;
+        const float* w1 = ws.wt + static_cast<size_t>(e1) * d + lane;
+        float a0 = 0.0f, a1 = 0.0f;
+        for (int m0 = 0; m0 < steps; m0 += kSelChunk) {
+            float v0[kSelChunk], v1[kSelChunk];
+            if (m0 + kSelChunk <= steps) {
 #pragma unroll
-            for (int m = 0; m < kSelXPer; ++m)
-                if (m < steps) acc = __fmaf_rn(xv[m], __ldg(wc + 32 * m), acc);
+                for (int j = 0; j < kSelChunk; ++j) {
+                    v0[j] = __ldg(w0 + 32 * (m0 + j));
+                    v1[j] = __ldg(w1 + 32 * (m0 + j));
+                }
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, m));
-            if (lane == 0) rows[warp][e] = b_r != nullptr ? __fadd_rn(acc, __ldg(b_r + e)) : acc;
+                for (int j = 0; j < kSelChunk; ++j) {
+                    const float xv = bf16_bits_to_float(xw[32 * (m0 + j)]);
+                    a0 = __fmaf_rn(xv, v0[j], a0);
+                    a1 = __fmaf_rn(xv, v1[j], a1);
+                }
+            } else {
+                for (int m = m0; m < steps; ++m) {
+                    const float xv = bf16_bits_to_float(xw[32 * m]);
+                    a0 = __fmaf_rn(xv, __ldg(w0 + 32 * m), a0);
+                    a1 = __fmaf_rn(xv, __ldg(w1 + 32 * m), a1);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            a0 = __fadd_rn(a0, __shfl_xor_sync(0xffffffffu, a0, m));
+            a1 = __fadd_rn(a1, __shfl_xor_sync(0xffffffffu, a1, m));
+        }
+        if (lane == 0) {
+            rows[warp][e0] = b_r != nullptr ? __fadd_rn(a0, __ldg(b_r + e0)) : a0;
+            rows[warp][e1] = b_r != nullptr ? __fadd_rn(a1, __ldg(b_r + e1)) : a1;
         }
     }
     __syncwarp();

@@ -11,9 +11,7 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 
 
 @pytest.fixture(scope="module")
-def moe():
-    from int4_expert_grouped_b200 import build
-    build.build()
+def moe(built_library):
     import int4_expert_grouped_b200 as m
     return m
 

@@ -24,10 +24,8 @@ W_REL = 1e-6          # routing weights
 
 
 @pytest.fixture(scope="module")
-def moe():
+def moe(built_library):
     assert torch.cuda.is_available(), "the gpu tests need a GPU"
-    from int4_expert_grouped_b200 import build
-    build.build()
     import int4_expert_grouped_b200 as m
     from int4_expert_grouped_b200.layer import MoeLayer, bf16_tensor
     m.MoeLayer, m.bf16_tensor = MoeLayer, bf16_tensor

@@ -17,10 +17,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")
-def env():
+def env(built_library):
     assert torch.cuda.is_available(), "the gpu tests need a GPU"
-    from int4_expert_grouped_b200 import build
-    build.build()
     import int4_expert_grouped_b200 as m
     from int4_expert_grouped_b200.layer import MoeLayer, bf16_tensor
     return m, MoeLayer, bf16_tensor
