@@ -35,6 +35,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer prefill tokens/s (int4 fused grouped GEMM) and % of roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+L2_BYTES = 126 << 20
 KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, down GEMM, combine
 KERNELS_PER_STEP_DECODE = 1  # one persistent kernel (batches of at most 8 tokens)
 
@@ -79,6 +80,45 @@ def algorithmic(s, counts):
     return dict(touched=touched, per_expert=per_expert, flops_gateup=flops_gateup,
                 flops_down=flops_down, flops=flops_gateup + flops_down, bytes=bytes_layer,
                 bytes_gateup=bytes_gateup)
+
+
+class ColdL2:
+    """Keeps every timed step's weights cold in L2.
+
+    Layers that touch more weight bytes than L2 holds get a 256 MiB write
+    before each step (outside the step's events).  Layers that touch few
+    (the small batches: 8 experts, 21 MB at one token) instead rotate over R
+    copies of the packed weights and W_r, R - 1 >= 2 x L2 / touched bytes, so
+    that each step reads a copy whose bytes left L2 R - 1 steps ago; no
+    other kernel runs between two steps."""
+
+    def __init__(self, layer, work, flush):
+        import torch
+        self.layer, self.flush = layer, flush
+        self.packs = self.wrs = None
+        touched = work["bytes"]
+        if 4 * work["touched"] <= layer.E and touched < L2_BYTES:
+            r = 1 + -(-2 * L2_BYTES // touched)
+            self.packs = [layer.packed] + [layer.packed.clone() for _ in range(r - 1)]
+            self.wrs = [layer.w_r] + [layer.w_r.clone() for _ in range(r - 1)]
+            torch.cuda.synchronize()
+            self.desc = ("weights rotated over %d copies of the packed experts and W_r (%.1f GB), "
+                         "each step's %.1f MB cold in L2; no flush kernel" %
+                         (r, r * layer.packed.numel() / 1e9, touched / 1e6))
+        else:
+            self.desc = "flushed between steps (256 MiB write outside the step events)"
+
+    def before(self, i):
+        if self.packs is None:
+            self.flush.fill_(i & 0xFF)
+        else:
+            self.layer.packed = self.packs[i % len(self.packs)]
+            self.layer.w_r = self.wrs[i % len(self.wrs)]
+
+    def release(self):
+        if self.packs is not None:
+            self.layer.packed, self.layer.w_r = self.packs[0], self.wrs[0]
+            self.packs = self.wrs = None
 
 
 class ClockSampler:
@@ -193,8 +233,8 @@ def layer_launches(layer, T):
     return KERNELS_PER_STEP_DECODE if layer.plan.forward_path(T) == 1 else KERNELS_PER_STEP
 
 
-def time_layer(layer, x, y, K, repeats, flush, stream, world=1):
-    """K layer calls with L2 flushed before each, `repeats` times.
+def time_layer(layer, x, y, K, repeats, cold, stream, world=1):
+    """K layer calls with the weights cold in L2 (`cold`), `repeats` times.
 
     Each call records the five stage events of moe_forward_timed on the
     launching stream; returns per-repeat mean step times (ms, max over ranks)
@@ -212,7 +252,7 @@ def time_layer(layer, x, y, K, repeats, flush, stream, world=1):
             dist.barrier()
         torch.cuda.synchronize()
         for i in range(K):
-            flush.fill_(i & 0xFF)  # evict L2 between steps (outside the step's events)
+            cold.before(i)  # outside the step's events
             layer.forward(x, y, events=evs[i])
         torch.cuda.synchronize()
         if world > 1:
@@ -247,7 +287,7 @@ def layer_roofline(work, ms, peaks):
 
 def other_configs(args, main_name, flush, stream, peaks):
     """The other layer configurations, each timed the same way (median of
-    repeats of K steps, L2 flushed before each step), for the same JSON line."""
+    repeats of K steps, weights cold in L2 as ColdL2 says), for the same JSON line."""
     import torch
     from int4_expert_grouped_b200.layer import MoeLayer, bf16_tensor
     out = {}
@@ -267,19 +307,21 @@ def other_configs(args, main_name, flush, stream, peaks):
         if code != 0:
             raise RuntimeError("%s: device status %d (%d)" % (name, code, detail))
         work = algorithmic(s, bufs["counts"].cpu().numpy())
-        for _ in range(3):
-            flush.fill_(1)
+        cold = ColdL2(layer, work, flush)
+        for i in range(3):
+            cold.before(i)
             layer.forward(x, y)
         torch.cuda.synchronize()
         K = args.steps if s.T < 32768 else max(3, args.steps // 2)
         clocks = ClockSampler(torch.cuda.current_device())
         clocks.start()
-        reps, ms, stages = time_layer(layer, x, y, K, args.repeats, flush, stream)
+        reps, ms, stages = time_layer(layer, x, y, K, args.repeats, cold, stream)
         clk = clocks.stop()
+        cold.release()
         roof = layer_roofline(work, ms, peaks)
         entry = {"workload": workload_desc(name, s, *mi.WORKLOADS[name][1:]), "tokens": s.T,
                  "ms_per_step": ms, "repeats_ms": reps, "tokens_per_s": s.T / (ms * 1e-3),
-                 "layer_roofline": roof, "stages_ms": stages, "steps": K,
+                 "layer_roofline": roof, "stages_ms": stages, "steps": K, "l2": cold.desc,
                  "gpu_launches_per_step": layer_launches(layer, s.T), "clocks": clk,
                  "kernels": "small-batch (decode)" if layer.plan.forward_path(s.T) == 1 else "batched"}
         if roof["bound"] == "hbm":
@@ -333,16 +375,18 @@ def run_ours(args, name):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
+    cold = ColdL2(layer, work, flush)
+    for i in range(max(args.warmup, 3)):
+        cold.before(i)
         layer.forward(x, y)
     torch.cuda.synchronize()
 
     K = args.steps
     clocks = ClockSampler(local)
     clocks.start()
-    reps, ms_per_step, stage_ms = time_layer(layer, x, y, K, args.repeats, flush, stream, world)
+    reps, ms_per_step, stage_ms = time_layer(layer, x, y, K, args.repeats, cold, stream, world)
     clk = clocks.stop()
+    cold.release()
     value = world * s.T / (ms_per_step * 1e-3)
 
     # end to end through the host-buffer entry point (pinned host memory)
@@ -376,7 +420,7 @@ def run_ours(args, name):
     tensor_bound = work["flops_gateup"] / (peaks["bf16_tflops"] * 1e12) >= \
         work["bytes_gateup"] / (peaks["hbm_gbs"] * 1e9)
     if tensor_bound:
-        # the kernel is timed alone between L2 flushes, well under a second:
+        # the kernel is timed alone with cold weights, well under a second:
         # the burst bf16 peak is its denominator; the sustained one is reported too
         achieved = work["flops_gateup"] / t_gu / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
@@ -403,7 +447,7 @@ def run_ours(args, name):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(name, s, seed, zipf), "tokens_per_gpu": s.T,
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "flushed between steps (256 MiB write outside the step events)",
+                   "l2": cold.desc,
                    "repeats": "median of %d repeats of %d steps" % (args.repeats, K)},
         "pct_of_layer_roofline": 100.0 * lroof["frac"],
         "layer_roofline": lroof,
