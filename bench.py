@@ -36,8 +36,11 @@ import moe_inputs as mi  # noqa: E402
 METRIC = "MoE-layer prefill tokens/s (int4 fused grouped GEMM) and % of roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 L2_BYTES = 126 << 20
-KERNELS_PER_STEP = 8  # logits, top-k, scan, scatter, dispatch, gate/up GEMM, down GEMM, combine
-KERNELS_PER_STEP_DECODE = 1  # one persistent kernel (batches of at most 8 tokens)
+# kernels one layer call launches, by moe_forward_path: fp32 router (logits,
+# top-k), scan, scatter, dispatch, gate/up GEMM, down GEMM, combine; the
+# small-batch kernel; the int8 tensor-core router (prep, approximate logits,
+# selection) and the rest as for the first
+KERNELS_PER_PATH = {0: 8, 1: 1, 2: 9}
 
 
 def build_library():
@@ -230,48 +233,64 @@ def run_reference(args, name):
 
 def layer_launches(layer, T):
     """Kernels one layer call launches (the library's launch sequence)."""
-    return KERNELS_PER_STEP_DECODE if layer.plan.forward_path(T) == 1 else KERNELS_PER_STEP
+    return KERNELS_PER_PATH[layer.plan.forward_path(T)]
 
 
 def time_layer(layer, x, y, K, repeats, cold, stream, world=1):
     """K layer calls with the weights cold in L2 (`cold`), `repeats` times.
 
-    Each call records the five stage events of moe_forward_timed on the
-    launching stream; returns per-repeat mean step times (ms, max over ranks)
-    and the mean stage times of the median repeat."""
+    Each call is bracketed by two CUDA events on the launching stream (the
+    L2 flush, when there is one, runs before the first); returns the
+    per-repeat mean step times (ms, max over ranks) and their median.  The
+    per-stage split comes from a separate pass (stage_times): the four events
+    moe_forward_timed records inside a call add their own gaps, a few us
+    each, which the step time must not carry."""
     import torch
     import torch.distributed as dist
     reps = []
     for _ in range(repeats):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-        for row in evs:
-            for e in row:
-                e.record(stream)  # create the handles before they are passed to the C API
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         for i in range(K):
             cold.before(i)  # outside the step's events
-            layer.forward(x, y, events=evs[i])
+            evs[i][0].record(stream)
+            layer.forward(x, y)
+            evs[i][1].record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        total = float(sum(r[0].elapsed_time(r[4]) for r in evs))
+        total = float(sum(r[0].elapsed_time(r[1]) for r in evs))
         if world > 1:
             t = torch.tensor([total], device="cuda")
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             total = float(t.item())
-        stages = {
-            "routing": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
-            "gate_up_gemm": float(np.mean([r[1].elapsed_time(r[2]) for r in evs])),
-            "down_gemm": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
-            "combine": float(np.mean([r[3].elapsed_time(r[4]) for r in evs])),
-        }
-        reps.append((total / K, stages))
-    order = sorted(range(repeats), key=lambda i: reps[i][0])
-    med = reps[order[repeats // 2]]
-    return [r[0] for r in reps], med[0], med[1]
+        reps.append(total / K)
+    return reps, sorted(reps)[repeats // 2]
+
+
+def stage_times(layer, x, y, K, cold, stream):
+    """Mean stage times (ms) over K calls of moe_forward_timed, which records
+    events after routing, after each GEMM and after the combine.  The
+    small-batch kernel is one launch: its whole time is under "routing"."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)  # create the handles before they are passed to the C API
+    torch.cuda.synchronize()
+    for i in range(K):
+        cold.before(i)
+        layer.forward(x, y, events=evs[i])
+    torch.cuda.synchronize()
+    return {
+        "routing": float(np.mean([r[0].elapsed_time(r[1]) for r in evs])),
+        "gate_up_gemm": float(np.mean([r[1].elapsed_time(r[2]) for r in evs])),
+        "down_gemm": float(np.mean([r[2].elapsed_time(r[3]) for r in evs])),
+        "combine": float(np.mean([r[3].elapsed_time(r[4]) for r in evs])),
+    }
 
 
 def layer_roofline(work, ms, peaks):
@@ -315,8 +334,9 @@ def other_configs(args, main_name, flush, stream, peaks):
         K = args.steps if s.T < 32768 else max(3, args.steps // 2)
         clocks = ClockSampler(torch.cuda.current_device())
         clocks.start()
-        reps, ms, stages = time_layer(layer, x, y, K, args.repeats, cold, stream)
+        reps, ms = time_layer(layer, x, y, K, args.repeats, cold, stream)
         clk = clocks.stop()
+        stages = stage_times(layer, x, y, K, cold, stream)
         cold.release()
         roof = layer_roofline(work, ms, peaks)
         entry = {"workload": workload_desc(name, s, *mi.WORKLOADS[name][1:]), "tokens": s.T,
@@ -384,8 +404,9 @@ def run_ours(args, name):
     K = args.steps
     clocks = ClockSampler(local)
     clocks.start()
-    reps, ms_per_step, stage_ms = time_layer(layer, x, y, K, args.repeats, cold, stream, world)
+    reps, ms_per_step = time_layer(layer, x, y, K, args.repeats, cold, stream, world)
     clk = clocks.stop()
+    stage_ms = stage_times(layer, x, y, K, cold, stream)
     cold.release()
     value = world * s.T / (ms_per_step * 1e-3)
 
@@ -413,26 +434,32 @@ def run_ours(args, name):
         raise RuntimeError("device status %d (%d) after timing" % (code, detail))
 
     peaks = load_peaks()
-    t_gu = stage_ms["gate_up_gemm"] * 1e-3
     lroof = layer_roofline(work, ms_per_step, peaks)
     decode = layer.plan.forward_path(s.T) == 1
-    gu_kernel = "decode expert kernel" if decode else "grouped_gemm_kernel<gate/up>"
-    tensor_bound = work["flops_gateup"] / (peaks["bf16_tflops"] * 1e12) >= \
-        work["bytes_gateup"] / (peaks["hbm_gbs"] * 1e9)
-    if tensor_bound:
-        # the kernel is timed alone with cold weights, well under a second:
+    if decode:
+        # one launch does the whole layer: its bytes are the touched experts'
+        # weights, W_r, x and y; its time is the step's
+        achieved = (work["bytes"] + 4 * s.d * s.E) / (ms_per_step * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "decode_layer_kernel", "peak_kind": "HBM copy, %s" % peaks["source"]}
+    elif work["flops_gateup"] / (peaks["bf16_tflops"] * 1e12) >= \
+            work["bytes_gateup"] / (peaks["hbm_gbs"] * 1e9):
+        # the gate/up GEMM, timed alone with cold weights, well under a second:
         # the burst bf16 peak is its denominator; the sustained one is reported too
+        t_gu = stage_ms["gate_up_gemm"] * 1e-3
         achieved = work["flops_gateup"] / t_gu / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "traffic": TRAFFIC_GATEUP.get(name), "kernel": gu_kernel,
+                "traffic": TRAFFIC_GATEUP.get(name), "kernel": "grouped_gemm_kernel<gate/up>",
                 "peak_kind": "bf16 burst, %s" % peaks["source"],
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
     else:
+        t_gu = stage_ms["gate_up_gemm"] * 1e-3
         achieved = work["bytes_gateup"] / t_gu / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": TRAFFIC_GATEUP.get(name),
-                "kernel": gu_kernel, "peak_kind": "HBM copy, %s" % peaks["source"]}
+                "kernel": "grouped_gemm_kernel<gate/up>", "peak_kind": "HBM copy, %s" % peaks["source"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -272,12 +272,19 @@ MOE_API moe_status_t moe_read_status(const void *ws, int32_t *code, int32_t *det
                              int32_t clear, void *stream);
 
 /*
- * Which kernels moe_forward runs at batch T for this plan: 1 for the
- * small-batch (decode) kernels, which stream the selected experts' weights
- * (wpnews page "Perplexity Lily: 1.35x Faster Local AI Than MLX on Mac",
- * section "Why MLX Falls Behind": prefill and decode are separate
- * workloads), 0 for the batched grouped-GEMM kernels, -1 if plan is NULL or
- * T is outside 0..T_max.  Host only; launches nothing.
+ * Which kernels moe_forward runs at batch T for this plan:
+ *   1  the small-batch (decode) kernel, one launch, which streams the
+ *      selected experts' weights (wpnews page "Perplexity Lily: 1.35x Faster
+ *      Local AI Than MLX on Mac", section "Why MLX Falls Behind": prefill and
+ *      decode are separate workloads);
+ *   0  the batched grouped-GEMM kernels with the fp32 router: eight launches
+ *      (router logits, top-k, scan, scatter, dispatch, gate/up GEMM, down
+ *      GEMM, combine);
+ *   2  the batched kernels with the int8 tensor-core router and its exact
+ *      recheck (T >= 1024): nine launches (router prep, approximate logits,
+ *      selection, then as for 0 from the scan on);
+ *  -1  plan is NULL or T is outside 0..T_max.
+ * All three give the same routing results.  Host only; launches nothing.
  */
 MOE_API int moe_forward_path(const moe_plan_t *plan, int32_t T);
 

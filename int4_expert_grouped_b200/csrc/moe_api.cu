@@ -415,7 +415,8 @@ moe_status_t moe_forward_host(const moe_plan_t* plan, int32_t T, const uint16_t*
 
 int moe_forward_path(const moe_plan_t* plan, int32_t T) {
     if (plan == nullptr || T < 0 || T > plan->s.T_max) return -1;
-    return moe::decode_supported(plan->s, T) ? 1 : 0;
+    if (moe::decode_supported(plan->s, T)) return 1;
+    return moe::router_fast_supported(T, plan->s.d, plan->s.E) ? 2 : 0;
 }
 
 moe_status_t moe_read_status(const void* ws, int32_t* code, int32_t* detail, int32_t clear,

@@ -65,18 +65,21 @@ constexpr int kDecComputeWarps = 8;
 constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;  // + one producer warp
 constexpr int kDecProducerWarp = kDecComputeWarps;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
-constexpr int kDecStages = 16;
-// One stage = two 64-wide K chunks of a slice's 64 gate and 64 up rows (two
-// consecutive half-blocks, one bulk copy), or two down blocks (128 rows x
-// 64 K each): 2 * half_block_bytes(group) bytes.
-constexpr int kDecStageBytes = 2 * half_block_bytes(32);
+constexpr int kDecStages = 8;
+// One stage = four 64-wide K chunks of a slice's 64 gate and 64 up rows (four
+// consecutive half-blocks), or up to four down blocks (128 rows x 64 K each;
+// a slice's blocks are consecutive over the output tiles): one bulk copy of
+// at most 4 * half_block_bytes(group) bytes.  Copies of 16 KB and more keep
+// the per-SM copy rate near its maximum; 4.6 KB copies ran at half of it.
+constexpr int kDecChunks = 4;
+constexpr int kDecStageBytes = kDecChunks * half_block_bytes(32);
 constexpr int kDecMaxAssign = 64;                          // T * k the path takes
 constexpr int kDecSlice = 64;                              // features per unit
 constexpr int kDecMaxSlices = 32;                          // f / 64
 constexpr int kDecMaxNTd = 64;                             // d / 128
 constexpr int kDecHStride = kDecSlice + 32;                // h row stride (elements) in shared memory
 constexpr int kDecRowTiles = kDecSlice / 8;                // 16-row MMA tiles of a slice: 8 gate + 8 up rows each
-static_assert(kDecStages % kDecComputeWarps == 0, "a ring slot is always used by the same compute warp");
+static_assert(kDecRowTiles == kDecComputeWarps, "compute warp w owns MMA row tile w of every stage");
 constexpr int kDecWRows = 256;                             // W_r rows per tensor load (box limit)
 constexpr uint32_t kDecMagic0 = 0x4D6F4544u, kDecMagic1 = 0x53796E63u;
 
@@ -351,7 +354,7 @@ __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
 
 // Layout of the dynamic shared memory (byte offsets; the base is 1024-aligned).
 struct DecSmem {
-    int ring, x, xsum, h, hsum, lg, red, route, bars, total;
+    int ring, x, xsum, h, hsum, lg, route, bars, total;
 };
 __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     DecSmem L;
@@ -367,7 +370,6 @@ __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     L.h = take(kDecodeMaxT * kDecHStride * 2);
     L.hsum = take(kDecodeMaxT * (kDecSlice / 32) * 4);
     L.lg = take(T * E * 4);
-    L.red = take(kDecComputeWarps / 2 * kDecRowTiles * 4 * 32 * 4);  // gate/up partial sums, half the warps
     L.route = take(static_cast<int>(sizeof(DecRoute)));
     L.bars = take((2 * kDecStages + 1) * 8);
     L.total = o + 1024;  // + slack to align the base
@@ -379,7 +381,7 @@ struct DecParams {
     const uint16_t* x;
     const float* b_r;
     const uint8_t* wgu;   // packed gate/up blocks [E][f/128][d/64][bb_gu]
-    const uint8_t* wdn;   // packed down blocks [E][d/128][f/64][bb_dn]
+    const uint8_t* wdn;   // packed down blocks [E][f/64][d/128][bb_dn]
     int bb_gu, bb_dn;
     int32_t *topk_idx, *counts, *offsets, *sorted_assign, *pos, *block_offsets, *block_map,
         *num_blocks;
@@ -465,7 +467,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     if (tid == 0) {
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(empty(s), 1);  // one compute warp uses each stage
+            mbar_init(empty(s), kDecComputeWarps);  // every compute warp uses every stage
         }
         mbar_init(wbar, 1);
         R.abort_local = 0;
@@ -599,6 +601,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     const int NT = f / 128, KC = d / kKChunk, NTd = d / 128, KCd = f / kKChunk;
     const int S = f / kDecSlice;
     const int u_total = nb * S;
+    const int NSd = (NTd + kDecChunks - 1) / kDecChunks;  // down stages per unit
 
     if (warp == kDecProducerWarp) {
         // the whole warp runs the loop; one elected lane issues the copies
@@ -610,7 +613,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int e = R.blk_e[b];
             const int j = fs >> 1, hh = fs & 1;  // 128-feature tile, half of it
             const uint8_t* gsrc = p.wgu + ((static_cast<size_t>(e) * NT + j) * 2 + hh) * KC * p.bb_dn;
-            for (int st = 0; st < KC / 2 + NTd / 2; ++st, ++q) {
+            const uint8_t* dsrc = p.wdn + (static_cast<size_t>(e) * KCd + fs) * NTd * p.bb_dn;
+            for (int st = 0; st < KC / kDecChunks + NSd; ++st, ++q) {
                 const int slot = q % kDecStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(empty(slot), ((q / kDecStages) & 1) ^ 1, &R.abort_local))) {
                     ok = false;
@@ -618,20 +622,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 }
                 if (elect_one()) {
                     const uint32_t dst = smem_u32(ring + slot * kDecStageBytes);
-                    mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(2 * p.bb_dn));
-                    if (st < KC / 2) {
-                        // K chunks 2 st, 2 st + 1 of the slice: consecutive half-blocks
-                        bulk_copy_g2s(dst, gsrc + static_cast<size_t>(2 * st) * p.bb_dn,
-                                      static_cast<uint32_t>(2 * p.bb_dn), full(slot));
-                    } else {
-                        // down blocks (expert, output tiles jd, jd + 1, K chunk fs)
-                        const int jd = 2 * (st - KC / 2);
-                        for (int h = 0; h < 2; ++h) {
-                            const uint8_t* blk =
-                                p.wdn + ((static_cast<size_t>(e) * NTd + jd + h) * KCd + fs) * p.bb_dn;
-                            bulk_copy_g2s(dst + h * p.bb_dn, blk, static_cast<uint32_t>(p.bb_dn), full(slot));
-                        }
-                    }
+                    // gate/up: K chunks 4 st .. 4 st + 3 of the slice; down:
+                    // output tiles 4 sd .. of K chunk fs; consecutive blocks
+                    const bool gu = st < KC / kDecChunks;
+                    const int first = gu ? kDecChunks * st : kDecChunks * (st - KC / kDecChunks);
+                    const int nblk = gu ? kDecChunks : min(kDecChunks, NTd - first);
+                    const uint32_t bytes = static_cast<uint32_t>(nblk * p.bb_dn);
+                    mbar_arrive_expect_tx(full(slot), bytes);
+                    bulk_copy_g2s(dst, (gu ? gsrc : dsrc) + static_cast<size_t>(first) * p.bb_dn, bytes,
+                                  full(slot));
                 }
                 __syncwarp();
             }
@@ -647,10 +646,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             }
         }
     } else {
-        // compute warps: MMA fragment coordinates
+        // compute warps: MMA fragment coordinates.  Every compute warp takes
+        // every stage of the ring; warp w owns MMA row tile w: gate rows of
+        // features 8w .. 8w + 7 as rows g and their up rows as g + 8 (gate/up
+        // stages), rows 16w .. 16w + 15 of each 128-row output tile (down
+        // stages).  A warp waits on a stage's phase only after it has used the
+        // slot's previous phase, so no wait runs two phases ahead.
         const int g = lane >> 2;
         const int c = lane & 3;
-        float* red = reinterpret_cast<float*>(smem + L.red);
+        const int fr = 8 * warp + g;
         uint32_t q = 0;
         const int nvd = d / 32;
         for (int u = cta; u < u_total; u += G) {
@@ -660,81 +664,47 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int n = R.blk_n[b];
             if (tid == 0) R.fail = 0;
             compute_sync();  // also: every warp is done with the previous unit's h rows
-            // Stage q of the call is used by compute warp q % 8, so the warp that
-            // waits on a ring slot's phase has itself used the slot's previous
-            // phase (a parity wait only tells a phase from the one before it).
-            // gate/up: warp w takes the K chunks whose stage is w mod 8; MMA tile
-            // r has the gate rows of features 8r .. 8r + 7 as rows g and the up
-            // rows as g + 8
             const int cg = min(g, n - 1), c0 = min(2 * c, n - 1), c1 = min(2 * c + 1, n - 1);
             const uint16_t* brow = xsh + (R.sa[row0 + cg] / k) * (d + 32) + 8 * c;
             const float* bs0 = xsum + (R.sa[row0 + c0] / k) * nvd;
             const float* bs1 = xsum + (R.sa[row0 + c1] / k) * nvd;
-            float acc[kDecRowTiles][4];
-#pragma unroll
-            for (int r = 0; r < kDecRowTiles; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
-            for (int st = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
-                 st < KC / 2; st += kDecComputeWarps) {
-                const uint32_t qs = q + st;
-                const int slot = qs % kDecStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (qs / kDecStages) & 1, &R.abort_local))) {
-                    if (lane == 0) {
-                        R.fail = 1;
-                        if (!vload(R.abort_local)) dec_fail(p, R, 505);
-                    }
+            // gate/up: K chunks in order, two per stage, into one accumulator
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            bool ok = true;
+            for (int st = 0; st < KC / kDecChunks; ++st, ++q) {
+                const int slot = q % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
+                    ok = false;
                     break;
                 }
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
+                for (int cc = 0; cc < kDecChunks; ++cc) {
                     const uint8_t* hb = ring + slot * kDecStageBytes + cc * p.bb_dn;  // half-block of chunk kc
-                    const int kc = 2 * st + cc;
-#pragma unroll
-                    for (int r = 0; r < kDecRowTiles; ++r) {
-                        const int fr = 8 * r + g;
-                        chunk_mma_rows<kGpc>(acc[r], hb + gu_nib_offset(0, fr), hb + gu_nib_offset(1, fr),
-                                             hb + gu_word_offset(0, fr, 0, kGpc), hb + gu_word_offset(1, fr, 0, kGpc),
-                                             c, brow + kKChunk * kc, bs0 + 2 * kc, bs1 + 2 * kc);
-                    }
+                    const int kc = kDecChunks * st + cc;
+                    chunk_mma_rows<kGpc>(acc, hb + gu_nib_offset(0, fr), hb + gu_nib_offset(1, fr),
+                                         hb + gu_word_offset(0, fr, 0, kGpc), hb + gu_word_offset(1, fr, 0, kGpc),
+                                         c, brow + kKChunk * kc, bs0 + 2 * kc, bs1 + 2 * kc);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(slot));
             }
-            q += KC / 2;
-            // the warps' partial sums added in a fixed tree: ((w0 + w4) + (w2 + w6))
-            // + ((w1 + w5) + (w3 + w7)), through half-size shared memory
-            compute_sync();
-            if (vload(R.fail)) break;
-#pragma unroll
-            for (int half = kDecComputeWarps / 2; half >= 1; half >>= 1) {
-                if (warp >= half && warp < 2 * half)
-#pragma unroll
-                    for (int r = 0; r < kDecRowTiles; ++r)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) red[(((warp - half) * kDecRowTiles + r) * 4 + i) * 32 + lane] = acc[r][i];
-                compute_sync();
-                if (warp < half)
-#pragma unroll
-                    for (int r = 0; r < kDecRowTiles; ++r)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[r][i] += red[((warp * kDecRowTiles + r) * 4 + i) * 32 + lane];
-                compute_sync();
-            }
-            // SwiGLU of the slice (warp 0 holds the sums), rounded to bf16, into
-            // shared memory [token][64]
-            if (warp == 0) {
-#pragma unroll
-                for (int r = 0; r < kDecRowTiles; ++r) {
-                    const int fr = 8 * r + g;
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const int col = 2 * c + e2;
-                        if (col < n)
-                            hsh[col * kDecHStride + fr] =
-                                bf16_round_bits(__fdividef(acc[r][e2] * acc[r][2 + e2], 1.0f + __expf(-acc[r][e2])));
-                    }
+            if (!ok) {
+                if (lane == 0) {
+                    R.fail = 1;
+                    if (!vload(R.abort_local)) dec_fail(p, R, 505);
                 }
             }
+            // SwiGLU of the warp's eight features, rounded to bf16, into shared
+            // memory [token][64]
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int col = 2 * c + e2;
+                if (ok && col < n)
+                    hsh[col * kDecHStride + fr] =
+                        bf16_round_bits(__fdividef(acc[e2] * acc[2 + e2], 1.0f + __expf(-acc[e2])));
+            }
             compute_sync();
+            if (vload(R.fail)) break;
             // the 32-wide vector sums of the h rows (K order), for the group folds
             if (tid < 2 * n) {
                 const int col = tid >> 1, v = tid & 1;
@@ -743,48 +713,38 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 hsum[col * 2 + v] = sacc;
             }
             compute_sync();
-            // down: warp w takes the output tiles whose stage is w mod 8, all 128
-            // rows of each (eight MMA tiles); K = the slice
+            // down: up to four 128-row output tiles per stage, K = the slice
             const uint16_t* hrow = hsh + cg * kDecHStride + 8 * c;
             const float* hs0 = hsum + c0 * 2;
             const float* hs1 = hsum + c1 * 2;
-            for (int sd = (warp - static_cast<int>(q % kDecComputeWarps) + kDecComputeWarps) % kDecComputeWarps;
-                 sd < NTd / 2; sd += kDecComputeWarps) {
-                const uint32_t qs = q + sd;
-                const int slot = qs % kDecStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (qs / kDecStages) & 1, &R.abort_local))) {
+            for (int sd = 0; sd < NSd; ++sd, ++q) {
+                const int slot = q % kDecStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(full(slot), (q / kDecStages) & 1, &R.abort_local))) {
                     if (lane == 0) {
                         R.fail = 1;
                         if (!vload(R.abort_local)) dec_fail(p, R, 506);
                     }
                     break;
                 }
-                for (int h = 0; h < 2; ++h) {
-                    const int jd = 2 * sd + h;
+                const int nblk = min(kDecChunks, NTd - kDecChunks * sd);
+                for (int h = 0; h < nblk; ++h) {
+                    const int jd = kDecChunks * sd + h;
                     const uint8_t* stage = ring + slot * kDecStageBytes + h * p.bb_dn;
-                    float o[kDecRowTiles][4];
-#pragma unroll
-                    for (int r = 0; r < kDecRowTiles; ++r) {
-                        o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.0f;
-                        chunk_mma<kGpc>(o[r], stage, 128 * 32, 16 * r + g, c, hrow, hs0, hs1);
-                    }
+                    float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    chunk_mma<kGpc>(o, stage, 128 * 32, 16 * warp + g, c, hrow, hs0, hs1);
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
                         const int col = 2 * c + e2;
                         if (col < n) {
-                            float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128;
-#pragma unroll
-                            for (int r = 0; r < kDecRowTiles; ++r) {
-                                dst[16 * r + g] = o[r][e2];
-                                dst[16 * r + g + 8] = o[r][2 + e2];
-                            }
+                            float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128 + 16 * warp;
+                            dst[g] = o[e2];
+                            dst[g + 8] = o[2 + e2];
                         }
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(slot));
             }
-            q += NTd / 2;
             compute_sync();
             if (vload(R.fail)) break;
         }

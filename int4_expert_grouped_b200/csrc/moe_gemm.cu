@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const int b = u / NT;
             const int j = u - b * NT;
             const int e = a.block_map[3 * b];
-            // down: blocks (e, j, c) in a row; gate/up: half-blocks (e, j, 0, c) and (e, j, 1, c)
+            // down: block (e, c, j) for chunk c (a chunk's output tiles are
+            // contiguous); gate/up: half-blocks (e, j, 0, c) and (e, j, 1, c)
             const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
             const size_t half_stride = static_cast<size_t>(KC) * (a.block_bytes / 2);
             for (int c = 0; c < KC; ++c, ++it) {
@@ -228,7 +229,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     mbar_arrive_expect_tx(wfull(s), a.block_bytes);
                     const uint32_t dst = sbase + C::kOffW + s * C::kWStageBytes;
                     if constexpr (kDown) {
-                        bulk_copy_g2s(dst, src + c * a.block_bytes, a.block_bytes, wfull(s));
+                        bulk_copy_g2s(dst, a.wpack + ((static_cast<size_t>(e) * KC + c) * NT + j) * a.block_bytes,
+                                      a.block_bytes, wfull(s));
                     } else {
                         const uint32_t hb = a.block_bytes / 2;
                         bulk_copy_g2s(dst, src + c * hb, hb, wfull(s));
@@ -557,11 +559,11 @@ __global__ void prepack_kernel(const PrepackSource s, int E, int group, uint8_t*
         const uint16_t* bsrc = second ? s.b1 : s.b0;
         const size_t row = static_cast<size_t>(e) * s.N + n;
         const uint8_t* qrow = qsrc + row * (s.K / 2) + c * 32;
-        // down: block (e, j, c); gate/up: half-block (e, j, half, c) (see packed_block_bytes)
+        // down: block (e, c, j); gate/up: half-block (e, j, half, c) (see packed_block_bytes)
         const int f = rr & 127;
         const int hb = half_block_bytes(group);
         uint8_t* dst = s.tiles == 1
-                           ? out + ((static_cast<size_t>(e) * s.NT + j) * KC + c) * bb
+                           ? out + ((static_cast<size_t>(e) * KC + c) * s.NT + j) * bb
                            : out + (((static_cast<size_t>(e) * s.NT + j) * 2 + (f >> 6)) * KC + c) * hb;
         const int nib_off = s.tiles == 1 ? rr * 32 : gu_nib_offset(second ? 1 : 0, f & 63);
         uint32_t words[8];

@@ -59,7 +59,9 @@ constexpr int kDecodeSyncBytes = 8192;  // flags of the small-batch kernel (work
 // Packed weight block: `tiles` 128-row A tiles of one 64-wide K chunk
 // (gate/up: the gate and the up rows of 128 features; down: 128 rows).
 // A down block is 128 rows x 32 bytes of nibbles, then per row and group one
-// (scale, bias) bf16 pair.  A gate/up block is two half-blocks of the same
+// (scale, bias) bf16 pair; the blocks of one K chunk (a 64-feature slice of
+// h) are stored over all output tiles in a row (layout [E][f/64][d/128][block]).
+// A gate/up block is two half-blocks of the same
 // form, one per 64 features: [64 gate rows][64 up rows] of nibbles, then the
 // gate rows' and the up rows' words; each half-block is stored with the same
 // half of the expert's other K chunks (layout [E][f/128][2][d/64][half-block]),

@@ -130,7 +130,7 @@ def test_prepack_and_host_checks(moe):
 def test_forward_path_choice(moe):
     # host-only query: small batches of a supported shape take the decode kernel
     p = moe.Plan(8192, 2048, 128, 8, 768, 64)
-    assert [p.forward_path(T) for T in (0, 1, 4, 8, 9, 8192)] == [0, 1, 1, 1, 0, 0]
+    assert [p.forward_path(T) for T in (0, 1, 4, 8, 9, 1023, 1024, 8192)] == [0, 1, 1, 1, 0, 0, 2, 2]
     assert p.forward_path(-1) == -1 and p.forward_path(8193) == -1
     tiny = moe.Plan(64, 256, 8, 2, 128, 32)
     assert tiny.forward_path(3) == 1 and tiny.forward_path(9) == 0

@@ -349,6 +349,7 @@ def test_chained_calls_read_previous_output(moe):
 # ---------------------------------------------------------------------------
 def route_only(moe, T, d, E, k, x_bits, w_r, b_r):
     plan = moe.Plan(T, d, E, k, 128, 64)
+    assert plan.forward_path(T) == 2  # the int8 tensor-core router
     ws = torch.empty(plan.info.workspace_bytes, dtype=torch.uint8, device="cuda")
     i32 = dict(dtype=torch.int32, device="cuda")
     out = {"topk_idx": torch.empty((T, k), **i32),
