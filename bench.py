@@ -89,7 +89,8 @@ class ColdL2:
     """Keeps every timed step's weights cold in L2.
 
     Layers that touch more weight bytes than L2 holds get a 256 MiB write
-    before each step (outside the step's events).  Layers that touch few
+    before each step (outside the step's events); the write also keeps the
+    stream busy while the host enqueues the step.  Layers that touch few
     (the small batches: 8 experts, 21 MB at one token) instead rotate over R
     copies of the packed weights and W_r, R - 1 >= 2 x L2 / touched bytes, so
     that each step reads a copy whose bytes left L2 R - 1 steps ago; no
@@ -112,11 +113,16 @@ class ColdL2:
             self.desc = "flushed between steps (256 MiB write outside the step events)"
 
     def before(self, i):
+        import torch
         if self.packs is None:
             self.flush.fill_(i & 0xFF)
         else:
             self.layer.packed = self.packs[i % len(self.packs)]
             self.layer.w_r = self.wrs[i % len(self.wrs)]
+            # keep the stream busy while the host enqueues the step, so that
+            # the step's start event is taken when the GPU reaches it, not
+            # while the host is still launching (about 25 us of spinning)
+            torch.cuda._sleep(50000)
 
     def release(self):
         if self.packs is not None:

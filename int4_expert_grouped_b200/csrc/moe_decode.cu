@@ -61,7 +61,7 @@
 namespace moe {
 namespace {
 
-constexpr int kDecComputeWarps = 8;
+constexpr int kDecComputeWarps = 16;
 constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;  // + one producer warp
 constexpr int kDecProducerWarp = kDecComputeWarps;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
@@ -79,7 +79,9 @@ constexpr int kDecMaxSlices = 32;                          // f / 64
 constexpr int kDecMaxNTd = 64;                             // d / 128
 constexpr int kDecHStride = kDecSlice + 32;                // h row stride (elements) in shared memory
 constexpr int kDecRowTiles = kDecSlice / 8;                // 16-row MMA tiles of a slice: 8 gate + 8 up rows each
-static_assert(kDecRowTiles == kDecComputeWarps, "compute warp w owns MMA row tile w of every stage");
+constexpr int kDecKHalves = kDecComputeWarps / kDecRowTiles;  // compute warps per MMA row tile
+static_assert(kDecKHalves == 2 && kDecChunks % kDecKHalves == 0,
+              "compute warps w and w + 8 own MMA row tile w % 8, each half of every stage");
 constexpr int kDecWRows = 256;                             // W_r rows per tensor load (box limit)
 constexpr uint32_t kDecMagic0 = 0x4D6F4544u, kDecMagic1 = 0x53796E63u;
 
@@ -354,7 +356,7 @@ __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
 
 // Layout of the dynamic shared memory (byte offsets; the base is 1024-aligned).
 struct DecSmem {
-    int ring, x, xsum, h, hsum, lg, route, bars, total;
+    int ring, x, xsum, h, hsum, lg, red, route, bars, total;
 };
 __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     DecSmem L;
@@ -370,6 +372,7 @@ __host__ __device__ inline DecSmem dec_smem_layout(int T, int d, int E, int f) {
     L.h = take(kDecodeMaxT * kDecHStride * 2);
     L.hsum = take(kDecodeMaxT * (kDecSlice / 32) * 4);
     L.lg = take(T * E * 4);
+    L.red = take(kDecRowTiles * 4 * 32 * 4);  // second-half gate/up sums
     L.route = take(static_cast<int>(sizeof(DecRoute)));
     L.bars = take((2 * kDecStages + 1) * 8);
     L.total = o + 1024;  // + slack to align the base
@@ -647,14 +650,20 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
         }
     } else {
         // compute warps: MMA fragment coordinates.  Every compute warp takes
-        // every stage of the ring; warp w owns MMA row tile w: gate rows of
-        // features 8w .. 8w + 7 as rows g and their up rows as g + 8 (gate/up
-        // stages), rows 16w .. 16w + 15 of each 128-row output tile (down
-        // stages).  A warp waits on a stage's phase only after it has used the
-        // slot's previous phase, so no wait runs two phases ahead.
+        // every stage of the ring; warps w and w + 8 own MMA row tile r = w % 8:
+        // gate rows of features 8r .. 8r + 7 as rows g and their up rows as
+        // g + 8 (gate/up stages), rows 16r .. 16r + 15 of each 128-row output
+        // tile (down stages); warp w < 8 takes the first half of each stage's
+        // K chunks or output tiles, warp w + 8 the second.  A warp waits on a
+        // stage's phase only after it has used the slot's previous phase, so
+        // no wait runs two phases ahead.
         const int g = lane >> 2;
         const int c = lane & 3;
-        const int fr = 8 * warp + g;
+        const int rt = warp % kDecRowTiles;   // MMA row tile
+        const int kh = warp / kDecRowTiles;   // which half of each stage's chunks / tiles
+        const int fr = 8 * rt + g;
+        float* red = reinterpret_cast<float*>(smem + L.red);
+        constexpr int kHalf = kDecChunks / kDecKHalves;  // chunks or tiles per warp and stage
         uint32_t q = 0;
         const int nvd = d / 32;
         for (int u = cta; u < u_total; u += G) {
@@ -668,7 +677,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const uint16_t* brow = xsh + (R.sa[row0 + cg] / k) * (d + 32) + 8 * c;
             const float* bs0 = xsum + (R.sa[row0 + c0] / k) * nvd;
             const float* bs1 = xsum + (R.sa[row0 + c1] / k) * nvd;
-            // gate/up: K chunks in order, two per stage, into one accumulator
+            // gate/up: this warp's half of each stage's K chunks, in order,
+            // into one accumulator
             float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             bool ok = true;
             for (int st = 0; st < KC / kDecChunks; ++st, ++q) {
@@ -678,7 +688,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     break;
                 }
 #pragma unroll
-                for (int cc = 0; cc < kDecChunks; ++cc) {
+                for (int ci = 0; ci < kHalf; ++ci) {
+                    const int cc = kh * kHalf + ci;
                     const uint8_t* hb = ring + slot * kDecStageBytes + cc * p.bb_dn;  // half-block of chunk kc
                     const int kc = kDecChunks * st + cc;
                     chunk_mma_rows<kGpc>(acc, hb + gu_nib_offset(0, fr), hb + gu_nib_offset(1, fr),
@@ -694,17 +705,26 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     if (!vload(R.abort_local)) dec_fail(p, R, 505);
                 }
             }
-            // SwiGLU of the warp's eight features, rounded to bf16, into shared
-            // memory [token][64]
+            // the two halves' sums, first half + second half
+            if (kh == 1)
 #pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-                const int col = 2 * c + e2;
-                if (ok && col < n)
-                    hsh[col * kDecHStride + fr] =
-                        bf16_round_bits(__fdividef(acc[e2] * acc[2 + e2], 1.0f + __expf(-acc[e2])));
-            }
+                for (int i = 0; i < 4; ++i) red[(rt * 4 + i) * 32 + lane] = acc[i];
             compute_sync();
             if (vload(R.fail)) break;
+            // SwiGLU of the row tile's eight features, rounded to bf16, into
+            // shared memory [token][64]
+            if (kh == 0) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] += red[(rt * 4 + i) * 32 + lane];
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int col = 2 * c + e2;
+                    if (col < n)
+                        hsh[col * kDecHStride + fr] =
+                            bf16_round_bits(__fdividef(acc[e2] * acc[2 + e2], 1.0f + __expf(-acc[e2])));
+                }
+            }
+            compute_sync();
             // the 32-wide vector sums of the h rows (K order), for the group folds
             if (tid < 2 * n) {
                 const int col = tid >> 1, v = tid & 1;
@@ -727,16 +747,16 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     break;
                 }
                 const int nblk = min(kDecChunks, NTd - kDecChunks * sd);
-                for (int h = 0; h < nblk; ++h) {
+                for (int h = kh * kHalf; h < min(nblk, (kh + 1) * kHalf); ++h) {
                     const int jd = kDecChunks * sd + h;
                     const uint8_t* stage = ring + slot * kDecStageBytes + h * p.bb_dn;
                     float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    chunk_mma<kGpc>(o, stage, 128 * 32, 16 * warp + g, c, hrow, hs0, hs1);
+                    chunk_mma<kGpc>(o, stage, 128 * 32, 16 * rt + g, c, hrow, hs0, hs1);
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
                         const int col = 2 * c + e2;
                         if (col < n) {
-                            float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128 + 16 * warp;
+                            float* dst = p.pdn + (static_cast<size_t>(row0 + col) * S + fs) * d + jd * 128 + 16 * rt;
                             dst[g] = o[e2];
                             dst[g + 8] = o[2 + e2];
                         }
