@@ -293,24 +293,49 @@ struct DecRoute {
 };
 
 // top-k (each (token, expert) pair finds its slot by counting the experts
-// ahead of it; ties go to the lower id; measured faster here than a warp
-// top-k per token), the softmax weights over the k slots, counts (integer
-// atomics), offsets (exclusive scan), one block per expert with rows
-// (ascending expert), and the stable scatter (rank of assignment a = number
-// of earlier assignments to its expert).  All kDecThreads threads.
+// ahead of it, P threads per pair over E / P experts each; ties go to the
+// lower id; measured faster here than a warp top-k per token), counts
+// (integer atomics, taken with the slots), the softmax weights over the k
+// slots, offsets and the block map (one exclusive scan of counts | blocks
+// << 16: counts sum to at most 64, blocks to at most E), one block per expert
+// with rows (ascending expert), and the stable scatter (rank of assignment a
+// = number of earlier assignments to its expert).  All kDecThreads threads;
+// R.cnt is zero on entry.
 __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int Tk = T * k;
-    if (tid < E) R.cnt[tid] = 0;
-    for (int it = tid; it < T * E; it += kDecThreads) {
-        const int t = it / E;
-        const int e = it - t * E;
-        const int slot = expert_slot(lg + t * E, E, e);
-        if (slot < k) {
-            R.idx[t * k + slot] = e;
-            R.sel[t * k + slot] = lg[it];
+    int P = 1;
+    while (P < 8 && 2 * P * T * E <= kDecThreads && (E / (2 * P)) % 4 == 0) P *= 2;
+    const int per = E / P;
+    const int n_it = T * E * P;
+    for (int base = warp * 32; base < n_it; base += kDecThreads) {  // warp-uniform: the shuffles below
+        const int it = base + lane;
+        const bool valid = it < n_it;  // whole groups of P lanes: n_it is a multiple of P
+        const int pair = it / P;
+        const int part = it - pair * P;
+        const int t = valid ? pair / E : 0;
+        const int e = valid ? pair - t * E : 0;
+        const float* row = lg + t * E;
+        const float v = row[e];
+        int r = 0;
+        if (valid) {
+            const float4* r4 = reinterpret_cast<const float4*>(row + part * per);
+            for (int j = 0; j < per / 4; ++j) {
+                const float4 u = r4[j];
+                const int e2 = part * per + 4 * j;
+                r += (u.x > v) | ((u.x == v) & (e2 < e));
+                r += (u.y > v) | ((u.y == v) & (e2 + 1 < e));
+                r += (u.z > v) | ((u.z == v) & (e2 + 2 < e));
+                r += (u.w > v) | ((u.w == v) & (e2 + 3 < e));
+            }
+        }
+        for (int m = 1; m < P; m <<= 1) r += __shfl_xor_sync(0xffffffffu, r, m);
+        if (valid && part == 0 && r < k) {
+            R.idx[t * k + r] = e;
+            R.sel[t * k + r] = v;
+            atomicAdd(&R.cnt[e], 1);
         }
     }
     __syncthreads();
@@ -318,19 +343,14 @@ __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
         const float wt = warp_slot_weights(lane < k ? R.sel[t * k + lane] : 0.0f, k, lane);
         if (lane < k) R.w[t * k + lane] = wt;
     }
-    __syncthreads();
-    for (int a = tid; a < Tk; a += kDecThreads) atomicAdd(&R.cnt[R.idx[a]], 1);
-    __syncthreads();
     const int c = tid < E ? R.cnt[tid] : 0;
+    const int nt = c > 0 ? 1 : 0;  // at most T <= 8 rows per expert: one block each
     int total = 0;
-    const int off = block_exclusive_scan<kDecThreads>(c, R.sh_warp, &total);
-    if (tid < E) R.off[tid] = off;
-    if (tid == 0) R.off[E] = total;
-    // at most T <= 8 rows per expert: one block of the block map each
-    const int nt = c > 0 ? 1 : 0;
-    int nb = 0;
-    const int bo = block_exclusive_scan<kDecThreads>(nt, R.sh_warp, &nb);
+    const int packed = block_exclusive_scan<kDecThreads>(c | (nt << 16), R.sh_warp, &total);
+    const int off = packed & 0xFFFF, bo = packed >> 16;
+    const int nb = total >> 16;
     if (tid < E) {
+        R.off[tid] = off;
         R.bo[tid] = bo;
         if (nt) {
             R.blk_e[bo] = tid;
@@ -339,6 +359,7 @@ __device__ void route_small(const float* lg, int T, int E, int k, DecRoute& R) {
         }
     }
     if (tid == 0) {
+        R.off[E] = total & 0xFFFF;
         R.bo[E] = nb;
         R.nb = nb;
     }
@@ -574,6 +595,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             lg[it] = p.b_r != nullptr ? __fadd_rn(S, __ldg(p.b_r + (it % E))) : S;
         }
     }
+    if (tid < E) R.cnt[tid] = 0;
     __syncthreads();
     const bool routed = !vload(R.abort_local);
     if (routed) route_small(lg, T, E, k, R);

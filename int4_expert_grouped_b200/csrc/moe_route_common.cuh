@@ -79,21 +79,6 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, 
     my_w = warp_slot_weights(my_v, k, lane);
 }
 
-// Slot of expert e among one token's E logits: the number of experts that
-// come before it in the order (logit descending, id ascending).  The experts
-// with slot < k are exactly the ones warp_topk selects, in the same order.
-__device__ __forceinline__ int expert_slot(const float* __restrict__ row, int E, int e) {
-    // better(Cand{u, e2}, Cand{v, e}) for two valid ids, without branches
-    const float v = row[e];
-    int r = 0;
-#pragma unroll 8
-    for (int e2 = 0; e2 < E; ++e2) {
-        const float u = row[e2];
-        r += (u > v) | ((u == v) & (e2 < e));
-    }
-    return r;
-}
-
 // Exclusive prefix sum of one int per thread over a CTA of kThreads threads
 // (a multiple of 32, at most 1024); *total receives the sum.  sh_warp needs
 // kThreads / 32 + 1 ints.  Every thread of the CTA must call it.
