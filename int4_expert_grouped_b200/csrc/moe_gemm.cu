@@ -8,17 +8,21 @@
 //   grouped_gemm_kernel   persistent, warp-specialised tcgen05 GEMM:
 //       gate/up: D0 = Wg xs^T, D1 = Wu xs^T over token rows in expert order,
 //                epilogue h = silu(D0) * D1 -> bf16 h rows
-//       down:    D = kDownTiles 128-row tiles of Wd times h^T, epilogue
-//                o = bf16(D) rows
+//       down:    D = 128-row tiles of Wd (one, or two in the streaming
+//                variant) times h^T, epilogue o = bf16(D) rows
 //                (the routing-weighted sum over a token's experts is a
 //                separate pass, so no output element is ever accumulated by
 //                two CTAs)
 //
-// One work unit = one block-map tile (<= 256 expert-ordered rows of one
-// expert) x one output tile of 128 features (gate/up: the gate and the up
-// rows of those features).  The weights are the MMA A operand (M = 128 per
-// tile), the tokens the B operand (N = rows rounded up to 16 <= 256), so a
-// partly filled tile wastes at most 15 columns.
+// One gate/up work unit = one block-map tile (<= 256 expert-ordered rows of
+// one expert) x one output tile of 128 features (the gate and the up rows of
+// those features).  One down unit = one half of a block-map tile (<= 128
+// rows) x two adjacent output tiles of 128 features: each token tile then
+// serves two output tiles (the down GEMM waited on its token tiles about a
+// quarter of the time with one), and the 256-column accumulator leaves room
+// for a second, so the epilogue overlaps the next unit.  The weights are the
+// MMA A operand (M = 128 per tile), the tokens the B operand (N = rows
+// rounded up to 16), so a partly filled tile wastes at most 15 columns.
 //
 // Shapes are set by two limits measured on B200: expanding int4 costs about
 // two instructions per weight, so every expanded weight must serve up to 256
@@ -58,7 +62,6 @@ constexpr int kNumEpiWarps = 4;
 constexpr int kGemmThreads = 16 * 32;
 constexpr int kTransformThreads = kNumTransformWarps * 32;
 constexpr int kATileBytes = 128 * 128;     // 128 rows x 64 bf16 (128B swizzle)
-constexpr int kBStageBytes = kBlockT * 128;  // up to 256 token rows x 64 bf16
 constexpr int kEpiRowBytes = 80;    // staging row: 32 bf16 + 16 bytes of padding
 constexpr uint32_t kTmemCols = 512;
 
@@ -67,18 +70,31 @@ constexpr uint32_t kTmemCols = 512;
 // is bound by reading the packed weights from HBM: a deep packed-weight ring
 // keeps more of them in flight per SM, at the cost of expanded-A and token
 // stages that such blocks do not need.
+//
+// Units.  Gate/up: (block, 128-feature tile): two A tiles (the tile's gate and
+// up rows) x the block's rows (N <= 256), one 512-column accumulator.  Down:
+// (block, 128-row output tile): one A tile x the block's rows, two 256-column
+// accumulators, so the epilogue of one unit overlaps the next unit's MMAs.
+// Down, streaming variant ("pair" units): (block, half of its rows, pair of
+// output tiles): two A tiles (the pair's packed blocks, adjacent in memory
+// for one K chunk) x at most 128 rows, so each token tile serves two output
+// tiles.  At 512 tokens that measured 72 against 89 us; with large blocks
+// N = 128 doubles the A operand's shared-memory reads per flop and the
+// expansion per token (319 against 250 us at 8192 tokens).
 template <bool kDown, bool kStream>
 struct Cfg {
-    static constexpr int kTiles = kDown ? kDownTiles : 2;     // A tiles (of 128 rows) per unit
+    static constexpr bool kPair = kDown && kStream;
+    static constexpr int kTiles = (kDown && !kPair) ? kDownTiles : 2;  // A tiles (of 128 rows) per unit
     static constexpr bool kOneTile = kTiles == 1;
+    static constexpr int kBlockN = kPair ? kBlockT / 2 : kBlockT;  // token rows per unit (MMA N at most)
     static constexpr int kNW = kStream ? (kOneTile ? 20 : 8) : (kOneTile ? 4 : 2);  // packed weight ring
     static constexpr int kNA = kStream ? 2 : (kOneTile ? 4 : 3);  // expanded bf16 A ring
     static constexpr int kNB = kStream ? 2 : 3;                   // token B ring
-    static constexpr int kAccBufs = kOneTile ? 2 : 1;         // TMEM accumulator buffers
-    static constexpr int kAccCols = kTiles * kBlockT;         // columns per buffer
+    static constexpr int kAccBufs = kDown ? 2 : 1;            // TMEM accumulator buffers
+    static constexpr int kAccCols = kTiles * kBlockN;         // columns per buffer
+    static constexpr int kBStageBytes = kBlockN * 128;        // token rows x 64 bf16
     static constexpr int kAStageBytes = kTiles * kATileBytes;
     static constexpr int kWStageBytes = packed_block_bytes(kTiles, 32);  // largest (group 32)
-    static constexpr int kNibbleBytes = kTiles * 128 * 32;
     static constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
     // transform warp groups; group g expands the chunks it with it % kGroups == g
     static constexpr int kGroups = kOneTile ? 2 : 1;
@@ -203,17 +219,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         *abort_flag = 1;
         report_error(a.status, MOE_ERR_DEVICE_TIMEOUT, (kDown ? 200 : 100) + where);
     };
+    // unit u: block b = u / NT; output tile j = u % NT; pair units: rows half
+    // (u % NT) / (NT / 2) of the block and output tile pair j.  Every role
+    // skips the same empty units (a second half of a block of <= 128 rows).
+    struct Unit {
+        int b, j, row0, rows;
+    };
+    auto unit_of = [&](int u) {
+        Unit x;
+        x.b = u / NT;
+        const int r = u - x.b * NT;
+        const int row0 = a.block_map[3 * x.b + 1];
+        const int rows = a.block_map[3 * x.b + 2];
+        if constexpr (C::kPair) {
+            const int half = r / (NT / 2);
+            x.j = r - half * (NT / 2);
+            x.row0 = row0 + half * C::kBlockN;
+            x.rows = min(C::kBlockN, rows - half * C::kBlockN);
+        } else {
+            x.j = r;
+            x.row0 = row0;
+            x.rows = rows;
+        }
+        return x;
+    };
 
     if (warp == kWarpWProducer) {
         // the whole warp runs the loop; one elected lane issues the copies
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-            const int b = u / NT;
-            const int j = u - b * NT;
-            const int e = a.block_map[3 * b];
-            // down: block (e, c, j) for chunk c (a chunk's output tiles are
-            // contiguous); gate/up: half-blocks (e, j, 0, c) and (e, j, 1, c)
+            const Unit un = unit_of(u);
+            if (un.rows <= 0) continue;
+            const int j = un.j;
+            const int e = a.block_map[3 * un.b];
+            // down: blocks (e, c, kTiles j ..) for chunk c, adjacent (a chunk's
+            // output tiles are contiguous); gate/up: half-blocks (e, j, 0, c)
+            // and (e, j, 1, c)
             const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
             const size_t half_stride = static_cast<size_t>(KC) * (a.block_bytes / 2);
             for (int c = 0; c < KC; ++c, ++it) {
@@ -226,12 +268,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 // test hook: withhold the first stage, so its consumers' waits run out
                 if (a.withhold_first && it == 0) continue;
                 if (elect_one()) {
-                    mbar_arrive_expect_tx(wfull(s), a.block_bytes);
                     const uint32_t dst = sbase + C::kOffW + s * C::kWStageBytes;
                     if constexpr (kDown) {
-                        bulk_copy_g2s(dst, a.wpack + ((static_cast<size_t>(e) * KC + c) * NT + j) * a.block_bytes,
-                                      a.block_bytes, wfull(s));
+                        // the unit's kTiles output tiles of chunk c, adjacent blocks
+                        const uint32_t bytes = C::kTiles * a.block_bytes;
+                        mbar_arrive_expect_tx(wfull(s), bytes);
+                        bulk_copy_g2s(dst,
+                                      a.wpack + ((static_cast<size_t>(e) * KC + c) * NT + C::kTiles * j) * a.block_bytes,
+                                      bytes, wfull(s));
                     } else {
+                        mbar_arrive_expect_tx(wfull(s), a.block_bytes);
                         const uint32_t hb = a.block_bytes / 2;
                         bulk_copy_g2s(dst, src + c * hb, hb, wfull(s));
                         bulk_copy_g2s(dst + hb, src + half_stride + c * hb, hb, wfull(s));
@@ -252,10 +298,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         uint32_t it = 0, ucount = 0;
         bool ok = true;
         bool ready = false;  // the current stage was already seen full
-        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x, ++ucount) {
-            const int b = u / NT;
-            const int rows = a.block_map[3 * b + 2];
-            const int N = (rows + 15) & ~15;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            const Unit un = unit_of(u);
+            if (un.rows <= 0) continue;
+            const int N = (un.rows + 15) & ~15;
             const uint32_t idesc = make_idesc_bf16(128, N);
             const int buf = ucount % C::kAccBufs;
             const uint32_t use = ucount / C::kAccBufs;
@@ -287,7 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 const uint32_t ra = mbar_test(afull(nx % C::kNA), (nx / C::kNA) & 1);
                 const uint32_t rb = mbar_test(bfull(nx % C::kNB), (nx / C::kNB) & 1);
                 const uint32_t abase = sbase + C::kOffA + sa * C::kAStageBytes;
-                const uint64_t db = make_sw128_desc(sbase + C::kOffB + sb * kBStageBytes);
+                const uint64_t db = make_sw128_desc(sbase + C::kOffB + sb * C::kBStageBytes);
                 uint64_t da[C::kTiles];
 #pragma unroll
                 for (int t = 0; t < C::kTiles; ++t) da[t] = make_sw128_desc(abase + t * kATileBytes);
@@ -297,7 +343,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                         const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
                         for (int t = 0; t < C::kTiles; ++t)
-                            mma_bf16(dacc + t * kBlockT, da[t] + 2 * kk, db + 2 * kk, idesc, acc);
+                            mma_bf16(dacc + t * C::kBlockN, da[t] + 2 * kk, db + 2 * kk, idesc, acc);
                     }
                     mma_commit(aempty(sa));
                     mma_commit(bempty(sb));
@@ -306,6 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             }
             if (ok && elect_one()) mma_commit(accfull(buf));
             __syncwarp();
+            ++ucount;
         }
         if (!ok) {
             if (elect_one()) mma_commit(drain_bar);
@@ -320,9 +367,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-            const int row0 = a.block_map[3 * (u / NT) + 1];
-            // the smallest box (256 >> bi rows) that covers the N rows the MMA reads
-            const int N = (a.block_map[3 * (u / NT) + 2] + 15) & ~15;
+            const Unit un = unit_of(u);
+            if (un.rows <= 0) continue;
+            const int row0 = un.row0;
+            // the smallest box (256 >> bi rows) that covers the N rows the MMA
+            // reads (N <= kBlockN, so the box fits the stage)
+            const int N = (un.rows + 15) & ~15;
             int bi = 0;
             while (bi + 1 < kBoxSizes && (kBlockT >> (bi + 1)) >= N) ++bi;
             const uint32_t box_bytes = static_cast<uint32_t>(kBlockT >> bi) * (kKChunk * 2);
@@ -335,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 }
                 if (elect_one()) {
                     mbar_arrive_expect_tx(bfull(s), box_bytes);
-                    tma_load_2d(sbase + C::kOffB + s * kBStageBytes, &a.bmap[bi], c * kKChunk, row0, bfull(s));
+                    tma_load_2d(sbase + C::kOffB + s * C::kBStageBytes, &a.bmap[bi], c * kKChunk, row0, bfull(s));
                 }
                 __syncwarp();
             }
@@ -346,8 +396,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 mbar_wait_drain(bfull(i % C::kNB), (i / C::kNB) & 1);
         }
     } else if (warp >= kWarpTransform0 && warp < kWarpTransform0 + kNumTransformWarps) {
-        // Two groups of transform warps take alternate chunks, so each warp
-        // pays one round of barrier waits per two chunks.
+        // One-tile units: two groups of transform warps take alternate chunks,
+        // so each warp pays one round of barrier waits per two chunks; two-tile
+        // units: all eight warps expand each chunk.
         const int ttid = threadIdx.x - kWarpTransform0 * 32;
         const int grp = ttid / C::kGroupThreads;
         const int gtid = ttid % C::kGroupThreads;
@@ -355,6 +406,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+            if (unit_of(u).rows <= 0) continue;
             for (int c = 0; c < KC; ++c, ++it) {
                 if (static_cast<int>(it % C::kGroups) != grp) continue;
                 const int sw = it % C::kNW;
@@ -380,9 +432,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 for (int rep = 0; rep < C::kTasks; ++rep) {
                     const int row = (gtid + C::kGroupThreads * rep) >> 1;
                     int nib_off, w_off;
-                    if constexpr (kDown) {
-                        nib_off = row * 32;
-                        w_off = C::kNibbleBytes + (row * gpc + g) * 4;
+                    if constexpr (kDown) {  // row: block (output tile) row >> 7 of the stage, row & 127 in it
+                        const int boff = (row >> 7) * a.block_bytes;
+                        nib_off = boff + (row & 127) * 32;
+                        w_off = boff + 128 * 32 + ((row & 127) * gpc + g) * 4;
                     } else {  // row: tile row >> 7, feature row & 127 in half-block (row & 127) >> 6
                         const int hoff = ((row & 127) >> 6) * hbytes;
                         nib_off = hoff + gu_nib_offset(row >> 7, row & 63);
@@ -426,11 +479,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         // feature octet (16 bytes), row c = lane % 8 the token within a group of 8
         const uint32_t st_addr = stg + (lane & 7) * kEpiRowBytes + (lane >> 3) * 16;
         uint32_t ucount = 0;
-        for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++ucount) {
-            const int b = u / NT;
-            const int j = u - b * NT;
-            const int row0 = a.block_map[3 * b + 1];
-            const int rows = a.block_map[3 * b + 2];
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+            const Unit un = unit_of(u);
+            if (un.rows <= 0) continue;
+            const int j = un.j;
+            const int row0 = un.row0;
+            const int rows = un.rows;
             const int ncb = (rows + 31) >> 5;
             const int buf = ucount % C::kAccBufs;
             const uint32_t use = ucount / C::kAccBufs;
@@ -439,15 +493,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 break;
             }
             tc_fence_after();
-            // gate/up: one output tile (gate at column 0, up at kBlockT); down:
-            // kTiles output tiles of 128 features at columns t * kBlockT
+            // gate/up: one output tile (gate at column 0, up at kBlockN); down:
+            // kTiles output tiles of 128 features at columns t * kBlockN
             constexpr int kOutTiles = kDown ? C::kTiles : 1;
 #pragma unroll 1
             for (int it = 0; it < kOutTiles * ncb; ++it) {
                 const int t = it / ncb;
                 const int cb = it - t * ncb;
                 const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols +
-                                    t * kBlockT;
+                                    t * C::kBlockN;
                 // p[h][i]: lane half h (features 16h + t/4 (+8)), register i
                 uint32_t p[2][8];
                 if constexpr (kDown) {
@@ -473,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t ta = tb + (static_cast<uint32_t>(16 * h) << 16) + cb * 32;
                         tmem_ld_16x256b_x4(ta, v[h]);
-                        tmem_ld_16x256b_x4(ta + kBlockT, uu[h]);
+                        tmem_ld_16x256b_x4(ta + C::kBlockN, uu[h]);
                     }
                     tmem_ld_wait();
 #pragma unroll
@@ -519,11 +573,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
                 }
                 __syncwarp();
             }
-            if (ncb == 0) {  // a block always has rows; keep the hand-back unconditional
+            if (ncb == 0) {  // a unit always has rows; keep the hand-back unconditional
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(accempty(buf));
             }
+            ++ucount;
         }
     }
 

@@ -52,7 +52,7 @@ constexpr int kRouteGroupT = 256; // tokens per scatter group (one histogram row
 constexpr int kBlockT = 256;      // block map tile height = largest MMA N
 constexpr int kKChunk = 64;       // K elements per pipeline stage (128 bytes bf16)
 constexpr int kDecodeMaxT = 8;    // largest batch the small-batch (decode) path takes
-constexpr int kDownTiles = 1;     // 128-row down-projection tiles per packed block and GEMM unit
+constexpr int kDownTiles = 1;     // 128-row down-projection tiles per packed block
 constexpr int kBoxSizes = 4;      // token-tile boxes of 256, 128, 64 and 32 rows
 constexpr int kDecodeSyncBytes = 8192;  // flags of the small-batch kernel (workspace bytes 256 ..)
 

@@ -25,41 +25,36 @@ import pytest
 
 GEMM_SRC = os.path.join(os.path.dirname(__file__), "..", "int4_expert_grouped_b200", "csrc",
                         "moe_gemm.cu")
-INTERNAL_H = os.path.join(os.path.dirname(__file__), "..", "int4_expert_grouped_b200", "csrc",
-                          "moe_internal.h")
 TRANSFORM_WARPS = 8
 EPILOGUE_WARPS = 4
 
 
 def kernel_configs():
     """(name, NW, NA, NB, G, acc_bufs) of the two projections in both ring
-    variants (large blocks; weight streaming for small blocks), from the source."""
+    variants (large blocks; weight streaming for small blocks), from the source.
+    Units of one A tile (down, large blocks) and of two (gate/up; down in the
+    streaming variant, where a unit pairs two output tiles) take the kOneTile
+    and the other branch of each ring size."""
     src = open(GEMM_SRC).read()
-    down_tiles = int(re.search(r"constexpr int kDownTiles = (\d+);", open(INTERNAL_H).read()).group(1))
+    n = r"(\d+)"
 
-    def pick(name):
-        m = re.search(r"static constexpr int %s = kOneTile \? (\d+) : (\d+);" % name, src)
+    def find(pattern, name):
+        m = re.search(pattern, src)
         assert m, name
-        return int(m.group(1)), int(m.group(2))
+        return [int(g) for g in m.groups()]
 
-    acc, g = pick("kAccBufs"), pick("kGroups")
-    m = re.search(r"static constexpr int kNW = kStream \? \(kOneTile \? (\d+) : (\d+)\) : "
-                  r"\(kOneTile \? (\d+) : (\d+)\);", src)
-    assert m, "kNW"
-    nw_s, nw = (int(m.group(1)), int(m.group(2))), (int(m.group(3)), int(m.group(4)))
-    m = re.search(r"static constexpr int kNA = kStream \? (\d+) : \(kOneTile \? (\d+) : (\d+)\);", src)
-    assert m, "kNA"
-    na_s, na = (int(m.group(1)),) * 2, (int(m.group(2)), int(m.group(3)))
-    m = re.search(r"static constexpr int kNB = kStream \? (\d+) : (\d+);", src)
-    assert m, "kNB"
-    nb_s, nb = int(m.group(1)), int(m.group(2))
-    # each pair is (value with one weight tile per unit, value with two);
-    # gate/up always has two tiles, down has kDownTiles
-    i = 0 if down_tiles == 1 else 1
-    return [("gate/up", nw[1], na[1], nb, g[1], acc[1]),
-            ("down", nw[i], na[i], nb, g[i], acc[i]),
-            ("gate/up, streaming", nw_s[1], na_s[1], nb_s, g[1], acc[1]),
-            ("down, streaming", nw_s[i], na_s[i], nb_s, g[i], acc[i])]
+    nw_s1, nw_s2, nw1, nw2 = find(r"static constexpr int kNW = kStream \? \(kOneTile \? %s : %s\) : "
+                                  r"\(kOneTile \? %s : %s\);" % (n, n, n, n), "kNW")
+    na_s, na1, na2 = find(r"static constexpr int kNA = kStream \? %s : \(kOneTile \? %s : %s\);"
+                          % (n, n, n), "kNA")
+    nb_s, nb = find(r"static constexpr int kNB = kStream \? %s : %s;" % (n, n), "kNB")
+    acc_dn, acc_gu = find(r"static constexpr int kAccBufs = kDown \? %s : %s;" % (n, n), "kAccBufs")
+    g1, g2 = find(r"static constexpr int kGroups = kOneTile \? %s : %s;" % (n, n), "kGroups")
+    assert re.search(r"kTiles = \(kDown && !kPair\) \? kDownTiles : 2;", src), "kTiles"
+    return [("gate/up", nw2, na2, nb, g2, acc_gu),
+            ("down", nw1, na1, nb, g1, acc_dn),
+            ("gate/up, streaming", nw_s2, na_s, nb_s, g2, acc_gu),
+            ("down, streaming (pairs)", nw_s2, na_s, nb_s, g2, acc_dn)]
 
 
 class Barrier:
