@@ -354,15 +354,16 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     g.num_blocks = r.nb;
     g.out = h;
     g.status = status;
+    // at most 64 rows per expert on average: the GEMMs are bound by reading the
+    // weights, so they keep more packed-weight stages in flight, and each unit
+    // takes one half (<= 128 rows) of a block
+    g.stream = static_cast<long long>(T) * s.k < 64ll * s.E ? 1 : 0;
     g.K = s.d;
-    g.NT = s.f / 128;
+    g.NT = (s.f / 128) * (g.stream ? 2 : 1);  // units per block: feature tiles (x halves)
     g.out_ld = s.f;
     g.group = s.group;
     g.block_bytes = plan->group_bytes;
     g.max_units = mb * g.NT;
-    // at most 64 rows per expert on average: the GEMMs are bound by reading the
-    // weights, so they keep more packed-weight stages in flight
-    g.stream = static_cast<long long>(T) * s.k < 64ll * s.E ? 1 : 0;
     // test hook (MOE_SHAPE_TEST_TIMEOUT): the gate/up GEMM withholds a stage and
     // its waits give up after 5 ms
     const bool test_timeout = (s.flags & MOE_SHAPE_TEST_TIMEOUT) != 0;

@@ -75,22 +75,25 @@ constexpr uint32_t kTmemCols = 512;
 // up rows) x the block's rows (N <= 256), one 512-column accumulator.  Down:
 // (block, 128-row output tile): one A tile x the block's rows, two 256-column
 // accumulators, so the epilogue of one unit overlaps the next unit's MMAs.
-// Down, streaming variant ("pair" units): (block, half of its rows, pair of
-// output tiles): two A tiles (the pair's packed blocks, adjacent in memory
-// for one K chunk) x at most 128 rows, so each token tile serves two output
-// tiles.  At 512 tokens that measured 72 against 89 us; with large blocks
-// N = 128 doubles the A operand's shared-memory reads per flop and the
-// expansion per token (319 against 250 us at 8192 tokens).
+// Streaming variant (few rows per expert): units take one half of a block's
+// rows (at most 128), so the token stages are half as large and twice as
+// many, and two accumulators fit.  Gate/up: (block, half, 128-feature tile).
+// Down ("pair" units): (block, half, pair of output tiles): two A tiles (the
+// pair's packed blocks, adjacent in memory for one K chunk), so each token
+// tile serves two output tiles.  At 512 tokens the down pairs measured 72
+// against 89 us; with large blocks N = 128 doubles the A operand's
+// shared-memory reads per flop and the expansion per token (319 against
+// 250 us at 8192 tokens).
 template <bool kDown, bool kStream>
 struct Cfg {
     static constexpr bool kPair = kDown && kStream;
     static constexpr int kTiles = (kDown && !kPair) ? kDownTiles : 2;  // A tiles (of 128 rows) per unit
     static constexpr bool kOneTile = kTiles == 1;
-    static constexpr int kBlockN = kPair ? kBlockT / 2 : kBlockT;  // token rows per unit (MMA N at most)
+    static constexpr int kBlockN = kStream ? kBlockT / 2 : kBlockT;  // token rows per unit (MMA N at most)
     static constexpr int kNW = kStream ? (kOneTile ? 20 : 8) : (kOneTile ? 4 : 2);  // packed weight ring
     static constexpr int kNA = kStream ? 2 : (kOneTile ? 4 : 3);  // expanded bf16 A ring
-    static constexpr int kNB = kStream ? 2 : 3;                   // token B ring
-    static constexpr int kAccBufs = kDown ? 2 : 1;            // TMEM accumulator buffers
+    static constexpr int kNB = kStream ? 4 : 3;                   // token B ring
+    static constexpr int kAccBufs = (kDown || kStream) ? 2 : 1;   // TMEM accumulator buffers
     static constexpr int kAccCols = kTiles * kBlockN;         // columns per buffer
     static constexpr int kBStageBytes = kBlockN * 128;        // token rows x 64 bf16
     static constexpr int kAStageBytes = kTiles * kATileBytes;
@@ -219,21 +222,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         *abort_flag = 1;
         report_error(a.status, MOE_ERR_DEVICE_TIMEOUT, (kDown ? 200 : 100) + where);
     };
-    // unit u: block b = u / NT; output tile j = u % NT; pair units: rows half
-    // (u % NT) / (NT / 2) of the block and output tile pair j.  Every role
-    // skips the same empty units (a second half of a block of <= 128 rows).
+    // unit u: block b = u / NT, output tile j = u % NT.  Streaming variant:
+    // first every block's first half of rows, then every block's second half
+    // (units u and u + nblk * NT / 2 are the two halves of one (block, tile)),
+    // with output tile (gate/up) or tile pair (down) j; so the units that are
+    // empty (a second half of a block of <= 128 rows) come last and the
+    // persistent grid deals the others out evenly.  Every role skips the same
+    // empty units.
+    const int nhu = *a.num_blocks * (NT / 2);  // units per half (streaming variant)
     struct Unit {
         int b, j, row0, rows;
     };
     auto unit_of = [&](int u) {
         Unit x;
-        x.b = u / NT;
-        const int r = u - x.b * NT;
+        int r;
+        int half = 0;
+        if constexpr (kStream) {
+            half = u >= nhu ? 1 : 0;
+            const int v = u - half * nhu;
+            x.b = v / (NT / 2);
+            r = v - x.b * (NT / 2);
+        } else {
+            x.b = u / NT;
+            r = u - x.b * NT;
+        }
         const int row0 = a.block_map[3 * x.b + 1];
         const int rows = a.block_map[3 * x.b + 2];
-        if constexpr (C::kPair) {
-            const int half = r / (NT / 2);
-            x.j = r - half * (NT / 2);
+        if constexpr (kStream) {
+            x.j = r;
             x.row0 = row0 + half * C::kBlockN;
             x.rows = min(C::kBlockN, rows - half * C::kBlockN);
         } else {
@@ -256,7 +272,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             // down: blocks (e, c, kTiles j ..) for chunk c, adjacent (a chunk's
             // output tiles are contiguous); gate/up: half-blocks (e, j, 0, c)
             // and (e, j, 1, c)
-            const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NT + j) * KC * a.block_bytes;
+            const int NTg = kStream ? NT / 2 : NT;  // gate/up feature tiles of an expert
+            const uint8_t* src = a.wpack + (static_cast<size_t>(e) * NTg + j) * KC * a.block_bytes;
             const size_t half_stride = static_cast<size_t>(KC) * (a.block_bytes / 2);
             for (int c = 0; c < KC; ++c, ++it) {
                 const int s = it % C::kNW;

@@ -48,13 +48,14 @@ def kernel_configs():
     na_s, na1, na2 = find(r"static constexpr int kNA = kStream \? %s : \(kOneTile \? %s : %s\);"
                           % (n, n, n), "kNA")
     nb_s, nb = find(r"static constexpr int kNB = kStream \? %s : %s;" % (n, n), "kNB")
-    acc_dn, acc_gu = find(r"static constexpr int kAccBufs = kDown \? %s : %s;" % (n, n), "kAccBufs")
+    acc2, acc1 = find(r"static constexpr int kAccBufs = \(kDown \|\| kStream\) \? %s : %s;" % (n, n),
+                      "kAccBufs")  # two buffers for down and for the streaming variant
     g1, g2 = find(r"static constexpr int kGroups = kOneTile \? %s : %s;" % (n, n), "kGroups")
     assert re.search(r"kTiles = \(kDown && !kPair\) \? kDownTiles : 2;", src), "kTiles"
-    return [("gate/up", nw2, na2, nb, g2, acc_gu),
-            ("down", nw1, na1, nb, g1, acc_dn),
-            ("gate/up, streaming", nw_s2, na_s, nb_s, g2, acc_gu),
-            ("down, streaming (pairs)", nw_s2, na_s, nb_s, g2, acc_dn)]
+    return [("gate/up", nw2, na2, nb, g2, acc1),
+            ("down", nw1, na1, nb, g1, acc2),
+            ("gate/up, streaming (half blocks)", nw_s2, na_s, nb_s, g2, acc2),
+            ("down, streaming (half blocks, tile pairs)", nw_s2, na_s, nb_s, g2, acc2)]
 
 
 class Barrier:
