@@ -399,7 +399,7 @@ route_scan_kernel(const int32_t* __restrict__ hist, int ng, int E, int BT,
 // (gbase) by a scan over warps, and pass 2 places every assignment: inside a
 // 32-assignment chunk the lanes of one expert are ranked by lane id.
 // ---------------------------------------------------------------------------
-constexpr int kScatterWarps = 8;
+constexpr int kScatterWarps = 32;
 
 __global__ void __launch_bounds__(kScatterWarps * 32)
 route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ gbase,
