@@ -151,6 +151,9 @@ struct RouterCfg {
 };
 using RouterCfg16 = RouterCfg<16, 8, 8, 256>;
 using RouterCfg8 = RouterCfg<8, 8, 16, 128>;
+// few tokens: half the experts per slice and 64-token tiles, so twice as many
+// CTAs share the work (each loads a W_r slice half as large)
+using RouterCfg8s = RouterCfg<8, 8, 8, 256>;
 constexpr int kRouterMinTile = 64;  // smallest tile of the configurations above
 
 template <class RC>
@@ -515,6 +518,9 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float*
                                  int32_t* status, cudaStream_t st) {
     // batches of at least one tile per SM use the shared-memory kernel
     if (T >= kRouterMinTile * 2) {
+        if (T <= 1024 && E % 8 == 0 && RouterCfg8s::smem_bytes(d) <= 227 * 1024)
+            return launch_router_smem<RouterCfg8s>(x, W, b, logits, T, d, E, hist, hist_n, status,
+                                                   st);
         if (E % 16 == 0 && RouterCfg16::smem_bytes(d) <= 227 * 1024)
             return launch_router_smem<RouterCfg16>(x, W, b, logits, T, d, E, hist, hist_n, status,
                                                    st);
