@@ -251,7 +251,8 @@ MOE_API moe_status_t moe_forward_host(const moe_plan_t *plan, int32_t T,
  *     (each part rounded up to 256); larger calls return
  *     MOE_ERR_WORKSPACE_TOO_SMALL before launching anything.
  *   The first call on a device looks up the array's device address (with
- *     that device current); make it before any stream capture begins.
+ *     that device current) and sets the router kernels' attributes for every
+ *     batch size; make it before any stream capture begins.
  *   Every call shares the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race and must be serialised by the caller.
  *   Device-side errors are recorded in the array and cannot be read back.

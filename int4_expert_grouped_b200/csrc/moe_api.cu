@@ -48,6 +48,7 @@ moe_status_t device_setup(int* num_sms) {
         if (moe::prepare_gemm_kernels() != cudaSuccess) return MOE_ERR_CUDA;
         if (moe::prepare_decode_kernels() != cudaSuccess) return MOE_ERR_CUDA;
         if (moe::prepare_router_fast() != cudaSuccess) return MOE_ERR_CUDA;
+        if (moe::prepare_router() != cudaSuccess) return MOE_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;

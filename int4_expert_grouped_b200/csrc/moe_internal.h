@@ -107,6 +107,10 @@ size_t router_fast_ws_bytes(int T, int d, int E);
 // [T][E] logits buffer.
 RouterFastWs router_fast_ws(uint8_t* base, float* L, int T, int d, int E);
 cudaError_t prepare_router_fast();
+// Shared-memory attributes of every fp32 router tiling (also run on a call's
+// first use of a tiling; done up front so that no later call makes it inside
+// a stream capture).
+cudaError_t prepare_router();
 // Top-k indices and weights and the per-group histograms (cleared here, as is
 // the status word) for T >= kFastRouterMinT tokens.
 cudaError_t launch_router_fast(const uint16_t* x, const float* W, const float* b, int T, int d, int E,

@@ -14,8 +14,9 @@
 // library holds kNoAllocScratchBytes of it until the process exits, and
 // every call shares it.  Host code cannot use the array's name as a device
 // address, so the first call on each device (with that device current) looks
-// the address up once with cudaGetSymbolAddress and keeps it; make that
-// first call before any stream capture begins.
+// the address up once with cudaGetSymbolAddress and keeps it, and sets the
+// routers' kernel attributes for every tiling; make that first call before
+// any stream capture begins.
 #include <atomic>
 #include <mutex>
 
@@ -46,6 +47,10 @@ moe_status_t scratch_address(void** out) {
         if (c.ready.load(std::memory_order_relaxed) == 0) {
             void* p = nullptr;
             if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
+                return MOE_ERR_CUDA;
+            // the routers' one-time kernel attributes, so that no later call
+            // sets them inside a stream capture
+            if (moe::prepare_router() != cudaSuccess || moe::prepare_router_fast() != cudaSuccess)
                 return MOE_ERR_CUDA;
             c.ptr = p;
             c.ready.store(1, std::memory_order_release);

@@ -513,6 +513,14 @@ static cudaError_t launch_router_smem(const uint16_t* x, const float* W, const f
                       smem, st, x, W, b, logits, T, d, E, hist, hist_n, status);
 }
 
+cudaError_t prepare_router() {
+    int n = 0;
+    cudaError_t e = router_smem_setup<RouterCfg16>(&n);
+    if (e == cudaSuccess) e = router_smem_setup<RouterCfg8>(&n);
+    if (e == cudaSuccess) e = router_smem_setup<RouterCfg8s>(&n);
+    return e;
+}
+
 cudaError_t launch_router_logits(const uint16_t* x, const float* W, const float* b,
                                  float* logits, int T, int d, int E, int32_t* hist, int hist_n,
                                  int32_t* status, cudaStream_t st) {
