@@ -236,6 +236,29 @@ def test_all_tokens_same_experts(moe):
     check_y(y[:300], oracle.forward(inp)["y"], "concentrated")
 
 
+def test_streaming_form_large_blocks(moe):
+    # Fewer than 64 rows per expert on average (T*k = 600 < 64*E) takes the
+    # GEMMs' streaming form, whose units are halves of a block's rows; a bias
+    # that puts expert 0 first for every token gives it 300 rows (a full
+    # 256-row block, both halves in use, and a 44-row block whose second half
+    # is empty), while the other experts get a few rows each.
+    shape = mi.Shape(T=300, d=256, E=64, k=2, f=128, group=32)
+    assert shape.T * shape.k < 64 * shape.E
+    inp = mi.make_inputs(shape, 8)
+    inp.b_r = np.zeros(64, dtype=np.float32)
+    inp.b_r[0] = 50.0
+    layer = moe.MoeLayer.from_inputs(inp)
+    x = moe.bf16_tensor(inp.x, "cuda")
+    bufs = layer.route_buffers(300)
+    y = layer.forward(x, route_out=bufs)
+    torch.cuda.synchronize()
+    assert layer.read_status() == (0, 0)
+    rref = oracle_route(inp)
+    assert rref["counts"][0] == 300
+    check_route(bufs, rref, 300, 2)
+    check_y(y[:300], oracle.forward(inp)["y"], "streaming form, large blocks")
+
+
 def test_every_expert_selected(moe):
     shape = mi.Shape(T=64, d=256, E=8, k=8, f=128, group=64)
     inp = mi.make_inputs(shape, 17)
