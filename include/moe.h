@@ -119,7 +119,8 @@ typedef struct moe_expert_weights {
  * Routing results (device pointers, caller-owned).  With T tokens:
  *   topk_idx      int32 [T, k]   experts per token, best first; ties go to
  *                                the lower expert id
- *   topk_w        fp32  [T, k]   softmax over the k selected logits
+ *   topk_w        fp32  [T, k]   softmax over the k selected logits (evaluated
+ *                                in double, rounded once to fp32)
  *   counts        int32 [E]      assignments per expert
  *   offsets       int32 [E+1]    exclusive prefix sum of counts
  *   sorted_assign int32 [T*k]    assignment a = t*k + j at expert-ordered row

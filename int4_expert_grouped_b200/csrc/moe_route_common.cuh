@@ -25,14 +25,17 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
 // Routing weights of one token by one warp: lane j < k holds the logit of
 // slot j; softmax over the k slots, w_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0),
 // the sum in a fixed xor butterfly order.  Returns lane j's weight (0 for
-// lanes >= k).
+// lanes >= k).  Evaluated in double and rounded once to fp32: l_j - l_0 is
+// then exact, whereas in fp32 its rounding alone moves exp(l_j - l_0) by up to
+// |l_j - l_0| * 2^-24 relative (3e-6 at a spread of 50).  Only k values per
+// token, so the cost does not show.
 __device__ __forceinline__ float warp_slot_weights(float my_v, int k, int lane) {
-    const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
-    const float ex = lane < k ? expf(__fsub_rn(my_v, l0)) : 0.0f;
-    float sum = ex;
+    const double l0 = static_cast<double>(__shfl_sync(0xffffffffu, my_v, 0));
+    const double ex = lane < k ? exp(static_cast<double>(my_v) - l0) : 0.0;
+    double sum = ex;
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, m));
-    return lane < k ? __fdiv_rn(ex, sum) : 0.0f;
+    for (int m = 16; m >= 1; m >>= 1) sum = __dadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, m));
+    return lane < k ? __double2float_rn(__ddiv_rn(ex, sum)) : 0.0f;
 }
 
 // Top-k of one token's E logits by one warp: lane holds experts lane,
