@@ -242,6 +242,18 @@ def layer_launches(layer, T):
     return KERNELS_PER_PATH[layer.plan.forward_path(T)]
 
 
+def max_over_ranks(value, world, device="cuda"):
+    """The largest of every rank's value (the slowest rank sets a replicated
+    step's time); every rank must call it, in the same order."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def time_layer(layer, x, y, K, repeats, cold, stream, world=1):
     """K layer calls with the weights cold in L2 (`cold`), `repeats` times.
 
@@ -268,11 +280,7 @@ def time_layer(layer, x, y, K, repeats, cold, stream, world=1):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        total = float(sum(r[0].elapsed_time(r[1]) for r in evs))
-        if world > 1:
-            t = torch.tensor([total], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            total = float(t.item())
+        total = max_over_ranks(float(sum(r[0].elapsed_time(r[1]) for r in evs)), world)
         reps.append(total / K)
     return reps, sorted(reps)[repeats // 2]
 
@@ -430,11 +438,7 @@ def run_ours(args, name):
         layer.forward_host(xh, yh)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / KE
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / KE, world)
     code, detail = layer.read_status()
     if code != 0:
         raise RuntimeError("device status %d (%d) after timing" % (code, detail))
