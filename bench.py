@@ -509,9 +509,10 @@ def run_ours(args, name):
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum (bytes) of one gate/up GEMM
-# launch from an ncu capture of the current kernel build (profiles/); workloads
+# launch from an ncu capture of the current kernel build (a one-pass metric
+# set on the full workload, profiles/ncu_grouped_gemm_t2048.md); workloads
 # without such a capture report None.
-TRAFFIC_GATEUP: dict = {}
+TRAFFIC_GATEUP: dict = {"prefill_t8192": 495.22e6 + 85.10e6}
 
 
 def main():
