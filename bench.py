@@ -512,7 +512,7 @@ def run_ours(args, name):
 # launch from an ncu capture of the current kernel build (a one-pass metric
 # set on the full workload, profiles/ncu_grouped_gemm_t2048.md); workloads
 # without such a capture report None.
-TRAFFIC_GATEUP: dict = {"prefill_t8192": 495.22e6 + 85.10e6}
+TRAFFIC_GATEUP: dict = {"prefill_t8192": 495.87e6 + 85.25e6}
 
 
 def main():

@@ -282,6 +282,20 @@ union BF2 {
 // i = 0..3, so masking with 0x000F000F and or-ing the bf16 pattern of 128
 // yields the pair (128 + q_2i, 128 + q_2i+1) exactly; subtracting 128 is exact
 // and the fused multiply-add q*s + b rounds once.
+// Nibble pair i of a packed word as bf16x2 (128 + q_lo, 128 + q_hi):
+// ((w >> 4i) & 0x000F000F) | 0x43004300.  For i > 0 the shift and the or run
+// as one integer multiply-add on the FMA pipe, ((w & mask_i) * 2^(32-4i)) >> 32
+// + 0x43004300 (the masked bits and the pattern share no bit), so the
+// half-rate logic pipe takes one operation per pair instead of two.
+__device__ __forceinline__ uint32_t nibble_pair_bf16(uint32_t w, int i) {
+    if (i == 0) return (w & 0x000F000Fu) | 0x43004300u;
+    uint32_t d;
+    asm("mad.hi.u32 %0, %1, %2, %3;"
+        : "=r"(d)
+        : "r"(w & (0x000F000Fu << (4 * i))), "r"(1u << (32 - 4 * i)), "r"(0x43004300u));
+    return d;
+}
+
 __device__ __forceinline__ uint4 expand8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
     BF2 k128;
     k128.u = 0x43004300u;
@@ -289,7 +303,7 @@ __device__ __forceinline__ uint4 expand8(uint32_t w, __nv_bfloat162 s2, __nv_bfl
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         BF2 v, o;
-        v.u = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+        v.u = nibble_pair_bf16(w, i);
         const __nv_bfloat162 q = __hsub2(v.h, k128.h);
         o.h = __hfma2(q, s2, b2);
         r[i] = o.u;

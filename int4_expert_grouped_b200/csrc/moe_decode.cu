@@ -153,9 +153,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 }
 
 // nibble pair i of a packed word as bf16 (128 + q_lo, 128 + q_hi)
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
-    return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
-}
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) { return nibble_pair_bf16(w, i); }
 
 // D += sum (128 + q) x over one 32-wide vector: wa, wb = word c of the vector
 // in rows g and g + 8; xb = the column's operands K 8c .. 8c+7
