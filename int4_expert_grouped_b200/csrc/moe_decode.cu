@@ -167,8 +167,10 @@ __device__ __forceinline__ void vector_mma(float (&D)[4], uint32_t wa, uint32_t 
 // columns 2c, 2c + 1
 __device__ __forceinline__ void group_fold(float (&acc)[4], const float (&D)[4], uint32_t sa,
                                            uint32_t sb, float xs0, float xs1) {
-    const float s0 = __uint_as_float(sa << 16);
-    const float s1 = __uint_as_float(sb << 16);
+    // the scales (low halves) by an integer multiply, which may issue on the
+    // FMA pipe; the logic pipe is the busier one in these calls
+    const float s0 = __uint_as_float(sa * 65536u);
+    const float s1 = __uint_as_float(sb * 65536u);
     const float c0 = fmaf(-128.0f, s0, __uint_as_float(sa & 0xFFFF0000u));
     const float c1 = fmaf(-128.0f, s1, __uint_as_float(sb & 0xFFFF0000u));
     acc[0] = fmaf(s0, D[0], fmaf(c0, xs0, acc[0]));
@@ -745,12 +747,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 }
             }
             compute_sync();
-            // the 32-wide vector sums of the h rows (K order), for the group folds
-            if (tid < 2 * n) {
-                const int col = tid >> 1, v = tid & 1;
-                float sacc = 0.0f;
-                for (int i = 0; i < 32; ++i) sacc += bf16_bits_to_float(hsh[col * kDecHStride + 32 * v + i]);
-                hsum[col * 2 + v] = sacc;
+            // the 32-wide vector sums of the h rows, for the group folds: warp
+            // 2 col + v sums vector v of row col with an xor butterfly (a fixed
+            // order)
+            if (warp < 2 * n) {
+                const int col = warp >> 1, v = warp & 1;
+                float sacc = bf16_bits_to_float(hsh[col * kDecHStride + 32 * v + lane]);
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) sacc = __fadd_rn(sacc, __shfl_xor_sync(0xffffffffu, sacc, m));
+                if (lane == 0) hsum[col * 2 + v] = sacc;
             }
             compute_sync();
             // down: up to four 128-row output tiles per stage, K = the slice
