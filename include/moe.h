@@ -241,6 +241,64 @@ MOE_API moe_status_t moe_forward_host(const moe_plan_t *plan, int32_t T,
                               void *stream);
 
 /*
+ * Expert parallelism: the layer's experts split over ranks (one process per
+ * GPU), rank r holding a contiguous range of them.  The scatter already puts
+ * the rows for one rank's experts next to each other, so each rank runs
+ *   moe_route            routing of its own tokens over all E experts
+ *   moe_dispatch         its token rows in expert order (one segment per rank)
+ *   (the caller sends segment r to rank r, e.g. an NCCL all-to-all)
+ *   moe_experts_forward  the grouped GEMMs over the rows it received, for its
+ *                        own experts (a plan and packed weights of just those)
+ *   (the caller sends the outputs back the same way)
+ *   moe_combine          the routing-weighted sum of its tokens' outputs
+ * The scatter with its block map (inblix, paragraph 3) is the step the
+ * exchange hangs on; the exchange itself is the caller's (NCCL over NVLink
+ * in int4_expert_grouped_b200/ep.py).  The three entries below run one part
+ * of moe_forward each, with the same arithmetic.
+ *
+ * moe_dispatch: xs[p] = x[sorted_assign[p] / k] for p < T*k.
+ *   x bf16 [T, d]; sorted_assign int32 [T*k] (from moe_route, values < T*k,
+ *   else MOE_ERR_DEVICE_BOUNDS detail 300 and row 0 is copied);
+ *   xs bf16 [T*k, d] (written).  ws: workspace_bytes (status word only).
+ */
+MOE_API moe_status_t moe_dispatch(const moe_plan_t *plan, int32_t T, const uint16_t *x,
+                                  const int32_t *sorted_assign, uint16_t *xs, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
+ * moe_experts_forward: o[p] = bf16(W_down^e (bf16(silu(W_gate^e xs[p]) *
+ * (W_up^e xs[p])))) for every row p of every block map entry (e, first row,
+ * rows); the expert ids index this plan's experts (its E, its packed
+ * weights).  Rounding as moe_forward's batched path.
+ *   rows      rows of xs and o, 0 <= rows <= T_max * k;
+ *   xs        bf16 [rows, d] device, the rows in any order;
+ *   block_map int32 [max_blocks, 3] device: entries of at most block_t rows
+ *             (moe_plan_info), each with expert < E, first row >= 0 and first
+ *             row + rows <= rows of xs; num_blocks int32 [1] device, at most
+ *             max_blocks.  A map out of range is not used: the call records
+ *             MOE_ERR_DEVICE_BOUNDS (detail 400) and writes nothing to o.
+ *             Rows outside every entry are left as they were in o.
+ *   o         bf16 [rows, d] device (written).
+ *   ws        workspace_bytes of device memory for this plan.
+ */
+MOE_API moe_status_t moe_experts_forward(const moe_plan_t *plan, int32_t rows,
+                                         const uint16_t *xs, const int32_t *block_map,
+                                         const int32_t *num_blocks, int32_t max_blocks,
+                                         const void *packed_w, uint16_t *o, void *ws,
+                                         size_t ws_bytes, void *stream);
+
+/*
+ * moe_combine: y[t] = bf16(sum_{j<k} topk_w[t,j] * o[pos[t*k+j]]), the sum in
+ * fp32 in slot order.  o bf16 [T*k, d] (row p = the expert output of
+ * expert-ordered row p); pos and topk_w from moe_route (pos values < T*k,
+ * else MOE_ERR_DEVICE_BOUNDS detail 301 and that slot counts as 0);
+ * y bf16 [T, d] (written).  ws: workspace_bytes (status word only).
+ */
+MOE_API moe_status_t moe_combine(const moe_plan_t *plan, int32_t T, const uint16_t *o,
+                                 const int32_t *pos, const float *topk_w, uint16_t *y, void *ws,
+                                 size_t ws_bytes, void *stream);
+
+/*
  * moe_route without a workspace, for callers that cannot allocate device
  * memory (code running under a stream capture that forbids allocation, a
  * runtime that owns every byte of device memory, a plugin host that hands a

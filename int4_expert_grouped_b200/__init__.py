@@ -12,6 +12,9 @@ Entry points (same names as include/moe.h):
     Plan.forward(...)                 moe_forward
     Plan.forward_host(...)            moe_forward_host
     Plan.read_status(ws)              moe_read_status
+    Plan.dispatch(...)                moe_dispatch         (expert parallelism,
+    Plan.experts_forward(...)         moe_experts_forward   see ep.py)
+    Plan.combine(...)                 moe_combine
 """
 from __future__ import annotations
 
@@ -94,17 +97,21 @@ _lib.moe_route_noalloc.argtypes = [_P, ctypes.c_int32, _P, _P, _P, ctypes.POINTE
 _lib.moe_forward_host.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_read_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                  ctypes.c_int32, _P]
+_lib.moe_dispatch.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.moe_experts_forward.argtypes = [_P, ctypes.c_int32, _P, _P, _P, ctypes.c_int32, _P, _P, _P,
+                                     ctypes.c_size_t, _P]
+_lib.moe_combine.argtypes = [_P, ctypes.c_int32, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_forward_path.argtypes = [_P, ctypes.c_int32]
 _lib.moe_forward_path.restype = ctypes.c_int
 for _fn in ("moe_plan_create", "moe_plan_info", "moe_prepack_weights", "moe_route",
             "moe_forward", "moe_forward_timed", "moe_forward_host", "moe_read_status",
-            "moe_route_noalloc"):
+            "moe_route_noalloc", "moe_dispatch", "moe_experts_forward", "moe_combine"):
     getattr(_lib, _fn).restype = ctypes.c_int
 
 EXPORTED = ("moe_abi_version", "moe_status_str", "moe_plan_create", "moe_plan_info",
             "moe_plan_destroy", "moe_prepack_weights", "moe_route", "moe_forward",
             "moe_forward_timed", "moe_forward_host", "moe_read_status", "moe_route_noalloc",
-            "moe_forward_path")
+            "moe_forward_path", "moe_dispatch", "moe_experts_forward", "moe_combine")
 
 
 def abi_version() -> int:
@@ -204,6 +211,24 @@ class Plan:
         _check(_lib.moe_forward_host(self._h, T, ptr(x_host), ptr(w_r), ptr(b_r), ptr(packed_w),
                                      ptr(y_host), ptr(ws), ws.numel() * ws.element_size(),
                                      _stream_ptr(stream)), "moe_forward_host")
+
+    def dispatch(self, T, x, sorted_assign, xs, ws, stream=None):
+        """moe_dispatch: xs[p] = x[sorted_assign[p] / k]."""
+        _check(_lib.moe_dispatch(self._h, T, ptr(x), ptr(sorted_assign), ptr(xs), ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream_ptr(stream)), "moe_dispatch")
+
+    def experts_forward(self, rows, xs, block_map, num_blocks, packed_w, o, ws, stream=None):
+        """moe_experts_forward over `rows` rows of xs; block_map int32 [n, 3] and
+        num_blocks int32 [>= 1] on the device (max_blocks = n)."""
+        _check(_lib.moe_experts_forward(self._h, rows, ptr(xs), ptr(block_map), ptr(num_blocks),
+                                        int(block_map.shape[0]), ptr(packed_w), ptr(o), ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream_ptr(stream)),
+               "moe_experts_forward")
+
+    def combine(self, T, o, pos, topk_w, y, ws, stream=None):
+        """moe_combine: y[t] = bf16(sum_j topk_w[t, j] o[pos[t k + j]])."""
+        _check(_lib.moe_combine(self._h, T, ptr(o), ptr(pos), ptr(topk_w), ptr(y), ptr(ws),
+                                ws.numel() * ws.element_size(), _stream_ptr(stream)), "moe_combine")
 
     def forward_path(self, T: int) -> int:
         """1 if moe_forward runs the small-batch kernels at batch T, 0 for the batched ones."""

@@ -261,6 +261,57 @@ moe_status_t moe_route(const moe_plan_t* plan, int32_t T, const uint16_t* x, con
                      static_cast<cudaStream_t>(stream));
 }
 
+// Steps 6-7: the gate/up GEMM (SwiGLU fused) and the down GEMM over
+// expert-ordered rows xs [rows, d] tiled by block_map (num_blocks entries on
+// the device, at most mb); h [rows, f] is scratch and o [rows, d] receives the
+// expert outputs (o may be xs: gate/up has finished reading xs when the down
+// GEMM starts).  after_gate_up: an event recorded between the two, or NULL.
+static moe_status_t run_experts(const moe_plan* plan, int rows, const uint16_t* xs, const int32_t* block_map,
+                         const int32_t* num_blocks, int mb, const void* packed_w, uint16_t* h, uint16_t* o,
+                         int32_t* status, bool test_timeout, int num_sms, cudaStream_t st,
+                         cudaEvent_t after_gate_up) {
+    const moe_shape_t& s = plan->s;
+    const uint8_t* wp = static_cast<const uint8_t*>(packed_w);
+    moe::GemmArgs g{};
+    g.wpack = wp;
+    g.block_map = block_map;
+    g.num_blocks = num_blocks;
+    g.out = h;
+    g.status = status;
+    // at most 64 rows per expert on average: the GEMMs are bound by reading the
+    // weights, so they keep more packed-weight stages in flight, and each unit
+    // takes one half (<= 128 rows) of a block
+    g.stream = static_cast<long long>(rows) < 64ll * s.E ? 1 : 0;
+    g.K = s.d;
+    g.NT = (s.f / 128) * (g.stream ? 2 : 1);  // units per block: feature tiles (x halves)
+    g.out_ld = s.f;
+    g.group = s.group;
+    g.block_bytes = plan->group_bytes;
+    g.max_units = mb * g.NT;
+    // test hook (MOE_SHAPE_TEST_TIMEOUT): the gate/up GEMM withholds a stage and
+    // its waits give up after 5 ms
+    g.withhold_first = test_timeout ? 1 : 0;
+    g.wait_ns = test_timeout ? 5000000ull : moe::kWaitTimeoutNs;
+    for (int i = 0; i < moe::kBoxSizes; ++i)
+        MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap[i], xs, static_cast<uint64_t>(rows), s.d, moe::kBlockT >> i));
+    MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
+    if (after_gate_up != nullptr) MOE_CUDA(cudaEventRecord(after_gate_up, st));
+
+    g.wpack = wp + align_up(plan->gu_packed, 256);
+    g.out = o;
+    g.K = s.f;
+    g.NT = s.d / (128 * moe::kDownTiles);
+    g.out_ld = s.d;
+    g.block_bytes = plan->down_block_bytes;
+    g.max_units = mb * g.NT;
+    g.withhold_first = 0;
+    g.wait_ns = moe::kWaitTimeoutNs;
+    for (int i = 0; i < moe::kBoxSizes; ++i)
+        MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap[i], h, static_cast<uint64_t>(rows), s.f, moe::kBlockT >> i));
+    MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
+    return MOE_OK;
+}
+
 moe_status_t moe_forward(const moe_plan_t* plan, int32_t T, const uint16_t* x, const float* W_r,
                          const float* b_r, const void* packed_w, uint16_t* y,
                          const moe_route_out_t* route_out, void* ws, size_t ws_bytes,
@@ -347,50 +398,89 @@ moe_status_t moe_forward_timed(const moe_plan_t* plan, int32_t T, const uint16_t
     MOE_CUDA(moe::launch_dispatch(x, r.sa, Tk, s.k, s.d, xs, status, num_sms, st));
     if (ev && !mark(ev->routed)) return MOE_ERR_CUDA;
 
-    const int mb = max_blocks_for(s, T);
-    const uint8_t* wp = static_cast<const uint8_t*>(packed_w);
-    moe::GemmArgs g{};
-    g.wpack = wp;
-    g.block_map = r.bm;
-    g.num_blocks = r.nb;
-    g.out = h;
-    g.status = status;
-    // at most 64 rows per expert on average: the GEMMs are bound by reading the
-    // weights, so they keep more packed-weight stages in flight, and each unit
-    // takes one half (<= 128 rows) of a block
-    g.stream = static_cast<long long>(T) * s.k < 64ll * s.E ? 1 : 0;
-    g.K = s.d;
-    g.NT = (s.f / 128) * (g.stream ? 2 : 1);  // units per block: feature tiles (x halves)
-    g.out_ld = s.f;
-    g.group = s.group;
-    g.block_bytes = plan->group_bytes;
-    g.max_units = mb * g.NT;
-    // test hook (MOE_SHAPE_TEST_TIMEOUT): the gate/up GEMM withholds a stage and
-    // its waits give up after 5 ms
     const bool test_timeout = (s.flags & MOE_SHAPE_TEST_TIMEOUT) != 0;
-    g.withhold_first = test_timeout ? 1 : 0;
-    g.wait_ns = test_timeout ? 5000000ull : moe::kWaitTimeoutNs;
-    for (int i = 0; i < moe::kBoxSizes; ++i)
-        MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap[i], xs, static_cast<uint64_t>(Tk), s.d, moe::kBlockT >> i));
-    MOE_CUDA(moe::launch_gemm_gateup(g, num_sms, st));
-    if (ev && !mark(ev->gate_up)) return MOE_ERR_CUDA;
-
     // the down outputs o reuse the storage of xs, which gate/up has finished reading
-    g.wpack = wp + align_up(plan->gu_packed, 256);
-    g.out = xs;
-    g.K = s.f;
-    g.NT = s.d / (128 * moe::kDownTiles);
-    g.out_ld = s.d;
-    g.block_bytes = plan->down_block_bytes;
-    g.max_units = mb * g.NT;
-    g.withhold_first = 0;
-    g.wait_ns = moe::kWaitTimeoutNs;
-    for (int i = 0; i < moe::kBoxSizes; ++i)
-        MOE_CUDA(moe::encode_bf16_rows_map(&g.bmap[i], h, static_cast<uint64_t>(Tk), s.f, moe::kBlockT >> i));
-    MOE_CUDA(moe::launch_gemm_down(g, num_sms, st));
+    const moe_status_t es = run_experts(plan, Tk, xs, r.bm, r.nb, max_blocks_for(s, T), packed_w, h, xs,
+                                        status, test_timeout, num_sms, st,
+                                        ev ? static_cast<cudaEvent_t>(ev->gate_up) : nullptr);
+    if (es != MOE_OK) return es;
     if (ev && !mark(ev->down)) return MOE_ERR_CUDA;
     MOE_CUDA(moe::launch_combine(xs, r.pos, r.w, T, s.k, s.d, y, status, num_sms, st));
     if (ev && !mark(ev->end)) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status_t moe_dispatch(const moe_plan_t* plan, int32_t T, const uint16_t* x,
+                          const int32_t* sorted_assign, uint16_t* xs, void* ws, size_t ws_bytes,
+                          void* stream) {
+    if (plan == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+    if (T < 0 || T > plan->s.T_max) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || sorted_assign == nullptr || xs == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ws) || (x && !aligned16(x)) || (sorted_assign && !aligned16(sorted_assign)) ||
+        (xs && !aligned16(xs)))
+        return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < plan->ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    int num_sms = 0;
+    const moe_status_t ds = device_setup(&num_sms);
+    if (ds != MOE_OK) return ds;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, plan->o_status);
+    MOE_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), st));
+    if (T == 0) return MOE_OK;
+    MOE_CUDA(moe::launch_dispatch(x, sorted_assign, T * plan->s.k, plan->s.k, plan->s.d, xs, status, num_sms, st));
+    return MOE_OK;
+}
+
+moe_status_t moe_experts_forward(const moe_plan_t* plan, int32_t rows, const uint16_t* xs,
+                                 const int32_t* block_map, const int32_t* num_blocks, int32_t max_blocks,
+                                 const void* packed_w, uint16_t* o, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    if (plan == nullptr || ws == nullptr || packed_w == nullptr) return MOE_ERR_INVALID_ARG;
+    const moe_shape_t& s = plan->s;
+    if (rows < 0 || static_cast<long long>(rows) > static_cast<long long>(s.T_max) * s.k)
+        return MOE_ERR_INVALID_ARG;
+    if (max_blocks < 0 || max_blocks > (1 << 24)) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (xs == nullptr || o == nullptr || block_map == nullptr || num_blocks == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ws) || !aligned16(packed_w) || (xs && !aligned16(xs)) || (o && !aligned16(o)) ||
+        (block_map && !aligned16(block_map)) || (num_blocks && !aligned16(num_blocks)))
+        return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < plan->ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    int num_sms = 0;
+    const moe_status_t ds = device_setup(&num_sms);
+    if (ds != MOE_OK) return ds;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, plan->o_status);
+    if (rows == 0) {
+        MOE_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), st));
+        return MOE_OK;
+    }
+    // the GEMMs read the checked entry count (0 if the map is out of range)
+    int32_t* nb_checked = at<int32_t>(ws, plan->o_nb);
+    MOE_CUDA(moe::launch_block_map_check(block_map, num_blocks, max_blocks, rows, s.E, kBlockT, nb_checked,
+                                         status, st));
+    return run_experts(plan, rows, xs, block_map, nb_checked, max_blocks, packed_w,
+                       at<uint16_t>(ws, plan->o_h), o, status, false, num_sms, st, nullptr);
+}
+
+moe_status_t moe_combine(const moe_plan_t* plan, int32_t T, const uint16_t* o, const int32_t* pos,
+                         const float* topk_w, uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+    if (plan == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+    if (T < 0 || T > plan->s.T_max) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (o == nullptr || pos == nullptr || topk_w == nullptr || y == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ws) || (o && !aligned16(o)) || (pos && !aligned16(pos)) || (topk_w && !aligned16(topk_w)) ||
+        (y && !aligned16(y)))
+        return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < plan->ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    int num_sms = 0;
+    const moe_status_t ds = device_setup(&num_sms);
+    if (ds != MOE_OK) return ds;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, plan->o_status);
+    MOE_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), st));
+    if (T == 0) return MOE_OK;
+    MOE_CUDA(moe::launch_combine(o, pos, topk_w, T, plan->s.k, plan->s.d, y, status, num_sms, st));
     return MOE_OK;
 }
 

@@ -139,7 +139,44 @@ combine_kernel(const uint16_t* __restrict__ o, const int32_t* __restrict__ pos,
     }
 }
 
+__global__ void __launch_bounds__(kThreads)
+block_map_check_kernel(const int32_t* __restrict__ block_map, const int32_t* __restrict__ num_blocks,
+                       int max_blocks, int n_rows, int E, int block_t, int32_t* __restrict__ nb_out,
+                       int32_t* status) {
+    __shared__ int bad;
+    if (threadIdx.x == 0) {
+        bad = 0;
+        status[0] = 0;  // the status word reports the most recent call
+        status[1] = 0;
+    }
+    __syncthreads();
+    const int nb = *num_blocks;
+    if (nb < 0 || nb > max_blocks) {
+        if (threadIdx.x == 0) bad = 1;
+    } else {
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+            const int e = block_map[3 * i];
+            const int r0 = block_map[3 * i + 1];
+            const int n = block_map[3 * i + 2];
+            if (e < 0 || e >= E || r0 < 0 || n < 0 || n > block_t || r0 > n_rows - n) atomicOr(&bad, 1);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        *nb_out = bad ? 0 : nb;
+        if (bad) report_error(status, MOE_ERR_DEVICE_BOUNDS, 400);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_block_map_check(const int32_t* block_map, const int32_t* num_blocks, int max_blocks,
+                                   int n_rows, int E, int block_t, int32_t* nb_out, int32_t* status,
+                                   cudaStream_t st) {
+    block_map_check_kernel<<<1, kThreads, 0, st>>>(block_map, num_blocks, max_blocks, n_rows, E, block_t,
+                                                   nb_out, status);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
                             uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st) {

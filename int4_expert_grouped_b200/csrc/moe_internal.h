@@ -181,6 +181,14 @@ cudaError_t prepare_gemm_kernels();
 // xs[p] = x[sorted_assign[p] / k] for p < T*k
 cudaError_t launch_dispatch(const uint16_t* x, const int32_t* sorted_assign, int Tk, int k, int d,
                             uint16_t* xs, int32_t* status, int num_sms, cudaStream_t st);
+// Check a caller-built block map before the GEMMs read it (moe_experts_forward):
+// at most max_blocks entries, each with expert < E, first row >= 0,
+// 0 <= rows <= block_t and first row + rows <= n_rows.  Clears the status
+// word (the call's first kernel), then writes the entry count to *nb_out, or
+// 0 with MOE_ERR_DEVICE_BOUNDS (detail 400) if any entry is out of range.
+cudaError_t launch_block_map_check(const int32_t* block_map, const int32_t* num_blocks, int max_blocks,
+                                   int n_rows, int E, int block_t, int32_t* nb_out, int32_t* status,
+                                   cudaStream_t st);
 // y[t] = bf16(sum_i topk_w[t*k+i] * o[pos[t*k+i]])
 cudaError_t launch_combine(const uint16_t* o, const int32_t* pos, const float* topk_w, int T,
                            int k, int d, uint16_t* y, int32_t* status, int num_sms,

@@ -23,7 +23,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe):
     names = declared_functions()
-    assert len(names) == 13
+    assert len(names) == 16
     for n in names:
         assert hasattr(moe.lib(), n), n
     assert set(names) == set(moe.EXPORTED)
@@ -125,6 +125,37 @@ def test_prepack_and_host_checks(moe):
     H = p.info.host_workspace_bytes
     assert lib.moe_forward_host(p.handle, 64, 0x1000, 0x2000, None, 0x3000, 0x4000, 0x5000, H - 1, None) == 4
     assert lib.moe_forward_host(p.handle, 64, None, 0x2000, None, 0x3000, 0x4000, 0x5000, H, None) == 1
+
+
+def test_expert_parallel_entry_checks(moe):
+    """moe_dispatch, moe_experts_forward and moe_combine reject bad arguments
+    before launching anything."""
+    p = moe.Plan(64, 256, 8, 2, 128, 32)
+    W = p.info.workspace_bytes
+    lib = moe.lib()
+    # moe_dispatch(plan, T, x, sorted_assign, xs, ws, ws_bytes, stream)
+    assert lib.moe_dispatch(None, 64, 0x1000, 0x2000, 0x3000, 0x5000, W, None) == 1
+    assert lib.moe_dispatch(p.handle, 65, 0x1000, 0x2000, 0x3000, 0x5000, W, None) == 1
+    assert lib.moe_dispatch(p.handle, 64, None, 0x2000, 0x3000, 0x5000, W, None) == 1
+    assert lib.moe_dispatch(p.handle, 64, 0x1000, 0x2004, 0x3000, 0x5000, W, None) == 3
+    assert lib.moe_dispatch(p.handle, 64, 0x1000, 0x2000, 0x3000, 0x5000, W - 1, None) == 4
+    # moe_experts_forward(plan, rows, xs, block_map, num_blocks, max_blocks,
+    #                     packed_w, o, ws, ws_bytes, stream); rows <= T_max * k
+    ef = lib.moe_experts_forward
+    assert ef(p.handle, 129, 0x1000, 0x2000, 0x3000, 4, 0x4000, 0x6000, 0x5000, W, None) == 1
+    assert ef(p.handle, -1, 0x1000, 0x2000, 0x3000, 4, 0x4000, 0x6000, 0x5000, W, None) == 1
+    assert ef(p.handle, 128, 0x1000, 0x2000, 0x3000, -1, 0x4000, 0x6000, 0x5000, W, None) == 1
+    assert ef(p.handle, 128, 0x1000, None, 0x3000, 4, 0x4000, 0x6000, 0x5000, W, None) == 1
+    assert ef(p.handle, 128, 0x1000, 0x2000, None, 4, 0x4000, 0x6000, 0x5000, W, None) == 1
+    assert ef(p.handle, 128, 0x1000, 0x2000, 0x3000, 4, None, 0x6000, 0x5000, W, None) == 1
+    assert ef(p.handle, 128, 0x1000, 0x2000, 0x3008, 4, 0x4000, 0x6000, 0x5000, W, None) == 3
+    assert ef(p.handle, 128, 0x1000, 0x2000, 0x3000, 4, 0x4000, 0x6002, 0x5000, W, None) == 3
+    assert ef(p.handle, 128, 0x1000, 0x2000, 0x3000, 4, 0x4000, 0x6000, 0x5000, W - 1, None) == 4
+    # moe_combine(plan, T, o, pos, topk_w, y, ws, ws_bytes, stream)
+    assert lib.moe_combine(p.handle, 64, 0x1000, None, 0x3000, 0x4000, 0x5000, W, None) == 1
+    assert lib.moe_combine(p.handle, 64, 0x1000, 0x2000, 0x3000, 0x4004, 0x5000, W, None) == 3
+    assert lib.moe_combine(p.handle, 64, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, W - 1, None) == 4
+    assert lib.moe_combine(p.handle, -1, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, W, None) == 1
 
 
 def test_forward_path_choice(moe):
