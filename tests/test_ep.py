@@ -141,3 +141,54 @@ def test_expert_parallel_forward_one_rank(ep):
     layer = ep.ExpertParallelMoE(OracleBackend(inp, 0, 16), 16)
     y = layer.forward(torch.from_numpy(inp.x.astype(np.int32))).numpy()
     np.testing.assert_allclose(y, oracle.forward(inp)["y"], rtol=1e-12, atol=1e-15)
+
+
+def _rank_leaves(rank, world, port, mode, out):
+    """Rank 1 leaves before the exchange (exits, or stalls without joining it);
+    rank 0's forward must end in an error from the process group (the closed
+    connection, or its 5 s timeout), not wait for ever."""
+    import datetime
+    import time
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, HERE)
+    from ep_stand_in import OracleBackend
+
+    from int4_expert_grouped_b200 import ep
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[rank] = "left"
+        if mode == "stall":
+            time.sleep(10)  # alive, but never joins the exchange
+        os._exit(0)  # gone without a word: no barrier, no destroy
+    inp = _inputs(32, 16, 4)
+    x = torch.from_numpy(inp.x[:16].astype(np.int32))
+    layer = ep.ExpertParallelMoE(OracleBackend(inp, 0, 8), 16, world, rank, group=dist.group.WORLD)
+    t0 = time.time()
+    try:
+        layer.forward(x)
+        out[rank] = "no error"
+    except RuntimeError as e:
+        out[rank] = "error after %.1f s: %s" % (time.time() - t0, str(e).splitlines()[0][:80])
+    os._exit(0)
+
+
+@pytest.mark.parametrize("mode", ["exit", "stall"])
+def test_expert_parallel_rank_that_leaves_ends_in_error(ep, mode):
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_leaves, args=(r, 2, port, mode, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert out[1] == "left"
+    assert out[0].startswith("error after"), out[0]
+    assert float(out[0].split()[2]) < 15.0, out[0]
