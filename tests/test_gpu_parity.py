@@ -4,10 +4,8 @@ Integer outputs (top-k indices, counts, offsets, scatter order, inverse
 positions, block map) must match bit for bit; routing weights within 1e-6
 relative; the layer output within |y - ref| <= 2e-2 * (1 + |ref|) with the
 relative RMS error also reported and bounded.  Small workloads are checked in
-full; the 8K-token prefill layer has every token's output checked, and the
-32K-token Zipf layer the outputs of the first and last token of every
-block-map entry and of every token of its most and least loaded experts (the
-oracle computes those one token at a time).
+full; the 8K-token and the 32K-token Zipf prefill layers have every token's
+output checked (the oracle computes them one token at a time).
 """
 import numpy as np
 import pytest
@@ -125,10 +123,10 @@ def block_entry_tokens(rref, k):
     return np.unique(np.concatenate([first, last]))
 
 
-def test_layer_t32768_zipf_every_block(moe):
-    # the Zipf-skewed 32768-token layer: routing in full; the output of at
-    # least one token of every block-map entry (its first and last rows), and
-    # of every token of the most and of the least loaded non-empty expert
+def test_layer_t32768_zipf_every_token(moe):
+    # the Zipf-skewed 32768-token layer: routing in full and the output of
+    # every token (the first and last rows of every block-map entry, and every
+    # row of the most and of the least loaded non-empty expert, among them)
     inp = workload("prefill_t32768_zipf")
     s = inp.shape
     layer = moe.MoeLayer.from_inputs(inp)
@@ -144,13 +142,15 @@ def test_layer_t32768_zipf_every_block(moe):
     hot = int(nonempty[np.argmax(counts[nonempty])])
     cold = int(nonempty[np.argmin(counts[nonempty])])
     expert_tokens = lambda e: sa[offsets[e]:offsets[e + 1]] // s.k
-    toks = np.unique(np.concatenate([block_entry_tokens(rref, s.k), expert_tokens(hot),
-                                     expert_tokens(cold)]))
-    print("checking %d of %d tokens (%d block-map entries; expert %d has %d rows, expert %d has %d)"
-          % (len(toks), s.T, rref["num_blocks"], hot, counts[hot], cold, counts[cold]))
+    toks = np.arange(s.T)
+    covered = np.unique(np.concatenate([block_entry_tokens(rref, s.k), expert_tokens(hot),
+                                        expert_tokens(cold)]))
+    assert covered.size > 0 and covered.max() < s.T
+    print("checking all %d tokens (%d block-map entries; expert %d has %d rows, expert %d has %d)"
+          % (s.T, rref["num_blocks"], hot, counts[hot], cold, counts[cold]))
     yref, idx, _ = oracle.token_outputs(inp, toks)
-    assert np.array_equal(idx, rref["topk_idx"][toks])
-    check_y(y[torch.from_numpy(toks).cuda()], yref, "prefill_t32768_zipf, every block")
+    assert np.array_equal(idx, rref["topk_idx"])
+    check_y(y[:s.T], yref, "prefill_t32768_zipf, every token")
 
 
 def test_route_entry_point_matches_forward(moe):
