@@ -20,8 +20,10 @@ forward on a rank's own tokens is:
 The received rows are laid out by source rank, and inside each source by local
 expert; the block map tiles each (expert, source) segment, experts first, so
 one expert's tiles run next to each other and share its weights in L2.  The
-results equal moe_forward's: every row meets the same GEMM arithmetic, only
-the tiling of rows differs.
+results equal those of moe_forward's batched kernels bit for bit: every row
+meets the same GEMM arithmetic, only the tiling of rows differs.  (For batches
+of at most 8 tokens moe_forward runs its small-batch kernel instead, which
+rounds differently.)
 
 The exchanges are torch.distributed all-to-alls (NCCL between GPUs).  The
 compute runs in a backend: ``LibraryBackend`` (the CUDA library) is the only
